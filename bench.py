@@ -1,0 +1,418 @@
+"""Benchmark: fine-grained top-K sparse attention on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole path -- indexer -> top-K -> sparse attention
+(for the two-stage workload: pool, coarse scores, coarse top-k, expand, fine
+scores, top-K, attention) -- over one synthetic batch.  The default workload is
+the 8K-token causal prefill (16 query heads, d=128, indexer 4 x 64, top-K 1024,
+window 128).  Each rank runs its own independent sequence (weak scaling, no
+collective on the data path).  One JSON line is printed by rank 0.
+
+Timing: per-step CUDA events on the launching stream, after W warm-up steps,
+with a 512 MB write between steps to flush the 126 MB L2 (outside the event
+brackets); the max over ranks is reported.  Per-stage events inside the step
+give each kernel's share and its roofline fraction.  `e2e` repeats the step
+through the same C-ABI calls with the inputs copied from pinned host memory and
+the output copied back inside the timed region.  `cpu_baseline` times the CPU
+fp64 oracle on a bounded sample of query rows of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "query tokens/s (indexer+top-K+sparse attn); % of HBM / tensor roofline"
+UNIT = "query tokens/s"
+FLUSH_BYTES = 512 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, src="fallback")
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def __exit__(self, *exc):
+        time.sleep(0.25)
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, reasons = [], 0.0, set()
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = max(mx, float(f[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- workloads
+def make_case(name, seed, device):
+    """Device-resident inputs, pinned host copies and a plan for one workload."""
+    import torch
+
+    from fine_grained_top_b200.pipeline import DecodePlan, PrefillPlan
+    from workloads import CONFIGS, gen_decode, gen_prefill
+
+    cfg = dict(CONFIGS[name])
+    inp = gen_prefill(seed=seed, **cfg) if cfg["kind"] != "decode" else gen_decode(seed=seed, **cfg)
+
+    def host(x):
+        if x.dtype == np.uint16:
+            t = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16)
+        else:
+            t = torch.from_numpy(np.ascontiguousarray(x))
+        return t.pin_memory()
+
+    hosts = {k: host(v) for k, v in inp.items() if isinstance(v, np.ndarray)}
+    devs = {k: v.to(device) for k, v in hosts.items()}
+    if cfg["kind"] == "decode":
+        B = cfg["B"]
+        if cfg.get("paged", False):
+            plan = DecodePlan(B, cfg["Hq"], cfg["d"], cfg["H_I"], cfg["D_I"], cfg["K"], cfg["W"], S_max=0,
+                              paged=True, max_pages=inp["page_table"].shape[1], pool_pages=inp["k"].shape[0],
+                              device=device)
+        else:
+            plan = DecodePlan(B, cfg["Hq"], cfg["d"], cfg["H_I"], cfg["D_I"], cfg["K"], cfg["W"],
+                              S_max=inp["k"].shape[1], device=device)
+        # per step a decode call receives the new tokens; the KV cache is resident state
+        step_inputs = ["q", "qI", "w", "lengths"]
+        units = B
+    else:
+        plan = PrefillPlan(cfg["N"], cfg["Hq"], cfg["d"], cfg["H_I"], cfg["D_I"], cfg["K"], cfg["W"],
+                           block=cfg.get("block"), keep=cfg.get("keep"), device=device)
+        step_inputs = ["q", "k", "v", "qI", "w", "kI"]
+        units = cfg["N"]
+    return dict(cfg=cfg, inp=inp, hosts=hosts, devs=devs, plan=plan, stages=plan.stages(devs), units=units,
+                step_inputs=step_inputs)
+
+
+def stage_work(case):
+    """Algorithmic work per kernel for one step: the bytes the method must move
+    through HBM (unique data, each once) and the flops it must run."""
+    cfg, plan, inp = case["cfg"], case["plan"], case["inp"]
+    K, W, Hq, d, H, D = cfg["K"], cfg["W"], cfg["Hq"], cfg["d"], cfg["H_I"], cfg["D_I"]
+    topk = plan.topk.cpu().numpy().astype(np.int64)
+    if cfg["kind"] == "decode":
+        lengths = inp["lengths"].astype(np.int64)
+        pos, rows, pairs = lengths - 1, len(lengths), int(lengths.sum())
+    else:
+        N = cfg["N"]
+        pos, rows, pairs = np.arange(N, dtype=np.int64), N, N * (N + 1) // 2
+    n_sel = ((topk >= 0) & (topk <= (pos - W)[:, None])).sum(1) + np.minimum(W, pos + 1)
+    sum_sel = int(n_sel.sum())
+    qI_b, w_b, idx_b = rows * H * D * 2, rows * H * 2, 4 * rows * K
+    q_b = rows * Hq * d * 2
+    work = {"sum_selected": sum_sel, "causal_pairs": pairs}
+    st = {}
+    if cfg["kind"] == "decode":
+        st["indexer"] = dict(bytes=qI_b + w_b + pairs * D * 2 + 4 * pairs, flops=2.0 * pairs * H * D, bound="hbm")
+        st["topk"] = dict(bytes=4 * pairs + idx_b, flops=0.0, bound="hbm")
+        st["attention"] = dict(bytes=2 * q_b + sum_sel * d * 2 * 2 + idx_b, flops=4.0 * Hq * d * sum_sel,
+                               bound="hbm")
+    else:
+        N = cfg["N"]
+        kv_b = 2 * N * d * 2
+        st["attention"] = dict(bytes=2 * q_b + kv_b + idx_b, flops=4.0 * Hq * d * sum_sel, bound="tensor")
+        if cfg["kind"] == "prefill":
+            st["indexer"] = dict(bytes=qI_b + w_b + N * D * 2 + 4 * pairs, flops=2.0 * pairs * H * D,
+                                 bound="hbm")
+            st["topk"] = dict(bytes=4 * pairs + idx_b, flops=0.0, bound="hbm")
+        else:
+            blk, keep = cfg["block"], cfg["keep"]
+            nb = N // blk
+            cpairs = int(sum(t // blk for t in range(N)))
+            fpairs = int(plan.n_cand.cpu().numpy().astype(np.int64).sum())
+            work.update(coarse_pairs=cpairs, fine_pairs=fpairs)
+            st["pool"] = dict(bytes=N * D * 2 + nb * D * 2, flops=float(N * D), bound="hbm")
+            st["block_counts"] = dict(bytes=4 * N, flops=0.0, bound="hbm")
+            st["coarse_indexer"] = dict(bytes=qI_b + w_b + nb * D * 2 + 4 * N + 4 * cpairs,
+                                        flops=2.0 * cpairs * H * D, bound="hbm")
+            st["coarse_topk"] = dict(bytes=4 * cpairs + 4 * N + 4 * N * keep, flops=0.0, bound="hbm")
+            st["expand"] = dict(bytes=4 * N * keep + 4 * fpairs + 4 * N, flops=0.0, bound="hbm")
+            st["fine_indexer"] = dict(bytes=qI_b + w_b + N * D * 2 + 4 * N + 8 * fpairs,
+                                      flops=2.0 * fpairs * H * D, bound="hbm")
+            st["fine_topk"] = dict(bytes=8 * fpairs + 4 * N + idx_b, flops=0.0, bound="hbm")
+    work["stages"] = st
+    return work
+
+
+def roofline_entry(kind, bytes_, flops, seconds, peaks):
+    if kind == "tensor":
+        ach = flops / seconds / 1e12
+        return {"bound": "tensor", "achieved": round(ach, 2), "peak": peaks["bf16"], "unit": "TFLOP/s",
+                "frac": round(ach / peaks["bf16"], 4)}
+    ach = bytes_ / seconds / 1e9
+    return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm"], "unit": "GB/s",
+            "frac": round(ach / peaks["hbm"], 4)}
+
+
+# --------------------------------------------------------------------------- CPU oracle
+def oracle_sample(case, n):
+    """Run the CPU fp64 oracle (all stages) on n sample units of the workload:
+    n evenly spaced query rows (prefill) or the first n sequences (decode).
+    Returns (seconds, description)."""
+    import oracle
+    cfg, inp = case["cfg"], case["inp"]
+    t0 = time.perf_counter()
+    if cfg["kind"] == "decode":
+        oracle.decode(inp, cfg["K"], cfg["W"], seqs=range(n))
+        desc = "%d of %d sequences, all stages" % (n, cfg["B"])
+    else:
+        rows = np.linspace(0, cfg["N"] - 1, n).astype(np.int64)
+        oracle.prefill(inp, cfg["K"], cfg["W"], rows=rows, block=cfg.get("block"), keep=cfg.get("keep"))
+        desc = "%d evenly spaced query rows of %d, all stages" % (n, cfg["N"])
+    return time.perf_counter() - t0, desc
+
+
+def oracle_calibrate(case, budget_s):
+    """Smallest power-of-4 sample (from 16 rows / 1 sequence) that takes about budget_s / 4 or more."""
+    cfg = case["cfg"]
+    total = cfg["B"] if cfg["kind"] == "decode" else cfg["N"]
+    n = 1 if cfg["kind"] == "decode" else 16
+    while True:
+        el, _ = oracle_sample(case, n)
+        if el >= budget_s / 4 or n >= total:
+            return n, el
+        n = min(total, n * 4)
+
+
+def oracle_rate(case, budget_s=8.0):
+    import oracle
+    n, _ = oracle_calibrate(case, budget_s)
+    el, desc = oracle_sample(case, n)
+    return n / el, desc, oracle.threads()
+
+
+# --------------------------------------------------------------------------- arms
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    device = "cuda:%d" % local_rank
+    torch.cuda.set_device(local_rank)
+    peaks = load_peaks()
+    case = make_case(args.workload, seed=rank, device=device)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
+    plan, d = case["plan"], case["devs"]
+    stage_list = case["stages"]
+
+    def step():
+        for _, fn in stage_list:
+            fn()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if int(plan.dev_status.item()) != 0:
+        raise RuntimeError("device status %d during warm-up" % int(plan.dev_status.item()))
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local_rank])
+        torch.cuda.synchronize()
+
+    # ---- device-resident timed steps, one event between consecutive kernels
+    ns = len(stage_list)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(ns + 1)] for _ in range(args.steps)]
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    gpu_idx = vis.split(",")[local_rank] if vis else str(local_rank)
+    barrier()
+    with ClockSampler(gpu_idx) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            for j, (_, fn) in enumerate(stage_list):
+                fn()
+                ev[i][j + 1].record(stream)
+        barrier()
+    step_ms = [ev[i][0].elapsed_time(ev[i][-1]) for i in range(args.steps)]
+    stage_ms = [[ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps)] for j in range(ns)]
+    total_ms = float(sum(step_ms))
+    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = case["units"] * world * args.steps / (total_ms / 1e3)
+
+    # ---- end to end through the C ABI with host buffers
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    out_host = torch.empty(plan.out.shape, dtype=plan.out.dtype, pin_memory=True)
+    h2d = sum(case["hosts"][k].numel() * case["hosts"][k].element_size() for k in case["step_inputs"])
+    d2h = out_host.numel() * out_host.element_size()
+    barrier()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        e2e_ev[i][0].record(stream)
+        for k in case["step_inputs"]:
+            d[k].copy_(case["hosts"][k], non_blocking=True)
+        step()
+        out_host.copy_(plan.out, non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    barrier()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
+    t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_value = case["units"] * world * args.steps / (float(t.item()) / 1e3)
+    if int(plan.dev_status.item()) != 0:
+        raise RuntimeError("device status %d" % int(plan.dev_status.item()))
+
+    if rank != 0:
+        return None
+    work = stage_work(case)
+    stages = {}
+    for (name, _), times in zip(stage_list, stage_ms):
+        sec = float(np.mean(times)) / 1e3
+        w = work["stages"][name]
+        stages[name] = dict(ms=round(sec * 1e3, 4),
+                            share=round(float(np.sum(times)) / max(1e-9, float(np.sum(step_ms))), 4),
+                            **roofline_entry(w["bound"], w["bytes"], w["flops"], sec, peaks))
+    dom = max(stages, key=lambda n: stages[n]["ms"])
+    roof = {k: v for k, v in stages[dom].items() if k not in ("ms", "share")}
+    w = work["stages"][dom]
+    roof["kernel"] = dom
+    roof["algorithmic"] = w["flops"] if roof["bound"] == "tensor" else w["bytes"]
+    roof["traffic"] = None
+    roof["peak_src"] = peaks["src"] + " (burst figure; kernel timed alone per step)"
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, **{k: v for k, v in case["cfg"].items() if k != "kind"},
+                   "parallelism": "replicas (an independent sequence per GPU)" if world > 1 else "single GPU",
+                   "l2": "flushed between steps (512 MB write outside the timed brackets)"},
+        "roofline": roof, "stages": stages,
+        "work": {k: v for k, v in work.items() if k != "stages"},
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": plan.launches() * args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        rate, sample, cores = oracle_rate(case)
+        line["cpu_baseline"] = {"value": round(rate, 2), "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": sample}
+    return line
+
+
+def run_reference(args, rank, world):
+    """The CPU fp64 oracle as the reference arm: same workload, metric and
+    unit; each step runs the oracle on a fixed bounded sample of query rows."""
+    if rank != 0:
+        return None
+    import oracle
+    from workloads import CONFIGS, config_inputs
+    cfg = CONFIGS[args.workload]
+    case = {"cfg": cfg, "inp": config_inputs(args.workload, seed=0)}
+    n, _ = oracle_calibrate(case, budget_s=4.0)          # also the first warm-up step
+    for _ in range(max(0, args.warmup - 1)):
+        oracle_sample(case, n)
+    times, desc = [], ""
+    for _ in range(args.steps):
+        el, desc = oracle_sample(case, n)
+        times.append(el)
+    total = float(sum(times))
+    value = n * args.steps / total
+    return {"metric": METRIC, "value": round(value, 3), "unit": UNIT, "impl": "reference", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total * 1e3 / args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": args.workload, **{k: v for k, v in cfg.items() if k != "kind"}},
+            "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="prefill_8k")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        import torch
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,416 @@
+// indexer.cu -- stage 1: lightweight-indexer scores on the 5th-generation
+// tensor cores.
+//
+//   I[t,s] = sum_j w[t,j] * ReLU(qI[t,j] . kI[s])
+//
+// ("Sparse Attention for Long-Context LLM Inference", section "Where Sparse
+// Attention Is Actually Sparse": a lightweight indexer scores history
+// positions and outputs candidate indices, without positional encoding;
+// "Sparse Attention in 2026", "The designs that shipped": the lightning
+// indexer is a small few-head low-precision scorer.)
+//
+// Tile mapping: keys on M, (query, head) pairs on N.  qI is stored
+// [rows, H_I, D_I], so QT consecutive queries x H_I heads are QT*H_I
+// consecutive rows of D_I bf16: one K-major B operand.  One tile:
+//     D[s, (t,j)] = kI[s] . qI[t,j]        M = 128 keys, N = 256 (or 16),
+// accumulated in fp32 in TMEM.  The epilogue thread owning TMEM lane s reads
+// the H_I adjacent columns of query t, applies ReLU and the weights w[t,:],
+// and writes scores[t, s]; a warp writes 32 consecutive floats per query.
+//
+// Warp roles (persistent CTAs, one per SM):
+//   warp 0     TMA producer (one elected lane) + TMEM allocator
+//   warp 1     MMA issuer (one elected lane): tcgen05.mma kind::f16
+//   warps 2..  epilogue, two TMEM accumulators in flight (double buffer)
+// Shared-memory ring of STAGES {A = 128 keys, B = N query-head rows} tiles,
+// filled by TMA with the 128B (D_I = 64) or 64B (D_I = 32) swizzle that the
+// UMMA K-major descriptors expect.
+#include <cudaTypedefs.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace sa {
+
+struct IdxKernelArgs {
+    const uint16_t *w;
+    const int32_t *page_table;
+    const int32_t *n_valid;
+    float *scores;
+    int64_t ld;
+    int *dev_status;
+    int max_pages, pool_pages;
+    int B, T, S;
+    int QT, QTN, KT;   // queries per tile, query tiles per batch, key tiles per batch
+    int n_items;
+};
+
+template <int N, int D_I>
+struct IdxCfg {
+    static constexpr int kBoxRows = 64;                       // A is loaded as 2 boxes of 64 keys
+    static constexpr int kABytes = 128 * D_I * 2;
+    static constexpr int kBBytes = N * D_I * 2;
+    static constexpr int kStageBytes = kABytes + kBBytes;
+    static constexpr int kStages = (N == 256) ? 4 : 8;
+    static constexpr int kEpiWarps = (N == 256) ? 8 : 4;
+    static constexpr int kThreads = (2 + kEpiWarps) * 32;
+    static constexpr uint32_t kTmemCols = (2 * N < 32) ? 32 : 2 * N;
+    static constexpr uint32_t kSwizzleBytes = D_I * 2;         // 128 or 64
+    static constexpr uint32_t kSbo = 8 * kSwizzleBytes;        // 8-row core group stride
+    static constexpr uint32_t kLayout = (D_I == 64) ? 2 : 4;   // UMMA layout: 128B / 64B swizzle
+    static constexpr int kEpiGroups = kEpiWarps / 4;
+    static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + 1024;
+};
+
+// Largest n_valid among the tile's queries (the tile's key extent).  Called
+// by a full warp; every role evaluates it identically to skip empty tiles.
+__device__ __forceinline__ int tile_extent(const IdxKernelArgs &a, int b, int qt, int lane) {
+    const int t0 = qt * a.QT, t1 = min(t0 + a.QT, a.T);
+    if (a.n_valid == nullptr) return a.S - a.T + t1;   // causal: last query's count
+    int m = 0;
+    for (int t = t0 + lane; t < t1; t += 32) m = max(m, a.n_valid[(int64_t)b * a.T + t]);
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    return min(m, a.S);
+}
+
+__device__ __forceinline__ void decode_item(const IdxKernelArgs &a, int item, int &b, int &qt, int &kt) {
+    const int per_b = a.QTN * a.KT;
+    b = item / per_b;
+    const int rem = item - b * per_b;
+    qt = rem / a.KT;
+    kt = rem - qt * a.KT;
+}
+
+template <int N, int D_I, int H_I>
+__global__ void __launch_bounds__(IdxCfg<N, D_I>::kThreads, 1)
+    indexer_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
+                      IdxKernelArgs a) {
+    using C = IdxCfg<N, D_I>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *stage_base = smem;
+    uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + C::kStages * C::kStageBytes);
+    uint64_t *empty_bar = full_bar + C::kStages;
+    uint64_t *tfull_bar = empty_bar + C::kStages;   // [2]
+    uint64_t *tempty_bar = tfull_bar + 2;           // [2]
+    uint64_t *drain_bar = tempty_bar + 2;           // [1]
+    uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(drain_bar + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&tfull_bar[i], 1); mbar_init(&tempty_bar[i], C::kEpiWarps); }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&map_k);
+        tma_prefetch_desc(&map_q);
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_base_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_base_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        int stage = 0;
+        uint32_t phase = 0;
+        int issued = 0;
+        for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
+            int b, qt, kt;
+            decode_item(a, item, b, qt, kt);
+            const int ext = tile_extent(a, b, qt, lane);
+            if (kt * 128 >= ext) continue;
+            bool ok = true;
+            if (lane == 0) {
+                ok = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag);
+                if (ok) {
+                    uint8_t *sa_ = stage_base + stage * C::kStageBytes;
+                    uint8_t *sb_ = sa_ + C::kABytes;
+                    int boxes[2] = {0, 0};
+                    int nbox = 0;
+                    for (int i = 0; i < 2; ++i) {
+                        const int s0 = kt * 128 + i * C::kBoxRows;
+                        if (s0 >= ext) break;
+                        if (a.page_table) {
+                            const int pid = a.page_table[(int64_t)b * a.max_pages + (s0 >> 6)];
+                            if (pid < 0 || pid >= a.pool_pages) { report(a.dev_status, SA_DEV_INDEX); continue; }
+                            boxes[i] = pid * 64;
+                        } else {
+                            boxes[i] = b * a.S + s0;
+                        }
+                        nbox |= 1 << i;
+                    }
+                    const uint32_t bytes = C::kBBytes + (uint32_t)__popc(nbox) * (C::kABytes / 2);
+                    mbar_arrive_expect_tx(&full_bar[stage], bytes);
+                    tma_load_2d(sb_, &map_q, 0, (b * a.T + qt * a.QT) * H_I, &full_bar[stage]);
+                    for (int i = 0; i < 2; ++i)
+                        if (nbox & (1 << i))
+                            tma_load_2d(sa_ + i * (C::kABytes / 2), &map_k, 0, boxes[i], &full_bar[stage]);
+                    ++issued;
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            __syncwarp();
+            if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+        }
+        // drain: wait (bounded) for this CTA's last loads to land before teardown
+        if (lane == 0 && *abort_flag) {
+            int s = stage;
+            uint32_t p = phase;
+            for (int i = 0; i < min(issued, C::kStages); ++i) {
+                if (--s < 0) { s = C::kStages - 1; p ^= 1u; }
+                volatile int no_abort = 0;
+                mbar_wait(&full_bar[s], p, &no_abort);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        constexpr uint32_t idesc = idesc_bf16_f32(128, N);
+        int stage = 0;
+        uint32_t phase = 0;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        bool any = false;
+        for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
+            int b, qt, kt;
+            decode_item(a, item, b, qt, kt);
+            const int ext = tile_extent(a, b, qt, lane);
+            if (kt * 128 >= ext) continue;
+            bool ok = true;
+            if (lane == 0) {
+                ok = mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag) &&
+                     mbar_wait(&full_bar[stage], phase, abort_flag);
+                if (ok) {
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(stage_base + stage * C::kStageBytes);
+                    const uint32_t b_addr = a_addr + C::kABytes;
+                    const uint32_t d_tmem = tmem_base + (uint32_t)(acc * N);
+#pragma unroll
+                    for (int k = 0; k < D_I / 16; ++k) {
+                        const uint64_t da = smem_desc(a_addr + k * 32, C::kSbo, C::kLayout);
+                        const uint64_t db = smem_desc(b_addr + k * 32, C::kSbo, C::kLayout);
+                        tc_mma_f16(d_tmem, da, db, idesc, k > 0 ? 1u : 0u);
+                    }
+                    tc_commit(&empty_bar[stage]);
+                    tc_commit(&tfull_bar[acc]);
+                    any = true;
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+            if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        }
+        if (lane == 0 && any) {   // all issued MMAs complete before TMEM is released
+            tc_commit(drain_bar);
+            volatile int no_abort = 0;
+            mbar_wait(drain_bar, 0, &no_abort);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int ew = warp - 2;
+        const int quad = warp & 3;             // TMEM lane quadrant this warp may access
+        const int grp = ew >> 2;               // which part of the tile's queries
+        const int q_per_grp = a.QT / C::kEpiGroups > 0 ? a.QT / C::kEpiGroups : 1;
+        const int q_lo = grp * q_per_grp, q_hi = min(a.QT, q_lo + q_per_grp);
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
+            int b, qt, kt;
+            decode_item(a, item, b, qt, kt);
+            const int ext = tile_extent(a, b, qt, lane);
+            if (kt * 128 >= ext) continue;
+            const bool ok = mbar_wait(&tfull_bar[acc], acc_phase, abort_flag);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const int s = kt * 128 + quad * 32 + lane;
+            const uint32_t t_row = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * N);
+            constexpr int QPL = 16 / H_I;   // queries per 16-column TMEM load
+            for (int q0 = q_lo; q0 < q_hi; q0 += QPL) {
+                uint32_t v[16];
+                tmem_ld_x16(t_row + (uint32_t)(q0 * H_I), v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int qq = 0; qq < QPL; ++qq) {
+                    const int t = qt * a.QT + q0 + qq;
+                    if (q0 + qq >= q_hi || t >= a.T) continue;
+                    const int64_t rowi = (int64_t)b * a.T + t;
+                    const int nv = a.n_valid ? a.n_valid[rowi] : a.S - a.T + t + 1;
+                    const uint16_t *wr = a.w + rowi * H_I;
+                    float sc = 0.f;
+#pragma unroll
+                    for (int j = 0; j < H_I; ++j) {
+                        const float wj = __uint_as_float((uint32_t)__ldg(wr + j) << 16);
+                        sc = fmaf(wj, fmaxf(__uint_as_float(v[qq * H_I + j]), 0.f), sc);
+                    }
+                    if (s < nv) a.scores[rowi * a.ld + s] = sc;
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+            if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0 && *abort_flag) report(a.dev_status, SA_DEV_TIMEOUT);
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// rows x D_I bf16, row-major; box = box_rows x D_I with the swizzle matching D_I.
+static bool make_map(CUtensorMap *m, const void *base, uint64_t rows, int D_I, int box_rows) {
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)D_I, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)D_I * 2};
+    cuuint32_t box[2] = {(cuuint32_t)D_I, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    const CUtensorMapSwizzle sw = (D_I == 64) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int N, int D_I, int H_I>
+static sa_status launch_tc(const IndexerArgs &a, cudaStream_t st) {
+    using C = IdxCfg<N, D_I>;
+    IdxKernelArgs k;
+    k.w = a.w; k.page_table = a.page_table; k.n_valid = a.n_valid; k.scores = a.scores; k.ld = a.ld;
+    k.dev_status = a.dev_status; k.max_pages = a.max_pages; k.pool_pages = a.pool_pages;
+    k.B = a.B; k.T = a.T; k.S = a.S;
+    k.QT = N / H_I;
+    k.QTN = (a.T + k.QT - 1) / k.QT;
+    k.KT = (a.S + 127) / 128;
+    const long long items = (long long)a.B * k.QTN * k.KT;
+    if (items > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
+    k.n_items = (int)items;
+    if (k.n_items == 0) return SA_OK;
+
+    CUtensorMap mk, mq;
+    const uint64_t k_rows = a.page_table ? (uint64_t)a.pool_pages * a.page_size : (uint64_t)a.B * a.S;
+    if (!make_map(&mk, a.kI, k_rows, D_I, C::kBoxRows)) return SA_ERR_CUDA;
+    if (!make_map(&mq, a.qI, (uint64_t)a.B * a.T * H_I, D_I, N)) return SA_ERR_CUDA;
+
+    auto kern = indexer_tc_kernel<N, D_I, H_I>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem) != cudaSuccess)
+        return SA_ERR_CUDA;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = k.n_items < sms ? k.n_items : sms;
+    kern<<<grid, C::kThreads, C::kSmem, st>>>(mk, mq, k);
+    return cuda_ok(cudaGetLastError());
+}
+
+template <int N, int D_I>
+static sa_status launch_tc_h(const IndexerArgs &a, cudaStream_t st) {
+    switch (a.H_I) {
+        case 1: return launch_tc<N, D_I, 1>(a, st);
+        case 2: return launch_tc<N, D_I, 2>(a, st);
+        case 4: return launch_tc<N, D_I, 4>(a, st);
+        case 8: return launch_tc<N, D_I, 8>(a, st);
+    }
+    return SA_ERR_UNSUPPORTED;
+}
+
+sa_status launch_indexer(const IndexerArgs &a, cudaStream_t st) {
+    const bool small = a.T * a.H_I <= 16;   // decode: a handful of queries per sequence
+    if (a.D_I == 64) return small ? launch_tc_h<16, 64>(a, st) : launch_tc_h<256, 64>(a, st);
+    if (a.D_I == 32) return small ? launch_tc_h<16, 32>(a, st) : launch_tc_h<256, 32>(a, st);
+    return SA_ERR_UNSUPPORTED;
+}
+
+// ------------------------------------------------------------------------
+// Fine pass over explicit candidates: one warp per query row, candidates
+// strided over lanes.  qI[t] and w[t] are staged in shared memory; each lane
+// reads its candidate's key row (D_I bf16) with 16-byte loads.  fp32 sums.
+// ------------------------------------------------------------------------
+template <int D_I, int H_I>
+__global__ void __launch_bounds__(256) indexer_cand_kernel(CandArgs a) {
+    constexpr int WPB = 8;
+    __shared__ float qs[WPB][H_I][D_I];
+    __shared__ float ws[WPB][H_I];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int t = blockIdx.x * WPB + warp;
+    if (t >= a.T) return;
+    for (int i = lane; i < H_I * D_I; i += 32)
+        qs[warp][i / D_I][i % D_I] = __uint_as_float((uint32_t)a.qI[(int64_t)t * H_I * D_I + i] << 16);
+    if (lane < H_I) ws[warp][lane] = __uint_as_float((uint32_t)a.w[(int64_t)t * H_I + lane] << 16);
+    __syncwarp();
+    int nc = a.n_cand[t];
+    if (nc < 0 || nc > a.ld_cand) { if (lane == 0) report(a.dev_status, SA_DEV_INDEX); nc = nc < 0 ? 0 : (int)a.ld_cand; }
+    const int32_t *cr = a.cand + (int64_t)t * a.ld_cand;
+    float *out = a.scores + (int64_t)t * a.ld;
+    for (int i = lane; i < nc; i += 32) {
+        const int s = cr[i];
+        if (s < 0 || s >= a.S) { report(a.dev_status, SA_DEV_INDEX); continue; }
+        const uint4 *kr = reinterpret_cast<const uint4 *>(a.kI + (int64_t)s * D_I);
+        float key[D_I];
+#pragma unroll
+        for (int c = 0; c < D_I / 8; ++c) {
+            const uint4 u = __ldg(kr + c);
+            const uint32_t wds[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                key[c * 8 + 2 * e] = __uint_as_float(wds[e] << 16);
+                key[c * 8 + 2 * e + 1] = __uint_as_float(wds[e] & 0xFFFF0000u);
+            }
+        }
+        float sc = 0.f;
+#pragma unroll
+        for (int j = 0; j < H_I; ++j) {
+            float dot = 0.f;
+#pragma unroll
+            for (int c = 0; c < D_I; ++c) dot = fmaf(qs[warp][j][c], key[c], dot);
+            sc = fmaf(ws[warp][j], fmaxf(dot, 0.f), sc);
+        }
+        out[i] = sc;
+    }
+}
+
+template <int D_I>
+static sa_status launch_cand_h(const CandArgs &a, cudaStream_t st) {
+    const dim3 grid((a.T + 7) / 8);
+    switch (a.H_I) {
+        case 1: indexer_cand_kernel<D_I, 1><<<grid, 256, 0, st>>>(a); break;
+        case 2: indexer_cand_kernel<D_I, 2><<<grid, 256, 0, st>>>(a); break;
+        case 4: indexer_cand_kernel<D_I, 4><<<grid, 256, 0, st>>>(a); break;
+        case 8: indexer_cand_kernel<D_I, 8><<<grid, 256, 0, st>>>(a); break;
+        default: return SA_ERR_UNSUPPORTED;
+    }
+    return cuda_ok(cudaGetLastError());
+}
+
+sa_status launch_indexer_candidates(const CandArgs &a, cudaStream_t st) {
+    if (a.T == 0) return SA_OK;
+    if (a.D_I == 64) return launch_cand_h<64>(a, st);
+    if (a.D_I == 32) return launch_cand_h<32>(a, st);
+    return SA_ERR_UNSUPPORTED;
+}
+
+}  // namespace sa

@@ -1,0 +1,84 @@
+// internal.h -- launchers shared between the C-ABI layer (sa_api.cu) and the
+// kernel files.  Nothing here is exported from libsa.so.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sa.h"
+
+namespace sa {
+
+struct TopkArgs {
+    const float *scores;
+    int64_t ld;
+    int rows, row_len;
+    const int32_t *n_valid;
+    const int32_t *cand;
+    int64_t ld_cand;
+    int K;
+    int32_t *out;
+    int *dev_status;
+    int chunk;   // columns per CTA (set by the launcher)
+};
+sa_status launch_topk(TopkArgs a, cudaStream_t st);
+int topk_max_row_len();
+
+struct IndexerArgs {
+    const uint16_t *qI, *w, *kI;
+    const int32_t *page_table;
+    int max_pages, pool_pages, page_size;
+    int B, T, S, H_I, D_I;
+    const int32_t *n_valid;
+    float *scores;
+    int64_t ld;
+    int *dev_status;
+};
+sa_status launch_indexer(const IndexerArgs &a, cudaStream_t st);
+
+struct CandArgs {
+    const uint16_t *qI, *w, *kI;
+    int T, S, H_I, D_I;
+    const int32_t *cand;
+    int64_t ld_cand;
+    const int32_t *n_cand;
+    float *scores;
+    int64_t ld;
+    int *dev_status;
+};
+sa_status launch_indexer_candidates(const CandArgs &a, cudaStream_t st);
+
+struct PrefillArgs {
+    const uint16_t *q, *k, *v;
+    const int32_t *topk;
+    int K, W, T, S, Hq, d;
+    float scale;
+    uint16_t *out;
+    float *lse;
+    int *dev_status;
+};
+sa_status launch_prefill(const PrefillArgs &a, cudaStream_t st);
+
+struct DecodeArgs {
+    const uint16_t *q, *k, *v;
+    const int32_t *page_table;
+    int max_pages, pool_pages, page_size, S_max;
+    const int32_t *seq_lens, *topk;
+    int K, W, B, Hq, d;
+    float scale;
+    uint16_t *out;
+    float *lse;
+    void *workspace;
+    int *dev_status;
+};
+size_t decode_workspace_bytes(int B, int Hq, int d, int K, int W);
+sa_status launch_decode(const DecodeArgs &a, cudaStream_t st);
+
+sa_status launch_pool(const uint16_t *kI, int S, int D_I, int block, uint16_t *kB, cudaStream_t st);
+sa_status launch_block_counts(int T, int S, int block, int32_t *n_blocks, cudaStream_t st);
+sa_status launch_expand(const int32_t *blocks, int T, int S, int keep, int block, int32_t *cand,
+                        int64_t ld_cand, int32_t *n_cand, int *dev_status, cudaStream_t st);
+
+inline sa_status cuda_ok(cudaError_t e) { return e == cudaSuccess ? SA_OK : SA_ERR_CUDA; }
+
+}  // namespace sa

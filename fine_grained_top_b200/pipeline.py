@@ -1,0 +1,143 @@
+"""The three-stage step built from the C-ABI calls, with buffers allocated once.
+
+A plan owns its intermediate buffers (torch device tensors) and enqueues the
+library's kernels on one stream; the host does no arithmetic of the method.
+
+    PrefillPlan    indexer -> top-K -> sparse attention for one causal
+                   sequence (optionally the two-stage coarse/fine selection)
+    DecodePlan     one new query per sequence over a contiguous or paged
+                   KV cache: indexer -> top-K -> split-K attention + merge
+
+``stages(inputs)`` returns the step as a list of (name, launch) pairs, one
+per C-ABI call, so that callers can time each kernel; ``run`` executes them.
+"""
+
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import (sa_coarse_block_counts, sa_decode_workspace_bytes, sa_expand_blocks, sa_indexer_scores,
+               sa_indexer_scores_candidates, sa_pool_index_keys, sa_sparse_attn_decode,
+               sa_sparse_attn_prefill, sa_topk_select)
+
+
+def _ld(n: int) -> int:
+    return max(4, (n + 3) // 4 * 4)
+
+
+class PrefillPlan:
+    """Buffers for one sequence of N tokens (queries at positions 0..N-1).
+    Inputs: dict with q [N,Hq,d], k/v [N,d], qI [N,H_I,D_I], w [N,H_I], kI [N,D_I]."""
+
+    def __init__(self, N, Hq, d, H_I, D_I, K, W, block=None, keep=None, device="cuda"):
+        self.N, self.Hq, self.d, self.H_I, self.D_I, self.K, self.W = N, Hq, d, H_I, D_I, K, W
+        self.block, self.keep = block, keep
+        self.scale = 1.0 / math.sqrt(d)
+        dev = torch.device(device)
+        i32, f32 = torch.int32, torch.float32
+        self.topk = torch.empty((N, K), dtype=i32, device=dev)
+        self.out = torch.empty((N, Hq, d), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((N, Hq), dtype=f32, device=dev)
+        self.dev_status = torch.zeros(1, dtype=i32, device=dev)
+        if block is None:
+            self.ld = _ld(N)
+            self.scores = torch.empty((N, self.ld), dtype=f32, device=dev)
+        else:
+            self.nb = N // block
+            self.ld_coarse = _ld(self.nb)
+            self.kB = torch.empty((max(self.nb, 1), D_I), dtype=torch.bfloat16, device=dev)
+            self.n_blocks = torch.empty(N, dtype=i32, device=dev)
+            self.coarse = torch.empty((N, self.ld_coarse), dtype=f32, device=dev)
+            self.blocks = torch.empty((N, keep), dtype=i32, device=dev)
+            self.ld_cand = _ld(keep * block + block)
+            self.cand = torch.empty((N, self.ld_cand), dtype=i32, device=dev)
+            self.n_cand = torch.empty(N, dtype=i32, device=dev)
+            self.fine = torch.empty((N, self.ld_cand), dtype=f32, device=dev)
+
+    def stages(self, x, stream=None):
+        N, K, ds, H, D = self.N, self.K, self.dev_status, self.H_I, self.D_I
+        attn = ("attention", lambda: sa_sparse_attn_prefill(
+            x["q"], x["k"], x["v"], self.topk, K, self.W, N, N, self.Hq, self.d, self.scale, self.out,
+            self.lse, ds, stream))
+        if self.block is None:
+            return [
+                ("indexer", lambda: sa_indexer_scores(x["qI"], x["w"], x["kI"], None, 0, 0, 64, 1, N, N, H, D,
+                                                      None, self.scores, self.ld, ds, stream)),
+                ("topk", lambda: sa_topk_select(self.scores, self.ld, N, N, None, None, 0, K, self.topk, ds,
+                                                stream)),
+                attn]
+        blk, keep = self.block, self.keep
+        return [
+            ("pool", lambda: sa_pool_index_keys(x["kI"], N, D, blk, self.kB, stream)),
+            ("block_counts", lambda: sa_coarse_block_counts(N, N, blk, self.n_blocks, stream)),
+            ("coarse_indexer", lambda: sa_indexer_scores(x["qI"], x["w"], self.kB, None, 0, 0, 64, 1, N, self.nb,
+                                                         H, D, self.n_blocks, self.coarse, self.ld_coarse, ds,
+                                                         stream)),
+            ("coarse_topk", lambda: sa_topk_select(self.coarse, self.ld_coarse, N, self.nb, self.n_blocks, None,
+                                                   0, keep, self.blocks, ds, stream)),
+            ("expand", lambda: sa_expand_blocks(self.blocks, N, N, keep, blk, self.cand, self.ld_cand,
+                                                self.n_cand, ds, stream)),
+            ("fine_indexer", lambda: sa_indexer_scores_candidates(x["qI"], x["w"], x["kI"], N, N, H, D,
+                                                                  self.cand, self.ld_cand, self.n_cand,
+                                                                  self.fine, self.ld_cand, ds, stream)),
+            ("fine_topk", lambda: sa_topk_select(self.fine, self.ld_cand, N, self.ld_cand, self.n_cand,
+                                                 self.cand, self.ld_cand, K, self.topk, ds, stream)),
+            attn]
+
+    def run(self, q, k, v, qI, w, kI, stream=None):
+        for _, fn in self.stages(dict(q=q, k=k, v=v, qI=qI, w=w, kI=kI), stream):
+            fn()
+        return self.out
+
+    def launches(self) -> int:
+        """Kernels one run() enqueues."""
+        return 3 if self.block is None else 8
+
+
+class DecodePlan:
+    """Buffers for B sequences, one query each, over a contiguous ([B, S_max, *])
+    or paged (pools [P, 64, *] + page_table [B, max_pages]) cache.
+    Inputs: dict with q [B,Hq,d], k/v/kI caches, qI [B,H_I,D_I], w [B,H_I],
+    lengths [B] int32 and, when paged, page_table."""
+
+    def __init__(self, B, Hq, d, H_I, D_I, K, W, S_max, paged=False, max_pages=0, pool_pages=0,
+                 device="cuda"):
+        self.B, self.Hq, self.d, self.H_I, self.D_I, self.K, self.W = B, Hq, d, H_I, D_I, K, W
+        self.paged, self.max_pages, self.pool_pages = paged, max_pages, pool_pages
+        self.S = max_pages * 64 if paged else S_max
+        self.S_max = S_max
+        self.scale = 1.0 / math.sqrt(d)
+        dev = torch.device(device)
+        self.ld = _ld(self.S)
+        self.scores = torch.empty((B, self.ld), dtype=torch.float32, device=dev)
+        self.topk = torch.empty((B, K), dtype=torch.int32, device=dev)
+        self.out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+        self.ws_bytes = sa_decode_workspace_bytes(B, Hq, d, K, W)
+        self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=dev)
+        self.dev_status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def stages(self, x, stream=None):
+        ds, pt = self.dev_status, x.get("page_table")
+        return [
+            ("indexer", lambda: sa_indexer_scores(x["qI"], x["w"], x["kI"], pt, self.max_pages, self.pool_pages,
+                                                  64, self.B, 1, self.S, self.H_I, self.D_I, x["lengths"],
+                                                  self.scores, self.ld, ds, stream)),
+            ("topk", lambda: sa_topk_select(self.scores, self.ld, self.B, self.S, x["lengths"], None, 0, self.K,
+                                            self.topk, ds, stream)),
+            ("attention", lambda: sa_sparse_attn_decode(
+                x["q"], x["k"], x["v"], pt, self.max_pages, self.pool_pages, 64, self.S_max, x["lengths"],
+                self.topk, self.K, self.W, self.B, self.Hq, self.d, self.scale, self.out, self.lse,
+                self.workspace, self.ws_bytes, ds, stream)),
+        ]
+
+    def run(self, q, k_cache, v_cache, qI, w, kI, seq_lens, page_table=None, stream=None):
+        x = dict(q=q, k=k_cache, v=v_cache, qI=qI, w=w, kI=kI, lengths=seq_lens, page_table=page_table)
+        for _, fn in self.stages(x, stream):
+            fn()
+        return self.out
+
+    def launches(self) -> int:
+        return 4   # indexer, top-K, split attention, merge

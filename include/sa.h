@@ -1,0 +1,233 @@
+/*
+ * sa.h -- C ABI of libsa.so: fine-grained top-K sparse attention on B200.
+ *
+ * The method (three stages, all queries of a token sharing one selection over
+ * one shared KV head):
+ *   1. a lightweight indexer scores every causal (query t, key s) pair,
+ *        I[t,s] = sum_j w[t,j] * ReLU(qI[t,j] . kI[s])
+ *      ("Sparse Attention for Long-Context LLM Inference", section "Where
+ *      Sparse Attention Is Actually Sparse": a lightweight indexer scores the
+ *      history and hands candidate indices to attention; "Sparse Attention in
+ *      2026", "The designs that shipped": the lightning indexer is a small,
+ *      few-head, low-precision scorer feeding top-k 2048), optionally after a
+ *      coarse pass over mean-pooled 64-token blocks ("Why fine-grained sparse
+ *      attention ...", section "What Fine-Grained Means");
+ *   2. each query keeps its K best keys (ties -> lower position) and always
+ *      the W most recent positions ("Sparse Attention", completesystemdesign,
+ *      mask diagrams: "+ always the local window");
+ *   3. exact softmax(q.k/sqrt(d)) v over only the selected keys
+ *      ("A Guide to Sparse Attention in Large Models", section 2, masked form
+ *      with Mask[i,j] = 1 iff j in S(i); section 4.2, index-based path).
+ *
+ * Conventions shared by every entry point
+ *   - Every pointer named in an argument list is DEVICE memory owned by the
+ *     caller, unless the comment says "host".  The library never allocates,
+ *     frees, or keeps a pointer past the call.
+ *   - All work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream).  The library never synchronises.
+ *   - The return value reports synchronous argument checks.  On any status
+ *     other than SA_OK nothing has been enqueued.
+ *   - `dev_status` (device int32, may be NULL) receives errors found while
+ *     kernels run: kernels OR SA_DEV_* bits into it.  The caller zeroes it
+ *     before the call and reads it after synchronising.  An out-of-range index
+ *     or page id is never dereferenced: the access is skipped and the bit set.
+ *   - bf16 values are passed as raw 16-bit patterns (sa_bf16).
+ *   - Supported shapes: d (attention head dim) in {64, 128}; D_I (indexer
+ *     dim) in {32, 64}; H_I in {1, 2, 4, 8}; 1 <= Hq <= 64 query heads;
+ *     page_size 64.  Other shapes return SA_ERR_UNSUPPORTED.  There is no
+ *     fallback path.
+ */
+#ifndef FINE_GRAINED_TOP_SA_H
+#define FINE_GRAINED_TOP_SA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t sa_bf16;                 /* raw bfloat16 bits */
+typedef struct CUstream_st *sa_stream;    /* same type as cudaStream_t */
+
+typedef enum {
+    SA_OK = 0,
+    SA_ERR_INVALID_ARG = 1,   /* NULL pointer, negative size, bad stride ...  */
+    SA_ERR_UNSUPPORTED = 2,   /* shape outside the supported set              */
+    SA_ERR_CUDA = 3,          /* a CUDA runtime call failed (launch, attr)    */
+    SA_ERR_TIMEOUT = 4,       /* (decoded from dev_status) a bounded wait gave up */
+    SA_ERR_INDEX = 5,         /* (decoded from dev_status) bad index / page id */
+    SA_ERR_WORKSPACE = 6      /* caller's workspace is smaller than required  */
+} sa_status;
+
+/* bits OR-ed into *dev_status by kernels */
+#define SA_DEV_INDEX   0x1    /* an index, candidate or page id out of range   */
+#define SA_DEV_ORDER   0x2    /* a top-K / candidate row not strictly ascending */
+#define SA_DEV_TIMEOUT 0x4    /* a bounded pipeline wait ran out               */
+
+/* Human-readable name of a status (static storage). */
+const char *sa_status_string(sa_status s);
+
+/* Maps a dev_status word (read back by the caller) to a status:
+ * SA_OK, SA_ERR_TIMEOUT or SA_ERR_INDEX. */
+sa_status sa_dev_status_decode(int word);
+
+/* Library ABI version (major * 100 + minor). */
+int sa_version(void);
+
+/* ------------------------------------------------------------------------
+ * Stage 1 -- indexer scores (tensor cores: tcgen05 MMA into TMEM, TMA loads)
+ *
+ *   scores[(b*T + t) * ld_scores + s] =
+ *       sum_{j < H_I} w[b,t,j] * max(0, sum_{c < D_I} qI[b,t,j,c] * kI_b[s,c])
+ *   for 0 <= s < n_valid[b*T + t]; no 1/sqrt(D_I), no softmax, no positional
+ *   term ("Where Sparse Attention Is Actually Sparse": the indexer omits
+ *   positional encoding).  Sums are fp32 (exact for the integer-valued inputs
+ *   used by the tests).  Columns s >= n_valid of a row are NOT written: their
+ *   contents are unspecified and every consumer bounds rows by n_valid.
+ *
+ *   qI        [B, T, H_I, D_I] bf16
+ *   w         [B, T, H_I] bf16
+ *   kI        contiguous (page_table == NULL): [B, S, D_I] bf16, sequence b's
+ *             key s at row b*S + s;
+ *             paged: a pool [P, page_size, D_I]; key s of sequence b at row
+ *             page_table[b*max_pages + s/page_size]*page_size + s%page_size.
+ *   n_valid   [B*T] number of leading key columns scored for each query row
+ *             (0 .. S); NULL means causal prefill with the T queries at the
+ *             last T of S positions: n_valid = S - T + t + 1.
+ *   scores    [B*T, ld_scores] fp32, ld_scores >= S and a multiple of 4.
+ *   Errors: SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_CUDA; device:
+ *   SA_DEV_INDEX for a page id outside [0, P) (P = pool_pages), or an
+ *   n_valid entry outside [0, S]; SA_DEV_TIMEOUT.
+ * ---------------------------------------------------------------------- */
+sa_status sa_indexer_scores(const sa_bf16 *qI, const sa_bf16 *w,
+                            const sa_bf16 *kI, const int32_t *page_table,
+                            int max_pages, int pool_pages, int page_size,
+                            int B, int T, int S, int H_I, int D_I,
+                            const int32_t *n_valid, float *scores,
+                            int64_t ld_scores, int *dev_status,
+                            sa_stream stream);
+
+/* Indexer scores over an explicit candidate list per query (the fine pass of
+ * the two-stage selection, "What Fine-Grained Means": the fine pass scores
+ * individual tokens inside the coarse candidates).
+ *   scores[t*ld_scores + i] = I[t, cand[t*ld_cand + i]] for i < n_cand[t];
+ *   entries i >= n_cand[t] are not written.
+ *   qI [T, H_I, D_I], w [T, H_I], kI [S, D_I] (contiguous), cand int32 with
+ *   every used entry in [0, S) (else SA_DEV_INDEX, entry skipped).
+ *   n_cand[t] must lie in [0, ld_cand] and ld_scores >= ld_cand. */
+sa_status sa_indexer_scores_candidates(const sa_bf16 *qI, const sa_bf16 *w,
+                                       const sa_bf16 *kI, int T, int S,
+                                       int H_I, int D_I, const int32_t *cand,
+                                       int64_t ld_cand, const int32_t *n_cand,
+                                       float *scores, int64_t ld_scores,
+                                       int *dev_status, sa_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Stage 2 -- top-K select ("Where Sparse Attention Is Actually Sparse": Top-K
+ * caps how many history positions take part in exact attention)
+ *
+ *   For each row r, among columns 0 <= col < n_valid[r] of
+ *   scores[r*ld_scores + col], keep the min(K, n_valid[r]) largest scores;
+ *   equal scores are ranked by lower position.  The position of a column is
+ *   the column itself, or cand_map[r*ld_cand + col] when cand_map != NULL, in
+ *   which case each row of cand_map must be strictly ascending over its valid
+ *   columns (as sa_expand_blocks writes it) so that "lower column" means
+ *   "lower position" (SA_DEV_ORDER otherwise).
+ *   topk[r*K + i], i < K: the kept positions in ascending order, then -1.
+ *   The result is unique, so it is bit-exact.
+ *
+ *   n_valid   [rows] or NULL (NULL: causal rows at the last `rows` of
+ *             `row_len` positions, n_valid = row_len - rows + r + 1).
+ *   Order-preserving keys: NaN scores are not supported; -inf sorts last.
+ *   Limits: row_len <= 393216; K >= 0.
+ *   Rows are split over a thread-block cluster (1..8 CTAs, distributed
+ *   shared memory for the histograms); no workspace is needed.
+ * ---------------------------------------------------------------------- */
+sa_status sa_topk_select(const float *scores, int64_t ld_scores, int rows,
+                         int row_len, const int32_t *n_valid,
+                         const int32_t *cand_map, int64_t ld_cand, int K,
+                         int32_t *topk, int *dev_status, sa_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Stage 3a -- sparse attention, prefill
+ *
+ *   Query t (t < T) sits at position p = S - T + t.  Its key set is
+ *     S(t) = {s in topk[t, :] : 0 <= s <= p - W} U {max(0, p-W+1) .. p}
+ *   (top-K entries inside the window are taken once, from the window), and
+ *     out[t,h,:] = sum_{s in S(t)} softmax_s(q[t,h,:] . k[s,:] * scale) v[s,:]
+ *   for every head h < Hq; all heads share S(t) and the single KV head.
+ *   lse[t,h] = log(sum_s exp(q.k*scale)) (natural log), if lse != NULL.
+ *   q [T, Hq, d], k/v [S, d], topk [T, K] ascending, -1 padded (as
+ *   sa_topk_select writes it), out [T, Hq, d] bf16, lse [T, Hq] fp32.
+ *   Softmax and accumulation are fp32; probabilities are rounded to bf16 for
+ *   the P.V product; out is rounded to bf16 (nearest even).
+ *   Device errors: a top-K entry > p sets SA_DEV_INDEX and is skipped; a row
+ *   that is not strictly ascending sets SA_DEV_ORDER.
+ * ---------------------------------------------------------------------- */
+sa_status sa_sparse_attn_prefill(const sa_bf16 *q, const sa_bf16 *k,
+                                 const sa_bf16 *v, const int32_t *topk, int K,
+                                 int W, int T, int S, int Hq, int d,
+                                 float scale, sa_bf16 *out, float *lse,
+                                 int *dev_status, sa_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Stage 3b -- sparse attention, decode (one new query per sequence)
+ *
+ *   Sequence b has seq_lens[b] tokens; its query sits at p = seq_lens[b] - 1
+ *   (its own k/v/kI already appended).  Key set and output as in prefill.
+ *   k_cache/v_cache: contiguous (page_table == NULL) [B, S_max, d]; paged:
+ *   pools [P, page_size, d] addressed through page_table [B, max_pages].
+ *   The selection is split into chunks processed by separate CTAs; their
+ *   partial softmax states go to `workspace` and a second kernel merges them
+ *   (log-sum-exp).  workspace: device memory of at least
+ *   sa_decode_workspace_bytes(B, Hq, d, K, W) bytes, 256-byte aligned, owned
+ *   by the caller; contents on entry do not matter.
+ *   Errors: SA_ERR_WORKSPACE if too small; device SA_DEV_INDEX for a bad
+ *   top-K entry or page id (skipped), SA_DEV_ORDER for a non-ascending row.
+ * ---------------------------------------------------------------------- */
+size_t sa_decode_workspace_bytes(int B, int Hq, int d, int K, int W);
+
+sa_status sa_sparse_attn_decode(const sa_bf16 *q, const sa_bf16 *k_cache,
+                                const sa_bf16 *v_cache,
+                                const int32_t *page_table, int max_pages,
+                                int pool_pages, int page_size, int S_max,
+                                const int32_t *seq_lens, const int32_t *topk,
+                                int K, int W, int B, int Hq, int d,
+                                float scale, sa_bf16 *out, float *lse,
+                                void *workspace, size_t workspace_bytes,
+                                int *dev_status, sa_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Two-stage selection helpers ("What Fine-Grained Means": a coarse block pass
+ * picks candidate regions cheaply, a fine pass picks top-K tokens inside
+ * them; section 2 "Learned Block Routing": blocks are mean-pooled over
+ * complete blocks and scored by dot product).
+ * ---------------------------------------------------------------------- */
+
+/* kB[b, c] = bf16(mean of kI[b*block + i, c], i < block) for the S/block
+ * complete blocks (a partial tail block is dropped).  The mean is an fp32 sum
+ * divided by `block`, rounded to bf16 (exact for integer-valued keys with
+ * |sum| <= 256 and a power-of-two block). */
+sa_status sa_pool_index_keys(const sa_bf16 *kI, int S, int D_I, int block,
+                             sa_bf16 *kB, sa_stream stream);
+
+/* n_blocks[t] = floor((S - T + t) / block): the number of complete blocks
+ * that lie entirely before the block holding query t -- the coarse pass's
+ * eligible blocks (and its n_valid for sa_indexer_scores / sa_topk_select). */
+sa_status sa_coarse_block_counts(int T, int S, int block, int32_t *n_blocks,
+                                 sa_stream stream);
+
+/* Candidates of the fine pass for query t at position p = S - T + t:
+ *   the tokens of the kept blocks (blocks[t, :keep], ascending, -1 padded, as
+ *   sa_topk_select writes it), then the tokens of p's own block up to p.
+ *   cand[t*ld_cand + i] for i < n_cand[t] (ascending); ld_cand >= keep*block +
+ *   block.  A block id >= floor(p/block) sets SA_DEV_INDEX and is skipped. */
+sa_status sa_expand_blocks(const int32_t *blocks, int T, int S, int keep,
+                           int block, int32_t *cand, int64_t ld_cand,
+                           int32_t *n_cand, int *dev_status, sa_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FINE_GRAINED_TOP_SA_H */

@@ -1,0 +1,284 @@
+"""GPU parity: every stage through the C ABI against the CPU fp64 oracle.
+
+Index sets (top-K, block selection, candidates) must match bit for bit;
+attention outputs within max-abs 2e-2 and mean-abs 2e-3 of the fp64 result.
+Inputs are the seeded synthetic workloads (workloads/); nothing here reads a
+stored GPU result.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from workloads import CONFIGS, config_inputs, gen_decode, gen_prefill
+from tests.gpu_helpers import assert_close_attention, dev, host_f64, status
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def sa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    import fine_grained_top_b200 as m
+    return m
+
+
+def _pl():
+    from fine_grained_top_b200.pipeline import DecodePlan, PrefillPlan
+    return PrefillPlan, DecodePlan
+
+
+def _to_dev(inp, names=("q", "k", "v", "qI", "w", "kI")):
+    return {n: dev(inp[n]) for n in names}
+
+
+# ====================================================================== top-K
+def _scores(rows, L, dist, rng):
+    if dist == "ties3":
+        return rng.integers(0, 3, size=(rows, L)).astype(np.float32)
+    if dist == "ints":
+        return rng.integers(0, 2000, size=(rows, L)).astype(np.float32)
+    return rng.standard_normal((rows, L)).astype(np.float32)
+
+
+@pytest.mark.parametrize("rows,L,K,dist", [
+    (37, 700, 64, "ties3"), (16, 5000, 1024, "ints"), (50, 17000, 700, "normal"),
+    (3, 40000, 100, "normal"), (8, 131072, 2048, "ints"), (4, 262144, 2048, "ties3"),
+    (5, 393216, 3000, "ints"), (9, 33, 40, "normal"), (64, 1023, 64, "ints"),
+])
+def test_topk_matches_oracle(sa, rows, L, K, dist):
+    rng = np.random.default_rng(rows * 7 + L)
+    sc = _scores(rows, L, dist, rng)
+    n_valid = rng.integers(0, L + 1, size=rows).astype(np.int32)
+    n_valid[0] = L
+    n_valid[-1] = min(L, K)
+    if rows > 2:
+        n_valid[1] = 0
+    ld = (L + 3) // 4 * 4
+    buf = np.full((rows, ld), np.nan, np.float32)
+    buf[:, :L] = sc
+    out = torch.empty((rows, K), dtype=torch.int32, device="cuda")
+    ds = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sa.sa_topk_select(dev(buf), ld, rows, L, dev(n_valid), None, 0, K, out, ds)
+    want = oracle.topk(sc.astype(np.float64), n_valid, K)
+    assert status(ds) == 0
+    assert np.array_equal(out.cpu().numpy(), want)
+
+
+def test_topk_causal_default_and_neg_inf(sa):
+    rng = np.random.default_rng(3)
+    rows, L, K = 300, 300, 37
+    sc = rng.integers(0, 5, size=(rows, L)).astype(np.float32)
+    sc[:, ::7] = -np.inf
+    out = torch.empty((rows, K), dtype=torch.int32, device="cuda")
+    sa.sa_topk_select(dev(sc), L, rows, L, None, None, 0, K, out)
+    want = oracle.topk(sc.astype(np.float64), np.arange(rows) + 1, K)
+    assert np.array_equal(out.cpu().numpy(), want)
+
+
+def test_topk_candidate_map(sa):
+    rng = np.random.default_rng(4)
+    rows, L, K = 40, 4160, 2048
+    sc = rng.integers(0, 50, size=(rows, L)).astype(np.float32)
+    cand = np.sort(rng.choice(1 << 20, size=(rows, L), replace=True), axis=1).astype(np.int32)
+    cand = cand + np.arange(L, dtype=np.int32)[None, :]          # strictly ascending
+    n_valid = rng.integers(1000, L + 1, size=rows).astype(np.int32)
+    out = torch.empty((rows, K), dtype=torch.int32, device="cuda")
+    ds = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sa.sa_topk_select(dev(sc), L, rows, L, dev(n_valid), dev(cand), L, K, out, ds)
+    want = oracle.topk(sc.astype(np.float64), n_valid, K, cand=cand)
+    assert status(ds) == 0
+    assert np.array_equal(out.cpu().numpy(), want)
+
+
+# ====================================================================== indexer
+@pytest.mark.parametrize("N,H_I,D_I,rows", [
+    (512, 2, 32, None), (1000, 4, 64, None), (300, 8, 64, None), (777, 1, 32, None),
+    (129, 4, 64, None), (1, 4, 64, None), (8192, 4, 64, 384),
+])
+def test_indexer_prefill_exact(sa, N, H_I, D_I, rows):
+    inp = gen_prefill(N=N, Hq=1, d=64, H_I=H_I, D_I=D_I, seed=N + H_I)
+    t = _to_dev(inp, ("qI", "w", "kI"))
+    ld = (N + 3) // 4 * 4
+    sc = torch.full((N, ld), float("nan"), device="cuda")
+    ds = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sa.sa_indexer_scores(t["qI"], t["w"], t["kI"], None, 0, 0, 64, 1, N, N, H_I, D_I, None, sc, ld, ds)
+    got = sc.cpu().numpy()
+    assert status(ds) == 0
+    r = np.arange(N) if rows is None else np.unique(np.r_[np.linspace(0, N - 1, rows).astype(int), 0, 127, 128])
+    want = oracle.indexer(inp["qI"][r], inp["w"][r], inp["kI"], r)
+    for i, t_ in enumerate(r):
+        assert np.array_equal(got[t_, :t_ + 1], want[i, :t_ + 1]), t_
+
+
+def test_indexer_decode_contiguous_and_paged(sa):
+    lengths = [131072, 5000, 1, 64, 65, 130000]
+    B = len(lengths)
+    for paged in (False, True):
+        inp = gen_decode(B=B, lengths=lengths, Hq=16, d=64, H_I=8, D_I=64, paged=paged, seed=5)
+        t = _to_dev(inp, ("qI", "w", "kI"))
+        sl = dev(inp["lengths"])
+        if paged:
+            S = inp["page_table"].shape[1] * 64
+            pt, mp, pp = dev(inp["page_table"]), inp["page_table"].shape[1], inp["kI"].shape[0]
+        else:
+            S, pt, mp, pp = inp["kI"].shape[1], None, 0, 0
+        sc = torch.full((B, S), float("nan"), device="cuda")
+        ds = torch.zeros(1, dtype=torch.int32, device="cuda")
+        sa.sa_indexer_scores(t["qI"], t["w"], t["kI"], pt, mp, pp, 64, B, 1, S, 8, 64, sl, sc, S, ds)
+        got = sc.cpu().numpy()
+        assert status(ds) == 0
+        for b, L in enumerate(lengths):
+            _, _, kI = oracle.decode_sequence(inp, b)
+            want = oracle.indexer(inp["qI"][b:b + 1], inp["w"][b:b + 1], kI, [L - 1])
+            assert np.array_equal(got[b, :L], want[0]), (paged, b)
+
+
+# ====================================================================== attention
+@pytest.mark.parametrize("N,Hq,d,K,W", [
+    (512, 4, 64, 64, 32), (700, 16, 128, 100, 17), (300, 20, 64, 50, 0), (257, 64, 128, 64, 64),
+    (90, 16, 128, 200, 8), (1, 16, 128, 4, 4), (200, 32, 64, 0, 5),
+])
+def test_prefill_attention_given_oracle_topk(sa, N, Hq, d, K, W):
+    inp = gen_prefill(N=N, Hq=Hq, d=d, H_I=2, D_I=32, seed=N + Hq)
+    t = _to_dev(inp, ("q", "k", "v"))
+    if K > 0:
+        sc = oracle.indexer(inp["qI"], inp["w"], inp["kI"], np.arange(N))
+        top = oracle.topk(sc, np.arange(N) + 1, K)
+        top_d = dev(top.astype(np.int32))
+    else:
+        top, top_d = np.zeros((N, 0), np.int64), None
+    out = torch.empty((N, Hq, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((N, Hq), dtype=torch.float32, device="cuda")
+    ds = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sa.sa_sparse_attn_prefill(t["q"], t["k"], t["v"], top_d, K, W, N, N, Hq, d, 1 / math.sqrt(d), out, lse, ds)
+    ptr, idx = oracle.selection(top, W, np.arange(N))
+    o, l = oracle.sparse_attention(inp["q"], inp["k"], inp["v"], ptr, idx, 1 / math.sqrt(d))
+    assert status(ds) == 0
+    assert_close_attention(host_f64(out), o, "out")
+    assert np.max(np.abs(host_f64(lse) - l)) < 1e-3
+
+
+# ====================================================================== end to end
+def _prefill_e2e(sa, inp, K, W, rows=None, block=None, keep=None):
+    PrefillPlan, _ = _pl()
+    N, Hq, d = inp["q"].shape
+    H_I, D_I = inp["qI"].shape[1:]
+    plan = PrefillPlan(N, Hq, d, H_I, D_I, K, W, block=block, keep=keep)
+    t = _to_dev(inp)
+    plan.run(t["q"], t["k"], t["v"], t["qI"], t["w"], t["kI"])
+    assert status(plan.dev_status) == 0
+    ref = oracle.prefill(inp, K, W, rows=rows, block=block, keep=keep)
+    r = np.arange(N) if rows is None else np.asarray(rows)
+    assert np.array_equal(plan.topk.cpu().numpy()[r], ref["topk"])
+    assert_close_attention(host_f64(plan.out)[r], ref["out"], "out")
+    assert np.max(np.abs(host_f64(plan.lse)[r] - ref["lse"])) < 1e-3
+    return plan, ref
+
+
+def test_e2e_prefill_512(sa):
+    c = CONFIGS["prefill_512"]
+    _prefill_e2e(sa, config_inputs("prefill_512"), c["K"], c["W"])
+
+
+def test_e2e_prefill_8k(sa):
+    c = CONFIGS["prefill_8k"]
+    inp = config_inputs("prefill_8k")
+    N = c["N"]
+    rows = np.unique(np.r_[np.linspace(0, N - 1, 160).astype(int), 1023, 1024, 1151, 1152, N - 1])
+    plan, _ = _prefill_e2e(sa, inp, c["K"], c["W"], rows=rows)
+    # every row's index set, bit for bit (the oracle's selection of all 8192 rows)
+    sc = oracle.indexer(inp["qI"], inp["w"], inp["kI"], np.arange(N))
+    want = oracle.topk(sc, np.arange(N) + 1, c["K"])
+    assert np.array_equal(plan.topk.cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("N,block,keep,K,W", [(1000, 64, 4, 100, 16), (4096, 64, 16, 512, 64),
+                                               (640, 64, 100, 300, 8)])
+def test_e2e_two_stage_small(sa, N, block, keep, K, W):
+    inp = gen_prefill(N=N, Hq=16, d=128, H_I=4, D_I=64, seed=N + keep)
+    _prefill_e2e(sa, inp, K, W, block=block, keep=keep)
+
+
+def test_e2e_two_stage_64k_sampled(sa):
+    c = CONFIGS["prefill_64k_two_stage"]
+    inp = config_inputs("prefill_64k_two_stage")
+    N = c["N"]
+    rows = np.unique(np.r_[np.linspace(0, N - 1, 40).astype(int), 63, 64, 4159, 4160, 4223, N - 1])
+    plan, ref = _prefill_e2e(sa, inp, c["K"], c["W"], rows=rows, block=c["block"], keep=c["keep"])
+    assert np.array_equal(plan.blocks.cpu().numpy()[rows], ref["blocks"])
+
+
+def _decode_e2e(sa, inp, K, W):
+    _, DecodePlan = _pl()
+    B, Hq, d = inp["q"].shape
+    H_I, D_I = inp["qI"].shape[1:]
+    paged = "page_table" in inp
+    t = _to_dev(inp)
+    sl = dev(inp["lengths"])
+    if paged:
+        pt = dev(inp["page_table"])
+        plan = DecodePlan(B, Hq, d, H_I, D_I, K, W, S_max=0, paged=True,
+                          max_pages=inp["page_table"].shape[1], pool_pages=inp["k"].shape[0])
+    else:
+        pt = None
+        plan = DecodePlan(B, Hq, d, H_I, D_I, K, W, S_max=inp["k"].shape[1])
+    plan.run(t["q"], t["k"], t["v"], t["qI"], t["w"], t["kI"], sl, pt)
+    assert status(plan.dev_status) == 0
+    ref = oracle.decode(inp, K, W)
+    assert np.array_equal(plan.topk.cpu().numpy(), ref["topk"])
+    assert_close_attention(host_f64(plan.out), ref["out"], "decode out")
+    assert np.max(np.abs(host_f64(plan.lse) - ref["lse"])) < 1e-3
+
+
+def test_e2e_decode_8x128k(sa):
+    c = CONFIGS["decode_8x128k"]
+    _decode_e2e(sa, config_inputs("decode_8x128k"), c["K"], c["W"])
+
+
+def test_e2e_decode_paged_16(sa):
+    c = CONFIGS["decode_paged_16x256k"]
+    _decode_e2e(sa, config_inputs("decode_paged_16x256k"), c["K"], c["W"])
+
+
+@pytest.mark.parametrize("lengths,K,W", [([1, 2, 63, 64, 65, 3000], 100, 16), ([5000, 700], 4096, 0),
+                                         ([129, 10000], 0, 600)])
+def test_decode_edge_lengths(sa, lengths, K, W):
+    for paged in (False, True):
+        inp = gen_decode(B=len(lengths), lengths=lengths, Hq=64, d=128, H_I=8, D_I=64, paged=paged, seed=11)
+        _decode_e2e(sa, inp, K, W)
+
+
+# ====================================================================== device errors
+def test_planted_bad_index_and_order_are_reported(sa):
+    N, Hq, d, K, W = 100, 16, 128, 8, 4
+    inp = gen_prefill(N=N, Hq=Hq, d=d, H_I=2, D_I=32, seed=1)
+    t = _to_dev(inp, ("q", "k", "v"))
+    top = np.tile(np.arange(K, dtype=np.int32), (N, 1))
+    top[50, 3] = 99            # beyond position 50
+    out = torch.empty((N, Hq, d), dtype=torch.bfloat16, device="cuda")
+    ds = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sa.sa_sparse_attn_prefill(t["q"], t["k"], t["v"], dev(top), K, W, N, N, Hq, d, 0.1, out, None, ds)
+    assert status(ds) & sa.SA_DEV_INDEX
+    assert torch.isfinite(out.float()).all()
+    top2 = np.tile(np.arange(K, dtype=np.int32), (N, 1))
+    top2[60, 2], top2[60, 3] = 5, 4   # not ascending
+    ds.zero_()
+    sa.sa_sparse_attn_prefill(t["q"], t["k"], t["v"], dev(top2), K, W, N, N, Hq, d, 0.1, out, None, ds)
+    assert status(ds) & sa.SA_DEV_ORDER
+
+
+def test_planted_bad_page_is_reported(sa):
+    inp = gen_decode(B=2, lengths=[300, 200], Hq=16, d=128, H_I=8, D_I=64, paged=True, seed=2)
+    inp["page_table"][1, 1] = 10 ** 6
+    _, DecodePlan = _pl()
+    t = _to_dev(inp)
+    plan = DecodePlan(2, 16, 128, 8, 64, 16, 8, S_max=0, paged=True, max_pages=inp["page_table"].shape[1],
+                      pool_pages=inp["k"].shape[0])
+    plan.run(t["q"], t["k"], t["v"], t["qI"], t["w"], t["kI"], dev(inp["lengths"]), dev(inp["page_table"]))
+    assert status(plan.dev_status) & sa.SA_DEV_INDEX
+    assert torch.isfinite(plan.out.float()).all()
