@@ -58,7 +58,10 @@ struct IdxCfg {
     static constexpr uint32_t kSbo = 8 * kSwizzleBytes;        // 8-row core group stride
     static constexpr uint32_t kLayout = (D_I == 64) ? 2 : 4;   // UMMA layout: 128B / 64B swizzle
     static constexpr int kEpiGroups = kEpiWarps / 4;
-    static constexpr size_t kSmem = 1024 + (size_t)kStages * kStageBytes + 1024;
+    // at least 116 KB so that exactly one persistent CTA (and one TMEM
+    // allocation) lands on each SM
+    static constexpr size_t kSmemUsed = 1024 + (size_t)kStages * kStageBytes + 1024;
+    static constexpr size_t kSmem = kSmemUsed > 118784 ? kSmemUsed : 118784;
 };
 
 // Largest n_valid among the tile's queries (the tile's key extent).  Called
@@ -242,7 +245,11 @@ __global__ void __launch_bounds__(IdxCfg<N, D_I>::kThreads, 1)
                     const int t = qt * a.QT + q0 + qq;
                     if (q0 + qq >= q_hi || t >= a.T) continue;
                     const int64_t rowi = (int64_t)b * a.T + t;
-                    const int nv = a.n_valid ? a.n_valid[rowi] : a.S - a.T + t + 1;
+                    int nv = a.n_valid ? a.n_valid[rowi] : a.S - a.T + t + 1;
+                    if (nv < 0 || nv > a.S) {   // never write outside the row
+                        if (kt == 0 && quad == 0 && lane == 0) report(a.dev_status, SA_DEV_INDEX);
+                        nv = nv < 0 ? 0 : a.S;
+                    }
                     const uint16_t *wr = a.w + rowi * H_I;
                     float sc = 0.f;
 #pragma unroll
