@@ -38,6 +38,8 @@ SIGNATURES = {
     "sa_decode_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32]),
     "sa_sparse_attn_decode": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _i32,
                                      _i32, _i32, _i32, _f32, _vp, _vp, _vp, _sz, _vp, _vp]),
+    "sa_sparse_attn_decode_noalloc": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _i32,
+                                             _i32, _i32, _i32, _i32, _f32, _vp, _vp, _vp, _vp]),
     "sa_pool_index_keys": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp]),
     "sa_coarse_block_counts": (_i32, [_i32, _i32, _i32, _vp, _vp]),
     "sa_expand_blocks": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _vp]),
@@ -52,7 +54,7 @@ class SAError(RuntimeError):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError("libsa.so is not built; run `python -m fine_grained_top_b200.build` "
+        raise ImportError("libsa.so is not built; run `python fine_grained_top_b200/build.py` "
                           "(there is no fallback path)")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in SIGNATURES.items():
@@ -125,6 +127,22 @@ def sa_sparse_attn_decode(q, k_cache, v_cache, page_table, max_pages, pool_pages
                                       Hq, d, float(scale), _ptr(out), _ptr(lse), _ptr(workspace),
                                       workspace_bytes, _ptr(dev_status), _stream(stream)),
            "sa_sparse_attn_decode")
+
+
+def sa_sparse_attn_decode_noalloc(q, k_cache, v_cache, page_table, max_pages, pool_pages, page_size, S_max,
+                                  seq_lens, topk, K, W, B, Hq, d, scale, out, lse=None, dev_status=None,
+                                  stream=None):
+    """Decode for callers that cannot allocate device memory: the split partials
+    go to a fixed 16 MiB array inside the library instead of a workspace.
+    Concurrent calls on one GPU share that array and must not overlap."""
+    _check(_lib.sa_sparse_attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(page_table),
+                                              max_pages, pool_pages, page_size, S_max, _ptr(seq_lens),
+                                              _ptr(topk), K, W, B, Hq, d, float(scale), _ptr(out), _ptr(lse),
+                                              _ptr(dev_status), _stream(stream)),
+           "sa_sparse_attn_decode_noalloc")
+
+
+SA_DECODE_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def sa_pool_index_keys(kI, S, D_I, block, kB, stream=None):

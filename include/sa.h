@@ -199,6 +199,42 @@ sa_status sa_sparse_attn_decode(const sa_bf16 *q, const sa_bf16 *k_cache,
                                 int *dev_status, sa_stream stream);
 
 /* ------------------------------------------------------------------------
+ * Decode without a caller workspace.  The pages have no counterpart: this is
+ * an interface convenience for callers that cannot allocate device memory --
+ * for example a plugin inside an engine that has reserved the GPU's memory for
+ * its own KV-cache pool and passes plugins only inputs and outputs, or a
+ * latency-critical loop where cudaMalloc / cudaFree (which may synchronise
+ * the device) must not run.
+ *
+ *   Same arguments, results and device errors as sa_sparse_attn_decode, minus
+ *   the workspace.  The split partials go to one fixed device array of
+ *   SA_DECODE_NOALLOC_SCRATCH_BYTES that every GPU loading this library holds
+ *   until the process exits.  Calls needing more than that
+ *   (sa_decode_workspace_bytes(B, Hq, d, K, W) > SA_DECODE_NOALLOC_SCRATCH_BYTES)
+ *   return SA_ERR_WORKSPACE and enqueue nothing.
+ *   All calls on a device share the array: calls that overlap on the GPU (two
+ *   streams, two host threads) race and must be serialised by the caller.
+ *   The array keeps the previous call's contents; nothing in it needs to start
+ *   at zero.  The first call on a device looks up the array's address on that
+ *   device (set-up, once per device); make that first call before any stream
+ *   capture.  This entry point never calls cudaMalloc, cudaFree or any
+ *   allocating routine.
+ * ---------------------------------------------------------------------- */
+#define SA_DECODE_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+sa_status sa_sparse_attn_decode_noalloc(const sa_bf16 *q,
+                                        const sa_bf16 *k_cache,
+                                        const sa_bf16 *v_cache,
+                                        const int32_t *page_table,
+                                        int max_pages, int pool_pages,
+                                        int page_size, int S_max,
+                                        const int32_t *seq_lens,
+                                        const int32_t *topk, int K, int W,
+                                        int B, int Hq, int d, float scale,
+                                        sa_bf16 *out, float *lse,
+                                        int *dev_status, sa_stream stream);
+
+/* ------------------------------------------------------------------------
  * Two-stage selection helpers ("What Fine-Grained Means": a coarse block pass
  * picks candidate regions cheaply, a fine pass picks top-K tokens inside
  * them; section 2 "Learned Block Routing": blocks are mean-pooled over
