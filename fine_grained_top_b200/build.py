@@ -1,6 +1,8 @@
 """Build libsa.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m fine_grained_top_b200.build [--force]
+    python fine_grained_top_b200/build.py [--force]
+
+(run as a file: importing the package itself requires the built library)
 
 Each csrc/*.cu is compiled to an object in parallel, then linked into
 fine_grained_top_b200/libsa.so with the CUDA runtime linked statically (the

@@ -13,8 +13,8 @@ from tests.conftest import ROOT
 
 @pytest.fixture(scope="module")
 def sa():
-    from fine_grained_top_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__.build()
     import fine_grained_top_b200 as m
     return m
 
