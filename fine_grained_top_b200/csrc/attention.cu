@@ -123,31 +123,27 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(AttnParams P)
     }
     const int nchunks = hi > lo ? (hi - lo + kChunk - 1) / kChunk : 0;
 
-    // ---- gather: thread -> (key tid/2, half of its 16-byte chunks)
-    auto gather = [&](int c, int buf) {
-        const int key = tid >> 1, half = tid & 1;
-        const int i = lo + c * kChunk + key;
-        int64_t row = -1;
-        if (i < hi) {
-            int s = (i < n_top) ? trow[i] : w0 + (i - n_top);
-            if (s < 0 || s > p) { report(P.dev_status, SA_DEV_INDEX); s = -1; }
-            if (s >= 0) {
-                if (DECODE && P.page_table) {
-                    const int pid = P.page_table[(int64_t)b * P.max_pages + (s >> 6)];
-                    if (pid < 0 || pid >= P.pool_pages) report(P.dev_status, SA_DEV_INDEX);
-                    else row = (int64_t)pid * 64 + (s & 63);
-                } else if (DECODE) {
-                    row = (int64_t)b * P.S_max + s;
-                } else {
-                    row = s;
-                }
-            }
+    // ---- gather: NCH consecutive lanes copy one key's row, so a warp
+    // instruction reads whole rows (full 32-byte sectors) from L2/HBM
+    auto key_row = [&](int i) -> int64_t {   // cache row of list entry i, -1 if none
+        if (i >= hi) return -1;
+        int s = (i < n_top) ? trow[i] : w0 + (i - n_top);
+        if (s < 0 || s > p) { report(P.dev_status, SA_DEV_INDEX); return -1; }
+        if (DECODE && P.page_table) {
+            const int pid = P.page_table[(int64_t)b * P.max_pages + (s >> 6)];
+            if (pid < 0 || pid >= P.pool_pages) { report(P.dev_status, SA_DEV_INDEX); return -1; }
+            return (int64_t)pid * 64 + (s & 63);
         }
-        if (half == 0) s_valid[buf][key] = row >= 0;
+        return DECODE ? (int64_t)b * P.S_max + s : (int64_t)s;
+    };
+    auto gather = [&](int c, int buf) {
         uint8_t *dk = sK + buf * TILE, *dv = sV + buf * TILE;
 #pragma unroll
-        for (int cc = 0; cc < NCH / 2; ++cc) {
-            const int ch = half * (NCH / 2) + cc;
+        for (int it = 0; it < kChunk * NCH / kAttnThreads; ++it) {
+            const int g = it * kAttnThreads + tid;
+            const int key = g / NCH, ch = g % NCH;
+            const int64_t row = key_row(lo + c * kChunk + key);
+            if (ch == 0) s_valid[buf][key] = row >= 0;
             const uint32_t off = swz<ROWB>(key, ch);
             if (row >= 0) {
                 cp_async16(dk + off, P.k + row * D + ch * 8);

@@ -60,7 +60,9 @@ struct IdxCfg {
     static constexpr int kEpiGroups = kEpiWarps / 4;
     // at least 116 KB so that exactly one persistent CTA (and one TMEM
     // allocation) lands on each SM
-    static constexpr size_t kSmemUsed = 1024 + (size_t)kStages * kStageBytes + 1024;
+    static constexpr int kGroupCols = N / kEpiGroups;                 // TMEM columns per epilogue warp
+    static constexpr size_t kStageW = (size_t)kEpiWarps * kGroupCols * 8;   // w (fp32) + n_valid per warp
+    static constexpr size_t kSmemUsed = 1024 + (size_t)kStages * kStageBytes + 1024 + kStageW;
     static constexpr size_t kSmem = kSmemUsed > 118784 ? kSmemUsed : 118784;
 };
 
@@ -98,6 +100,8 @@ __global__ void __launch_bounds__(IdxCfg<N, D_I>::kThreads, 1)
     uint64_t *drain_bar = tempty_bar + 2;           // [1]
     uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(drain_bar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_slot + 1);
+    float *w_stage = reinterpret_cast<float *>(smem + C::kStages * C::kStageBytes + 1024);
+    int *nv_stage = reinterpret_cast<int *>(w_stage + C::kEpiWarps * C::kGroupCols);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -218,11 +222,18 @@ __global__ void __launch_bounds__(IdxCfg<N, D_I>::kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue
+        // Warp (quad, grp) owns TMEM lanes quad*32.. (keys) and the tile's
+        // query group grp (C::kGroupCols columns = q_per_grp queries x H_I).
         const int ew = warp - 2;
-        const int quad = warp & 3;             // TMEM lane quadrant this warp may access
-        const int grp = ew >> 2;               // which part of the tile's queries
-        const int q_per_grp = a.QT / C::kEpiGroups > 0 ? a.QT / C::kEpiGroups : 1;
-        const int q_lo = grp * q_per_grp, q_hi = min(a.QT, q_lo + q_per_grp);
+        const int quad = warp & 3;
+        const int grp = ew >> 2;
+        constexpr int QPL = 16 / H_I;                        // queries per 16-column TMEM load
+        constexpr int NLD = C::kGroupCols / 16;             // TMEM loads per item
+        constexpr int BATCH = NLD < 4 ? NLD : 4;
+        const int q_per_grp = C::kGroupCols / H_I;
+        const int q_lo = grp * q_per_grp;
+        float *ws = w_stage + ew * C::kGroupCols;
+        int *nvs = nv_stage + ew * C::kGroupCols;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
@@ -230,34 +241,46 @@ __global__ void __launch_bounds__(IdxCfg<N, D_I>::kThreads, 1)
             decode_item(a, item, b, qt, kt);
             const int ext = tile_extent(a, b, qt, lane);
             if (kt * 128 >= ext) continue;
+            // stage this group's weights and row lengths while the MMA runs
+            const int t_base = qt * a.QT + q_lo;
+            const int nq = max(0, min(q_per_grp, a.T - t_base));
+            const int64_t row0 = (int64_t)b * a.T + t_base;
+            for (int i = lane; i < nq * H_I; i += 32)
+                ws[i] = __uint_as_float((uint32_t)a.w[row0 * H_I + i] << 16);
+            for (int i = lane; i < nq; i += 32) {
+                int nv = a.n_valid ? a.n_valid[row0 + i] : a.S - a.T + t_base + i + 1;
+                if (nv < 0 || nv > a.S) {   // never write outside the row
+                    report(a.dev_status, SA_DEV_INDEX);
+                    nv = nv < 0 ? 0 : a.S;
+                }
+                nvs[i] = nv;
+            }
+            __syncwarp();
             const bool ok = mbar_wait(&tfull_bar[acc], acc_phase, abort_flag);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
             const int s = kt * 128 + quad * 32 + lane;
-            const uint32_t t_row = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * N);
-            constexpr int QPL = 16 / H_I;   // queries per 16-column TMEM load
-            for (int q0 = q_lo; q0 < q_hi; q0 += QPL) {
-                uint32_t v[16];
-                tmem_ld_x16(t_row + (uint32_t)(q0 * H_I), v);
+            const uint32_t t_cols = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * N + grp * C::kGroupCols);
+            float *out = a.scores + row0 * a.ld + s;
+#pragma unroll
+            for (int l0 = 0; l0 < NLD; l0 += BATCH) {
+                uint32_t v[BATCH][16];
+#pragma unroll
+                for (int bb = 0; bb < BATCH; ++bb) tmem_ld_x16(t_cols + (uint32_t)((l0 + bb) * 16), v[bb]);
                 tmem_ld_wait();
 #pragma unroll
-                for (int qq = 0; qq < QPL; ++qq) {
-                    const int t = qt * a.QT + q0 + qq;
-                    if (q0 + qq >= q_hi || t >= a.T) continue;
-                    const int64_t rowi = (int64_t)b * a.T + t;
-                    int nv = a.n_valid ? a.n_valid[rowi] : a.S - a.T + t + 1;
-                    if (nv < 0 || nv > a.S) {   // never write outside the row
-                        if (kt == 0 && quad == 0 && lane == 0) report(a.dev_status, SA_DEV_INDEX);
-                        nv = nv < 0 ? 0 : a.S;
-                    }
-                    const uint16_t *wr = a.w + rowi * H_I;
-                    float sc = 0.f;
+                for (int bb = 0; bb < BATCH; ++bb) {
 #pragma unroll
-                    for (int j = 0; j < H_I; ++j) {
-                        const float wj = __uint_as_float((uint32_t)__ldg(wr + j) << 16);
-                        sc = fmaf(wj, fmaxf(__uint_as_float(v[qq * H_I + j]), 0.f), sc);
+                    for (int qq = 0; qq < QPL; ++qq) {
+                        const int q = (l0 + bb) * QPL + qq;
+                        if (q < nq) {
+                            float sc = 0.f;
+#pragma unroll
+                            for (int j = 0; j < H_I; ++j)
+                                sc = fmaf(ws[q * H_I + j], fmaxf(__uint_as_float(v[bb][qq * H_I + j]), 0.f), sc);
+                            if (s < nvs[q]) out[(int64_t)q * a.ld] = sc;
+                        }
                     }
-                    if (s < nv) a.scores[rowi * a.ld + s] = sc;
                 }
             }
             tc_fence_before();

@@ -6,14 +6,17 @@
 // scores ranked by lower position, emitted in ascending position order.
 //
 // Design (sm_100a):
-//   * one row per thread-block cluster of G = 1..8 CTAs; CTA c of the cluster
-//     owns a contiguous chunk of the row, loaded once from HBM with 16-byte
-//     vector loads into shared memory as order-preserving uint32 keys;
-//   * exact radix select over the keys, 4 passes of 8 bits: per-CTA
-//     histograms (warp-aggregated shared atomics via match.any), summed over
-//     the cluster through distributed shared memory (no global workspace);
-//   * after the passes the K-th key tau is known exactly, together with how
-//     many keys equal to tau must be taken (the lowest-positioned ones);
+//   * one row per thread-block cluster of G = 1..16 CTAs; CTA c of the
+//     cluster owns a contiguous chunk of the row, loaded once from HBM with
+//     16-byte vector loads into shared memory as order-preserving uint32 keys;
+//   * exact radix select over the keys in three passes of 12, 10 and 10 bits.
+//     The first histogram is built while the chunk is loaded; the later
+//     passes only count keys that match the prefix chosen so far.  Per-CTA
+//     histograms are summed over the cluster through distributed shared
+//     memory (no global workspace).  When the threshold bin is taken whole,
+//     the remaining passes are skipped;
+//   * the K-th key tau (to the resolved precision) is then known, together
+//     with how many keys equal to it must be taken (the lowest-positioned);
 //   * ordered compaction: warp ballots count "> tau" and "== tau" keys in
 //     column order, a scan over warps and over the cluster's CTAs gives every
 //     kept key its output slot, so the output comes out ascending.
@@ -25,19 +28,82 @@ namespace sa {
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kTopkChunkTarget = 16384;   // columns per CTA before adding CTAs
-constexpr int kTopkMaxChunk = 49152;      // 192 KB of keys per CTA
-constexpr int kTopkMaxCluster = 8;
+constexpr int kTopkMaxChunk = 32768;      // 128 KB of keys per CTA
+constexpr int kTopkMaxCluster = 16;
+constexpr int kBinsA = 4096;              // first pass: top 12 bits
 
 int topk_max_row_len() { return kTopkMaxChunk * kTopkMaxCluster; }
 
+// Sum the CTAs' histograms (G > 1) and find the bin holding the need-th
+// largest key.  Every thread returns (digit, count above it, count in it).
+template <int G, int BINS>
+__device__ __forceinline__ void find_threshold(const uint32_t *hl, uint32_t *hsum, uint32_t need,
+                                               uint32_t *scan_tmp, uint32_t *sel, int tid) {
+    constexpr int PER = BINS / kTopkThreads;   // bins per thread (8 or 2)
+    const int lane = tid & 31, warp = tid >> 5;
+    const uint32_t *h = hl;
+    if (G > 1) {
+        cluster_sync();   // every CTA's histogram is complete
+        for (int i = tid; i < BINS; i += kTopkThreads) {
+            uint32_t s = 0;
+#pragma unroll
+            for (int c = 0; c < G; ++c) s += dsmem_ld_u32(&hl[i], (uint32_t)c);
+            hsum[i] = s;
+        }
+        __syncthreads();
+        h = hsum;
+    }
+    // thread i owns bins BINS-1-PER*i .. BINS-PER*i (scanned from the top down)
+    uint32_t cnt[PER], lsum = 0;
+#pragma unroll
+    for (int k = 0; k < PER; ++k) { cnt[k] = h[BINS - 1 - PER * tid - k]; lsum += cnt[k]; }
+    uint32_t incl = lsum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    if (lane == 31) scan_tmp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t t = lane < kTopkWarps ? scan_tmp[lane] : 0u, x = t;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t v = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += v;
+        }
+        if (lane < kTopkWarps) scan_tmp[32 + lane] = x - t;   // exclusive warp offsets
+    }
+    __syncthreads();
+    const uint32_t excl = scan_tmp[32 + warp] + incl - lsum;
+    if (excl < need && need <= excl + lsum) {
+        uint32_t acc = excl;
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            if (acc + cnt[k] >= need) {
+                sel[0] = (uint32_t)(BINS - 1 - PER * tid - k);
+                sel[1] = acc;
+                sel[2] = cnt[k];
+                break;
+            }
+            acc += cnt[k];
+        }
+    }
+    __syncthreads();
+}
+
 template <int G>
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
-    extern __shared__ __align__(16) uint32_t keys[];   // [chunk]
-    __shared__ uint32_t hist_local[2][256];
-    __shared__ uint32_t hist[256];
+    // dynamic smem: keys[chunk] | hist_local[G > 1 ? 2 : 1][4096] | (G > 1) hist_sum[4096]
+    extern __shared__ __align__(16) uint32_t dsm[];
+    uint32_t *keys = dsm;
+    uint32_t *hist0 = dsm + a.chunk;
+    uint32_t *hist1 = (G > 1) ? hist0 + kBinsA : hist0;
+    uint32_t *hsum = (G > 1) ? hist1 + kBinsA : nullptr;
+    __shared__ uint32_t scan_tmp[64];
+    __shared__ uint32_t sel[3];
     __shared__ uint32_t warp_gt[kTopkWarps], warp_eq[kTopkWarps];
     __shared__ uint32_t cta_counts[2];
-    __shared__ uint32_t sel_digit, sel_above;
 
     const int r = blockIdx.x / G;
     const uint32_t rank = (G > 1) ? cluster_rank() : 0u;
@@ -77,7 +143,9 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
         return;   // uniform over the cluster: no distributed smem was touched
     }
 
-    // ---- load the chunk as order-preserving keys
+    // ---- load the chunk as order-preserving keys, counting the top 12 bits
+    for (int i = tid; i < kBinsA; i += kTopkThreads) hist0[i] = 0u;
+    __syncthreads();
     {
         const int len4 = len >> 2;   // c0 and ld are multiples of 4, base 16-byte aligned
         const float4 *src4 = reinterpret_cast<const float4 *>(row + c0);
@@ -86,72 +154,45 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
             uint4 k;
             k.x = order_key(f.x); k.y = order_key(f.y); k.z = order_key(f.z); k.w = order_key(f.w);
             reinterpret_cast<uint4 *>(keys)[i] = k;
+            atomicAdd(&hist0[k.x >> 20], 1u);
+            atomicAdd(&hist0[k.y >> 20], 1u);
+            atomicAdd(&hist0[k.z >> 20], 1u);
+            atomicAdd(&hist0[k.w >> 20], 1u);
         }
-        for (int i = (len4 << 2) + tid; i < len; i += kTopkThreads) keys[i] = order_key(row[c0 + i]);
+        for (int i = (len4 << 2) + tid; i < len; i += kTopkThreads) {
+            const uint32_t k = order_key(row[c0 + i]);
+            keys[i] = k;
+            atomicAdd(&hist0[k >> 20], 1u);
+        }
     }
+    __syncthreads();
 
-    // ---- exact radix select of the K-th largest key
-    uint32_t prefix = 0u, mask = 0u;
-    uint32_t need = (uint32_t)a.K;   // keys still to take among those matching `prefix`
-    for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
-        uint32_t *hl = hist_local[pass & 1];
-        if (tid < 256) hl[tid] = 0u;
+    uint32_t need = (uint32_t)a.K;      // keys still to take among those matching `prefix`
+    find_threshold<G, kBinsA>(hist0, hsum, need, scan_tmp, sel, tid);
+    uint32_t prefix = sel[0] << 20, mask = 0xFFF00000u;
+    need -= sel[1];
+    bool whole = sel[2] == need;        // the threshold bin is taken entirely
+    // two 10-bit refinements over the keys that match the prefix
+#pragma unroll 1
+    for (int pass = 1; pass < 3 && !whole; ++pass) {
+        const int shift = pass == 1 ? 10 : 0;
+        // Peers read this CTA's histogram of pass p only before the cluster
+        // barrier of pass p+1, so the buffer of pass p-1 is free to reuse.
+        uint32_t *hl = (pass & 1) ? hist1 : hist0;
+        for (int i = tid; i < 1024; i += kTopkThreads) hl[i] = 0u;
         __syncthreads();
-        for (int base = 0; base < len; base += kTopkThreads) {
-            const int i = base + tid;
-            uint32_t bin = 256u;   // sentinel: not counted
-            if (i < len) {
-                const uint32_t u = keys[i];
-                if ((u & mask) == prefix) bin = (u >> shift) & 255u;
-            }
-            const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-            if (bin < 256u && lane == __ffs(peers) - 1) atomicAdd(&hl[bin], (uint32_t)__popc(peers));
+        for (int i = tid; i < len; i += kTopkThreads) {
+            const uint32_t u = keys[i];
+            if ((u & mask) == prefix) atomicAdd(&hl[(u >> shift) & 1023u], 1u);
         }
         __syncthreads();
-        if (G > 1) {
-            cluster_sync();
-            if (tid < 256) {
-                uint32_t s = 0;
-#pragma unroll
-                for (int c = 0; c < G; ++c) s += dsmem_ld_u32(&hl[tid], (uint32_t)c);
-                hist[tid] = s;
-            }
-        } else if (tid < 256) {
-            hist[tid] = hl[tid];
-        }
-        __syncthreads();
-        if (warp == 0) {
-            // lane l owns bins 255-8l .. 248-8l, scanned from the top down
-            uint32_t cnt[8], lsum = 0;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) { cnt[k] = hist[255 - 8 * lane - k]; lsum += cnt[k]; }
-            uint32_t incl = lsum;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += v;
-            }
-            const uint32_t excl = incl - lsum;
-            if (excl < need && need <= incl) {
-                uint32_t acc = excl;
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    if (acc + cnt[k] >= need) {
-                        sel_digit = 255u - 8u * lane - k;
-                        sel_above = acc;
-                        break;
-                    }
-                    acc += cnt[k];
-                }
-            }
-        }
-        __syncthreads();
-        need -= sel_above;
-        prefix |= sel_digit << shift;
-        mask |= 0xFFu << shift;
+        find_threshold<G, 1024>(hl, hsum, need, scan_tmp, sel, tid);
+        prefix |= sel[0] << shift;
+        mask |= 1023u << shift;
+        need -= sel[1];
+        whole = sel[2] == need;
     }
-    const uint32_t tau = prefix;   // the K-th largest key; `need` keys equal to it are kept
+    const uint32_t tau = prefix, tmask = mask;   // keep: (u&tmask) > tau, and `need` of (u&tmask) == tau
 
     // ---- ordered compaction
     const int sub = ((len + kTopkThreads - 1) / kTopkThreads) * 32;   // per-warp span, multiple of 32
@@ -159,7 +200,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     uint32_t gt = 0, eq = 0;
     for (int i = w0 + lane; i < w0 + sub; i += 32) {
         const bool valid = i < w1;
-        const uint32_t u = valid ? keys[i] : 0u;
+        const uint32_t u = valid ? (keys[i] & tmask) : 0u;
         gt += __popc(__ballot_sync(0xffffffffu, valid && u > tau));
         eq += __popc(__ballot_sync(0xffffffffu, valid && u == tau));
     }
@@ -187,7 +228,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     const uint32_t lt = lanemask_lt();
     for (int i = w0 + lane; i < w0 + sub; i += 32) {
         const bool valid = i < w1;
-        const uint32_t u = valid ? keys[i] : 0u;
+        const uint32_t u = valid ? (keys[i] & tmask) : 0u;
         const bool is_gt = valid && u > tau, is_eq = valid && u == tau;
         const uint32_t bg = __ballot_sync(0xffffffffu, is_gt), be = __ballot_sync(0xffffffffu, is_eq);
         const uint32_t gt_before = run_gt + __popc(bg & lt), eq_before = run_eq + __popc(be & lt);
@@ -206,6 +247,8 @@ template <int G>
 static sa_status launch_topk_g(const TopkArgs &a, size_t smem, cudaStream_t st) {
     auto kern = topk_kernel<G>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return SA_ERR_CUDA;
+    if (G > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
         return SA_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.rows * G));
@@ -229,12 +272,14 @@ sa_status launch_topk(TopkArgs a, cudaStream_t st) {
     chunk = (chunk + 3) & ~3;
     if (chunk > kTopkMaxChunk) return SA_ERR_UNSUPPORTED;
     a.chunk = chunk;
-    const size_t smem = (size_t)chunk * 4 + 16;
+    const size_t hist_words = (g > 1) ? 3 * kBinsA : kBinsA;
+    const size_t smem = ((size_t)chunk + hist_words) * 4;
     switch (g) {
         case 1: return launch_topk_g<1>(a, smem, st);
         case 2: return launch_topk_g<2>(a, smem, st);
         case 4: return launch_topk_g<4>(a, smem, st);
-        default: return launch_topk_g<8>(a, smem, st);
+        case 8: return launch_topk_g<8>(a, smem, st);
+        default: return launch_topk_g<16>(a, smem, st);
     }
 }
 

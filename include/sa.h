@@ -140,8 +140,8 @@ sa_status sa_indexer_scores_candidates(const sa_bf16 *qI, const sa_bf16 *w,
  *   n_valid   [rows] or NULL (NULL: causal rows at the last `rows` of
  *             `row_len` positions, n_valid = row_len - rows + r + 1).
  *   Order-preserving keys: NaN scores are not supported; -inf sorts last.
- *   Limits: row_len <= 393216; K >= 0.
- *   Rows are split over a thread-block cluster (1..8 CTAs, distributed
+ *   Limits: row_len <= 524288; K >= 0.
+ *   Rows are split over a thread-block cluster (1..16 CTAs, distributed
  *   shared memory for the histograms); no workspace is needed.
  * ---------------------------------------------------------------------- */
 sa_status sa_topk_select(const float *scores, int64_t ld_scores, int rows,

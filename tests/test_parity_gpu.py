@@ -48,7 +48,8 @@ def _scores(rows, L, dist, rng):
 @pytest.mark.parametrize("rows,L,K,dist", [
     (37, 700, 64, "ties3"), (16, 5000, 1024, "ints"), (50, 17000, 700, "normal"),
     (3, 40000, 100, "normal"), (8, 131072, 2048, "ints"), (4, 262144, 2048, "ties3"),
-    (5, 393216, 3000, "ints"), (9, 33, 40, "normal"), (64, 1023, 64, "ints"),
+    (5, 393216, 3000, "ints"), (2, 524288, 2048, "normal"), (9, 33, 40, "normal"), (64, 1023, 64, "ints"),
+    (300, 8192, 1024, "ties3"), (33, 16384, 16000, "ties3"),
 ])
 def test_topk_matches_oracle(sa, rows, L, K, dist):
     rng = np.random.default_rng(rows * 7 + L)
