@@ -9,10 +9,12 @@ the 8K-token causal prefill (16 query heads, d=128, indexer 4 x 64, top-K 1024,
 window 128).  Each rank runs its own independent sequence (weak scaling, no
 collective on the data path).  One JSON line is printed by rank 0.
 
-Timing: per-step CUDA events on the launching stream, after W warm-up steps,
-with a 512 MB write between steps to flush the 126 MB L2 (outside the event
-brackets); the max over ranks is reported.  Per-stage events inside the step
-give each kernel's share and its roofline fraction.  `e2e` repeats the step
+Timing: the step (every C-ABI call of the path) is captured once as a CUDA
+graph and replayed W times to warm up, then K times, each replay after a
+512 MB write that flushes the 126 MB L2 and bracketed by CUDA events on the
+replay stream; the max over ranks of the summed step times is reported.  For
+each kernel's share and roofline fraction, one graph per kernel is replayed in
+step order with an event between consecutive kernels.  `e2e` repeats the step
 through the same C-ABI calls with the inputs copied from pinned host memory and
 the output copied back inside the timed region.  `cpu_baseline` times the CPU
 fp64 oracle on a bounded sample of query rows of the same workload.
@@ -268,22 +270,35 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier(device_ids=[local_rank])
         torch.cuda.synchronize()
 
-    # ---- device-resident timed steps, one event between consecutive kernels
+    # ---- device-resident timed steps.  The step -- every C-ABI call of the
+    # path -- is captured once as a CUDA graph and replayed, so host launch
+    # overhead cannot starve the GPU.  Each replay follows a 512 MB write that
+    # flushes L2 and is bracketed by CUDA events on the replay stream.
     ns = len(stage_list)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(ns + 1)] for _ in range(args.steps)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    stage_graphs = []
+    for _, fn in stage_list:   # one graph per kernel, for the per-kernel shares
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        stage_graphs.append(g)
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        graph.replay()
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     gpu_idx = vis.split(",")[local_rank] if vis else str(local_rank)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     barrier()
     with ClockSampler(gpu_idx) as clk:
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
             ev[i][0].record(stream)
-            for j, (_, fn) in enumerate(stage_list):
-                fn()
-                ev[i][j + 1].record(stream)
+            graph.replay()
+            ev[i][1].record(stream)
         barrier()
-    step_ms = [ev[i][0].elapsed_time(ev[i][-1]) for i in range(args.steps)]
-    stage_ms = [[ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(args.steps)] for j in range(ns)]
+    step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = float(sum(step_ms))
     t = torch.tensor([total_ms], dtype=torch.float64, device=device)
     if world > 1:
@@ -291,6 +306,20 @@ def run_ours(args, rank, world, local_rank):
     total_ms = float(t.item())
     ms_per_step = total_ms / args.steps
     value = case["units"] * world * args.steps / (total_ms / 1e3)
+
+    # per-kernel times: the stage graphs replayed back to back in step order,
+    # an event between consecutive kernels (not part of the reported value)
+    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(ns + 1)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        sev[i][0].record(stream)
+        for j, g in enumerate(stage_graphs):
+            g.replay()
+            sev[i][j + 1].record(stream)
+    torch.cuda.synchronize()
+    stage_ms = [[sev[i][j].elapsed_time(sev[i][j + 1]) for i in range(args.steps)] for j in range(ns)]
+    staged_ms = [sev[i][0].elapsed_time(sev[i][-1]) for i in range(args.steps)]
+    del graph, stage_graphs
 
     # ---- end to end through the C ABI with host buffers
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -324,7 +353,7 @@ def run_ours(args, rank, world, local_rank):
         sec = float(np.mean(times)) / 1e3
         w = work["stages"][name]
         stages[name] = dict(ms=round(sec * 1e3, 4),
-                            share=round(float(np.sum(times)) / max(1e-9, float(np.sum(step_ms))), 4),
+                            share=round(float(np.sum(times)) / max(1e-9, float(np.sum(staged_ms))), 4),
                             **roofline_entry(w["bound"], w["bytes"], w["flops"], sec, peaks))
     dom = max(stages, key=lambda n: stages[n]["ms"])
     roof = {k: v for k, v in stages[dom].items() if k not in ("ms", "share")}
@@ -339,7 +368,8 @@ def run_ours(args, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": args.workload, **{k: v for k, v in case["cfg"].items() if k != "kind"},
                    "parallelism": "replicas (an independent sequence per GPU)" if world > 1 else "single GPU",
-                   "l2": "flushed between steps (512 MB write outside the timed brackets)"},
+                   "l2": "flushed between steps (512 MB write outside the timed brackets)",
+                   "launch": "step replayed as a captured CUDA graph"},
         "roofline": roof, "stages": stages,
         "work": {k: v for k, v in work.items() if k != "stages"},
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": int(h2d),

@@ -16,7 +16,8 @@ from __future__ import annotations
 import ctypes
 import os
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsa.so")
+# SA_LIBRARY may name another build of the same library (e.g. a tuning variant)
+LIB_PATH = os.environ.get("SA_LIBRARY") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsa.so")
 
 SA_OK, SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_CUDA = 0, 1, 2, 3
 SA_ERR_TIMEOUT, SA_ERR_INDEX, SA_ERR_WORKSPACE = 4, 5, 6

@@ -20,6 +20,8 @@
 // and their log-sum-exp to the workspace; decode_merge_kernel combines them.
 #include <math_constants.h>
 
+#include <algorithm>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -27,7 +29,15 @@ namespace sa {
 
 constexpr int kAttnThreads = 128;
 constexpr int kChunk = 64;           // keys per pipeline stage
-constexpr int kDecodeSplit = 128;    // keys per decode CTA
+#ifndef SA_ATTN_STAGES
+#define SA_ATTN_STAGES 2
+#endif
+constexpr int kStages = SA_ATTN_STAGES;   // gathered K/V chunks in flight + 1
+constexpr int kDecodeSplit = 128;    // keys per CTA on the split-K decode path
+constexpr int kMaxDecodeCluster = 16; // CTAs per sequence on the cluster decode path
+// kernel modes: one query per CTA; decode split-K through a workspace; decode
+// with one thread-block cluster per sequence merging through shared memory
+constexpr int kPrefill = 0, kDecodeSplitK = 1, kDecodeCluster = 2;
 
 struct AttnParams {
     const uint16_t *q, *k, *v;
@@ -39,6 +49,7 @@ struct AttnParams {
     int max_pages, pool_pages, S_max;
     const int32_t *seq_lens;
     int B, n_splits;
+    int list_cap;                     // entries of the per-CTA key list in shared memory
     uint16_t *out;
     float *lse;
     float *ws_o, *ws_lse;
@@ -51,8 +62,9 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
     return (uint32_t)(r * ROWB + ((c ^ (r & 7)) << 4));
 }
 
-template <int D, int HT, bool DECODE>
+template <int D, int HT, int MODE>
 __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(AttnParams P) {
+    constexpr bool DECODE = MODE != kPrefill;
     constexpr int KSPLIT = 4 / HT;          // warps sharing one head tile
     constexpr int KPW = kChunk / KSPLIT;    // keys per warp per chunk
     constexpr int ROWB = D * 2;
@@ -63,9 +75,9 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(AttnParams P)
 
     extern __shared__ __align__(128) uint8_t sm[];
     uint8_t *sK = sm;                        // [2][64][D]
-    uint8_t *sV = sm + 2 * TILE;             // [2][64][D]
-    uint8_t *sQ = sm + 4 * TILE;             // [HT*16][D]
-    __shared__ int32_t s_valid[2][kChunk];
+    uint8_t *sV = sm + kStages * TILE;       // [kStages][64][D]
+    uint8_t *sQ = sm + 2 * kStages * TILE;   // [HT*16][D]
+    int32_t *s_rows = reinterpret_cast<int32_t *>(sQ + HT * 16 * ROWB);   // [list_cap] cache rows, -1 = none
     __shared__ int s_ntop;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -114,7 +126,11 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(AttnParams P)
     const int n_top = s_ntop;
     const int w0 = max(0, p - P.W + 1);
     const int n = (p >= 0) ? n_top + (p - w0 + 1) : 0;
-    if (DECODE) {
+    if (MODE == kDecodeCluster) {      // CTA `rank` of the cluster takes an equal slice
+        const int G = (int)cluster_size(), per = (n + G - 1) / G;
+        lo = (int)cluster_rank() * per;
+        hi = min(n, lo + per);
+    } else if (MODE == kDecodeSplitK) {
         lo = blockIdx.x * kDecodeSplit;
         hi = min(n, lo + kDecodeSplit);
     } else {
@@ -123,27 +139,38 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(AttnParams P)
     }
     const int nchunks = hi > lo ? (hi - lo + kChunk - 1) / kChunk : 0;
 
+    // ---- this CTA's key list as cache rows, built once in shared memory
+    // (entry i < n_top is a top-K position, the rest is the window)
+    const int n_list = hi > lo ? hi - lo : 0;
+    for (int j = tid; j < nchunks * kChunk; j += kAttnThreads) {
+        const int i = lo + j;
+        int32_t row = -1;
+        if (i < hi) {
+            const int s = (i < n_top) ? trow[i] : w0 + (i - n_top);
+            if (s < 0 || s > p) {
+                report(P.dev_status, SA_DEV_INDEX);
+            } else if (DECODE && P.page_table) {
+                const int pid = P.page_table[(int64_t)b * P.max_pages + (s >> 6)];
+                if (pid < 0 || pid >= P.pool_pages) report(P.dev_status, SA_DEV_INDEX);
+                else row = pid * 64 + (s & 63);
+            } else {
+                row = DECODE ? b * P.S_max + s : s;
+            }
+        }
+        s_rows[j] = row;
+    }
+    (void)n_list;
+    __syncthreads();
+
     // ---- gather: NCH consecutive lanes copy one key's row, so a warp
     // instruction reads whole rows (full 32-byte sectors) from L2/HBM
-    auto key_row = [&](int i) -> int64_t {   // cache row of list entry i, -1 if none
-        if (i >= hi) return -1;
-        int s = (i < n_top) ? trow[i] : w0 + (i - n_top);
-        if (s < 0 || s > p) { report(P.dev_status, SA_DEV_INDEX); return -1; }
-        if (DECODE && P.page_table) {
-            const int pid = P.page_table[(int64_t)b * P.max_pages + (s >> 6)];
-            if (pid < 0 || pid >= P.pool_pages) { report(P.dev_status, SA_DEV_INDEX); return -1; }
-            return (int64_t)pid * 64 + (s & 63);
-        }
-        return DECODE ? (int64_t)b * P.S_max + s : (int64_t)s;
-    };
     auto gather = [&](int c, int buf) {
         uint8_t *dk = sK + buf * TILE, *dv = sV + buf * TILE;
 #pragma unroll
         for (int it = 0; it < kChunk * NCH / kAttnThreads; ++it) {
             const int g = it * kAttnThreads + tid;
             const int key = g / NCH, ch = g % NCH;
-            const int64_t row = key_row(lo + c * kChunk + key);
-            if (ch == 0) s_valid[buf][key] = row >= 0;
+            const int64_t row = s_rows[c * kChunk + key];
             const uint32_t off = swz<ROWB>(key, ch);
             if (row >= 0) {
                 cp_async16(dk + off, P.k + row * D + ch * 8);
@@ -155,15 +182,19 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(AttnParams P)
         }
     };
 
-    // ---- Q tile (rows >= Hq are zero) with the first gather group
+    // ---- Q tile (rows >= Hq are zero), then the first gathers
     for (int idx = tid; idx < HT * 16 * NCH; idx += kAttnThreads) {
         const int r = idx / NCH, ch = idx % NCH;
         const uint32_t off = swz<ROWB>(r, ch);
         if (r < P.Hq) cp_async16(sQ + off, qrow + (int64_t)r * D + ch * 8);
         else *reinterpret_cast<uint4 *>(sQ + off) = make_uint4(0, 0, 0, 0);
     }
-    if (nchunks > 0) gather(0, 0);
-    cp_async_commit();
+    cp_async_commit();                        // group 0: Q
+#pragma unroll
+    for (int c = 0; c < kStages - 1; ++c) {   // groups 1 .. kStages-1: the first chunks
+        if (c < nchunks) gather(c, c);
+        cp_async_commit();
+    }
 
     float acc[DT][4];
 #pragma unroll
@@ -171,7 +202,7 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(AttnParams P)
     float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, l0 = 0.f, l1 = 0.f;
     uint32_t qf[D / 16][4];
 
-    cp_async_wait<0>();
+    cp_async_wait<kStages - 1>();             // Q has landed; chunks may still be in flight
     __syncthreads();
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
@@ -180,10 +211,10 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(AttnParams P)
     }
 
     for (int c = 0; c < nchunks; ++c) {
-        const int buf = c & 1;
-        if (c + 1 < nchunks) gather(c + 1, buf ^ 1);
+        const int buf = c % kStages;
+        if (c + kStages - 1 < nchunks) gather(c + kStages - 1, (c + kStages - 1) % kStages);
         cp_async_commit();
-        cp_async_wait<1>();
+        cp_async_wait<kStages - 1>();
         __syncthreads();
 
         const uint8_t *tk = sK + buf * TILE, *tv = sV + buf * TILE;
@@ -209,7 +240,7 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(AttnParams P)
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
             const int key = kbase + j * 8 + 2 * (lane & 3);
-            const bool v0 = s_valid[buf][key], v1 = s_valid[buf][key + 1];
+            const bool v0 = s_rows[c * kChunk + key] >= 0, v1 = s_rows[c * kChunk + key + 1] >= 0;
             s[j][0] = v0 ? s[j][0] * P.scale_log2 : -CUDART_INF_F;
             s[j][1] = v1 ? s[j][1] * P.scale_log2 : -CUDART_INF_F;
             s[j][2] = v0 ? s[j][2] * P.scale_log2 : -CUDART_INF_F;
@@ -264,61 +295,144 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(AttnParams P)
     }
     cp_async_wait<0>();
 
-    // ---- combine the KSPLIT warps of each head tile through shared memory
+    // ---- final softmax state of each head row (quad-reduce the row sums)
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-    __syncthreads();
-    float *red_acc = reinterpret_cast<float *>(sm);             // [4][16][D]
-    float *red_m = red_acc + 4 * 16 * D;                          // [4][16]
-    float *red_l = red_m + 4 * 16;                                // [4][16]
-    {
+    __syncthreads();   // every warp is done with the K/V tiles, which are reused below
+    // cluster path: this CTA's normalised partial output and log2-sum-exp,
+    // kept in shared memory (after the reduction area) for the other CTAs
+    float *part_o = reinterpret_cast<float *>(sm + 4 * 16 * D * 4 + 4 * 4 * 16 * 4);   // [HT*16][D]
+    float *part_lse = part_o + HT * 16 * D;                                             // [HT*16]
+    // write row h's normalised output at dims (col, col+1) and, once, its lse
+    auto emit2 = [&](int h, int col, float o0, float o1, bool with_lse, float lse2) {
+        if (h >= P.Hq) return;
+        if (MODE == kDecodeCluster) {
+            *reinterpret_cast<float2 *>(&part_o[h * D + col]) = make_float2(o0, o1);
+            if (with_lse) part_lse[h] = lse2;
+        } else if (MODE == kDecodeSplitK) {
+            const int64_t slot = ((int64_t)b * P.n_splits + blockIdx.x) * P.Hq + h;
+            *reinterpret_cast<float2 *>(&P.ws_o[slot * D + col]) = make_float2(o0, o1);
+            if (with_lse) P.ws_lse[slot] = lse2;
+        } else {
+            const int64_t orow = (int64_t)b * P.Hq + h;
+            *reinterpret_cast<uint32_t *>(&P.out[orow * D + col]) = pack_bf16(o0, o1);
+            if (with_lse && P.lse) P.lse[orow] = lse2 * 0.69314718055994531f;
+        }
+    };
+    if (KSPLIT == 1) {
+        // this warp alone holds its 16 heads: normalise in registers
+        const int g = lane >> 2;
+        const float inv0 = l0 > 0.f ? 1.f / l0 : 0.f, inv1 = l1 > 0.f ? 1.f / l1 : 0.f;
+        const float lse0 = l0 > 0.f ? m0 + __log2f(l0) : -CUDART_INF_F;
+        const float lse1 = l1 > 0.f ? m1 + __log2f(l1) : -CUDART_INF_F;
+#pragma unroll
+        for (int j = 0; j < DT; ++j) {
+            const int col = j * 8 + 2 * (lane & 3);
+            emit2(ht * 16 + g, col, acc[j][0] * inv0, acc[j][1] * inv0, j == 0 && (lane & 3) == 0, lse0);
+            emit2(ht * 16 + g + 8, col, acc[j][2] * inv1, acc[j][3] * inv1, j == 0 && (lane & 3) == 0, lse1);
+        }
+    } else {
+        // KSPLIT warps hold partial states of the same heads: combine them in
+        // shared memory with per-row weights computed once
+        float *red_acc = reinterpret_cast<float *>(sm);   // [4 warps][16][D]
+        float *red_m = red_acc + 4 * 16 * D;               // [4][16]
+        float *red_l = red_m + 4 * 16;                     // [4][16]
+        float *row_w = red_l + 4 * 16;                     // [HT*16][KSPLIT] merge weights / L
+        float *row_lse = row_w + 4 * 16;                   // [HT*16]
         const int g = lane >> 2;
         float *ra = red_acc + warp * 16 * D;
 #pragma unroll
         for (int j = 0; j < DT; ++j) {
             const int col = j * 8 + 2 * (lane & 3);
-            ra[g * D + col] = acc[j][0];
-            ra[g * D + col + 1] = acc[j][1];
-            ra[(g + 8) * D + col] = acc[j][2];
-            ra[(g + 8) * D + col + 1] = acc[j][3];
+            *reinterpret_cast<float2 *>(&ra[g * D + col]) = make_float2(acc[j][0], acc[j][1]);
+            *reinterpret_cast<float2 *>(&ra[(g + 8) * D + col]) = make_float2(acc[j][2], acc[j][3]);
         }
         if ((lane & 3) == 0) {
             red_m[warp * 16 + g] = m0; red_m[warp * 16 + g + 8] = m1;
             red_l[warp * 16 + g] = l0; red_l[warp * 16 + g + 8] = l1;
         }
+        __syncthreads();
+        if (tid < HT * 16) {
+            const int rt = tid >> 4, rr = tid & 15;
+            float mstar = -CUDART_INF_F;
+#pragma unroll
+            for (int k2 = 0; k2 < KSPLIT; ++k2) mstar = fmaxf(mstar, red_m[(rt * KSPLIT + k2) * 16 + rr]);
+            const float mb = (mstar == -CUDART_INF_F) ? 0.f : mstar;
+            float f[KSPLIT], L = 0.f;
+#pragma unroll
+            for (int k2 = 0; k2 < KSPLIT; ++k2) {
+                f[k2] = exp2f(red_m[(rt * KSPLIT + k2) * 16 + rr] - mb);
+                L += red_l[(rt * KSPLIT + k2) * 16 + rr] * f[k2];
+            }
+            const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+            for (int k2 = 0; k2 < KSPLIT; ++k2) row_w[tid * KSPLIT + k2] = f[k2] * inv;
+            row_lse[tid] = L > 0.f ? mb + __log2f(L) : -CUDART_INF_F;
+        }
+        __syncthreads();
+        for (int idx = tid; idx < HT * 16 * D / 2; idx += kAttnThreads) {
+            const int r = idx / (D / 2), col = 2 * (idx % (D / 2));
+            const int rt = r >> 4, rr = r & 15;
+            float o0 = 0.f, o1 = 0.f;
+#pragma unroll
+            for (int k2 = 0; k2 < KSPLIT; ++k2) {
+                const float wgt = row_w[r * KSPLIT + k2];
+                const float2 v = *reinterpret_cast<const float2 *>(&red_acc[((rt * KSPLIT + k2) * 16 + rr) * D + col]);
+                o0 = fmaf(wgt, v.x, o0);
+                o1 = fmaf(wgt, v.y, o1);
+            }
+            emit2(r, col, o0, o1, col == 0, row_lse[r]);
+        }
     }
-    __syncthreads();
-    for (int idx = tid; idx < HT * 16 * D; idx += kAttnThreads) {
-        const int r = idx / D, dim = idx % D;
-        const int h = r;   // head index (row of the Q tile)
-        if (h >= P.Hq) continue;
-        const int rt = r >> 4, rr = r & 15;
-        float mstar = -CUDART_INF_F;
-#pragma unroll
-        for (int k2 = 0; k2 < KSPLIT; ++k2) mstar = fmaxf(mstar, red_m[(rt * KSPLIT + k2) * 16 + rr]);
-        const float mb = (mstar == -CUDART_INF_F) ? 0.f : mstar;
-        float L = 0.f, o = 0.f;
-#pragma unroll
-        for (int k2 = 0; k2 < KSPLIT; ++k2) {
-            const int wv = rt * KSPLIT + k2;
-            const float f = exp2f(red_m[wv * 16 + rr] - mb);
-            L += red_l[wv * 16 + rr] * f;
-            o += red_acc[(wv * 16 + rr) * D + dim] * f;
+    if (MODE == kDecodeCluster) {
+        // merge the G partial states of this sequence through distributed
+        // shared memory: CTA `rank` produces heads [rank*hpr, rank*hpr + hpr).
+        // The G log-sum-exps of those heads are staged locally first; the
+        // partial outputs are then read with all G loads in flight.
+        __shared__ float s_wt[kMaxDecodeCluster * 8];   // [hpr <= 8][G] weights
+        __shared__ float s_inv[8], s_lse[8];
+        cluster_sync();
+        const int G = (int)cluster_size(), rank = (int)cluster_rank();
+        const int hpr = (P.Hq + G - 1) / G;
+        if (tid < hpr * G) {
+            const int hh = tid / G, c = tid % G, h = rank * hpr + hh;
+            s_wt[hh * kMaxDecodeCluster + c] =
+                h < P.Hq ? __uint_as_float(dsmem_ld_u32(&part_lse[h], (uint32_t)c)) : -CUDART_INF_F;
         }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-        const float lse2 = L > 0.f ? mb + __log2f(L) : -CUDART_INF_F;   // log2 domain
-        if (DECODE) {
-            const int64_t slot = ((int64_t)b * P.n_splits + blockIdx.x) * P.Hq + h;
-            P.ws_o[slot * D + dim] = o * inv;
-            if (dim == 0) P.ws_lse[slot] = lse2;
-        } else {
+        __syncthreads();
+        if (tid < hpr) {
+            float M = -CUDART_INF_F;
+            for (int c = 0; c < G; ++c) M = fmaxf(M, s_wt[tid * kMaxDecodeCluster + c]);
+            const float mb = (M == -CUDART_INF_F) ? 0.f : M;
+            float L = 0.f;
+            for (int c = 0; c < G; ++c) {
+                const float f = exp2f(s_wt[tid * kMaxDecodeCluster + c] - mb);
+                s_wt[tid * kMaxDecodeCluster + c] = f;
+                L += f;
+            }
+            s_inv[tid] = L > 0.f ? 1.f / L : 0.f;
+            s_lse[tid] = L > 0.f ? mb + __log2f(L) : -CUDART_INF_F;
+        }
+        __syncthreads();
+        for (int idx = tid; idx < hpr * D; idx += kAttnThreads) {
+            const int hh = idx / D, h = rank * hpr + hh, dim = idx % D;
+            if (h >= P.Hq) continue;
+            float v[kMaxDecodeCluster];
+#pragma unroll
+            for (int c = 0; c < kMaxDecodeCluster; ++c)
+                v[c] = c < G ? __uint_as_float(dsmem_ld_u32(&part_o[h * D + dim], (uint32_t)c)) : 0.f;
+            float o = 0.f;
+#pragma unroll
+            for (int c = 0; c < kMaxDecodeCluster; ++c)
+                if (c < G) o += s_wt[hh * kMaxDecodeCluster + c] * v[c];
             const int64_t orow = (int64_t)b * P.Hq + h;
-            const __nv_bfloat16 ob = __float2bfloat16_rn(o * inv);
+            const __nv_bfloat16 ob = __float2bfloat16_rn(o * s_inv[hh]);
             P.out[orow * D + dim] = *reinterpret_cast<const uint16_t *>(&ob);
-            if (dim == 0 && P.lse) P.lse[orow] = lse2 * 0.69314718055994531f;
+            if (dim == 0 && P.lse) P.lse[orow] = s_lse[hh] * 0.69314718055994531f;
         }
+        cluster_sync();   // the other CTAs may still read this CTA's partials
     }
 }
 
@@ -343,28 +457,46 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(AttnParams P) {
     if (dim == 0 && P.lse) P.lse[(int64_t)b * P.Hq + h] = (L > 0.f ? mb + __log2f(L) : -CUDART_INF_F) * 0.69314718055994531f;
 }
 
-template <int D, int HT, bool DECODE>
-static sa_status launch_attn(const AttnParams &p, dim3 grid, cudaStream_t st) {
+template <int D, int HT, int MODE>
+static sa_status launch_attn(const AttnParams &p, dim3 grid, int cluster, cudaStream_t st) {
     constexpr int TILE = kChunk * D * 2;
-    const size_t smem = 4 * TILE + HT * 16 * D * 2;
-    auto kern = sparse_attn_kernel<D, HT, DECODE>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return SA_ERR_CUDA;
-    kern<<<grid, kAttnThreads, smem, st>>>(p);
-    return cuda_ok(cudaGetLastError());
+    size_t smem = 2 * kStages * TILE + HT * 16 * D * 2 + (size_t)p.list_cap * 4;
+    if (MODE == kDecodeCluster) {   // the partials live after the reduction area
+        const size_t need = 4 * 16 * D * 4 + 4 * 4 * 16 * 4 + (size_t)HT * 16 * (D + 1) * 4;
+        smem = smem > need ? smem : need;
+    }
+    auto kern = sparse_attn_kernel<D, HT, MODE>;
+    if (prepare_kernel<sparse_attn_kernel<D, HT, MODE>>(smem, cluster > 8) != cudaSuccess) return SA_ERR_CUDA;
+    if (cluster <= 1) {
+        kern<<<grid, kAttnThreads, smem, st>>>(p);
+        return cuda_ok(cudaGetLastError());
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kAttnThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_ok(cudaLaunchKernelEx(&cfg, kern, p));
 }
 
-template <bool DECODE>
-static sa_status launch_attn_shape(const AttnParams &p, int d, dim3 grid, cudaStream_t st) {
+template <int MODE>
+static sa_status launch_attn_shape(const AttnParams &p, int d, dim3 grid, int cluster, cudaStream_t st) {
     const int ht = (p.Hq + 15) / 16;
     if (d == 128) {
-        if (ht == 1) return launch_attn<128, 1, DECODE>(p, grid, st);
-        if (ht == 2) return launch_attn<128, 2, DECODE>(p, grid, st);
-        if (ht <= 4) return launch_attn<128, 4, DECODE>(p, grid, st);
+        if (ht == 1) return launch_attn<128, 1, MODE>(p, grid, cluster, st);
+        if (ht == 2) return launch_attn<128, 2, MODE>(p, grid, cluster, st);
+        if (ht <= 4) return launch_attn<128, 4, MODE>(p, grid, cluster, st);
     } else if (d == 64) {
-        if (ht == 1) return launch_attn<64, 1, DECODE>(p, grid, st);
-        if (ht == 2) return launch_attn<64, 2, DECODE>(p, grid, st);
-        if (ht <= 4) return launch_attn<64, 4, DECODE>(p, grid, st);
+        if (ht == 1) return launch_attn<64, 1, MODE>(p, grid, cluster, st);
+        if (ht == 2) return launch_attn<64, 2, MODE>(p, grid, cluster, st);
+        if (ht <= 4) return launch_attn<64, 4, MODE>(p, grid, cluster, st);
     }
     return SA_ERR_UNSUPPORTED;
 }
@@ -383,7 +515,8 @@ sa_status launch_prefill(const PrefillArgs &a, cudaStream_t st) {
     AttnParams p = base_params(a.q, a.k, a.v, a.topk, a.K, a.W, a.Hq, a.d, a.scale, a.out, a.lse, a.dev_status);
     p.T = a.T;
     p.S = a.S;
-    return launch_attn_shape<false>(p, a.d, dim3((unsigned)a.T), st);
+    p.list_cap = (a.K + a.W + kChunk - 1) / kChunk * kChunk;
+    return launch_attn_shape<kPrefill>(p, a.d, dim3((unsigned)a.T), 1, st);
 }
 
 static int decode_splits(int K, int W) { return (K + W + kDecodeSplit - 1) / kDecodeSplit; }
@@ -399,12 +532,23 @@ sa_status launch_decode(const DecodeArgs &a, cudaStream_t st) {
     AttnParams p = base_params(a.q, a.k, a.v, a.topk, a.K, a.W, a.Hq, a.d, a.scale, a.out, a.lse, a.dev_status);
     p.page_table = a.page_table; p.max_pages = a.max_pages; p.pool_pages = a.pool_pages; p.S_max = a.S_max;
     p.seq_lens = a.seq_lens; p.B = a.B;
+    // Fast path: one cluster of G CTAs per sequence, each taking about
+    // (K + W) / G keys, merged through distributed shared memory.
+    // (at least ceil(Hq / 8) CTAs: the merge gives each CTA at most 8 heads)
+    const int G = std::min(kMaxDecodeCluster, std::max({1, (a.K + a.W + kDecodeSplit - 1) / kDecodeSplit,
+                                                        (a.Hq + 7) / 8}));
+    const int per_cta = (a.K + a.W + G - 1) / G;
+    if (!a.force_split_k && per_cta <= 1024) {
+        p.list_cap = (per_cta + kChunk - 1) / kChunk * kChunk;
+        return launch_attn_shape<kDecodeCluster>(p, a.d, dim3((unsigned)G, (unsigned)a.B), G, st);
+    }
     p.n_splits = decode_splits(a.K, a.W);
+    p.list_cap = kDecodeSplit;
     const size_t slots = (size_t)a.B * p.n_splits * a.Hq;
     p.ws_o = reinterpret_cast<float *>(a.workspace);
     p.ws_lse = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(a.workspace) +
                                          (((slots * a.d * 4) + 255) & ~size_t(255)));
-    sa_status s = launch_attn_shape<true>(p, a.d, dim3((unsigned)p.n_splits, (unsigned)a.B), st);
+    sa_status s = launch_attn_shape<kDecodeSplitK>(p, a.d, dim3((unsigned)p.n_splits, (unsigned)a.B), 1, st);
     if (s != SA_OK) return s;
     const dim3 mg((unsigned)a.B, (unsigned)a.Hq);
     if (a.d == 128) decode_merge_kernel<128><<<mg, 128, 0, st>>>(p);

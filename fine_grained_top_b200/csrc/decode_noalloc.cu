@@ -75,6 +75,9 @@ extern "C" sa_status sa_sparse_attn_decode_noalloc(const sa_bf16 *q, const sa_bf
     if (page_table) {
         if (page_size != 64) return SA_ERR_UNSUPPORTED;
         if (max_pages <= 0 || pool_pages <= 0) return SA_ERR_INVALID_ARG;
+        if ((int64_t)pool_pages * 64 > INT32_MAX) return SA_ERR_UNSUPPORTED;
+    } else if ((int64_t)B * S_max > INT32_MAX) {
+        return SA_ERR_UNSUPPORTED;
     }
     if (decode_workspace_bytes(B, Hq, d, K, W) > (size_t)SA_DECODE_NOALLOC_SCRATCH_BYTES)
         return SA_ERR_WORKSPACE;   // the partial results would not fit in the fixed array
@@ -87,6 +90,7 @@ extern "C" sa_status sa_sparse_attn_decode_noalloc(const sa_bf16 *q, const sa_bf
         a.pool_pages = pool_pages; a.page_size = page_size; a.S_max = page_table ? max_pages * 64 : S_max;
         a.seq_lens = seq_lens; a.topk = topk; a.K = K; a.W = W; a.B = B; a.Hq = Hq; a.d = d; a.scale = scale;
         a.out = out; a.lse = lse; a.workspace = scratch; a.dev_status = dev_status;
+        a.force_split_k = true;   // the split-K kernels, with their partials in the fixed array
         return launch_decode(a, reinterpret_cast<cudaStream_t>(stream));
     } catch (...) {
         return SA_ERR_CUDA;

@@ -61,8 +61,7 @@ struct IdxCfg {
     // at least 116 KB so that exactly one persistent CTA (and one TMEM
     // allocation) lands on each SM
     static constexpr int kGroupCols = N / kEpiGroups;                 // TMEM columns per epilogue warp
-    static constexpr size_t kStageW = (size_t)kEpiWarps * kGroupCols * 8;   // w (fp32) + n_valid per warp
-    static constexpr size_t kSmemUsed = 1024 + (size_t)kStages * kStageBytes + 1024 + kStageW;
+    static constexpr size_t kSmemUsed = 1024 + (size_t)kStages * kStageBytes + 1024;
     static constexpr size_t kSmem = kSmemUsed > 118784 ? kSmemUsed : 118784;
 };
 
@@ -100,8 +99,6 @@ __global__ void __launch_bounds__(IdxCfg<N, D_I>::kThreads, 1)
     uint64_t *drain_bar = tempty_bar + 2;           // [1]
     uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(drain_bar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_slot + 1);
-    float *w_stage = reinterpret_cast<float *>(smem + C::kStages * C::kStageBytes + 1024);
-    int *nv_stage = reinterpret_cast<int *>(w_stage + C::kEpiWarps * C::kGroupCols);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -232,8 +229,8 @@ __global__ void __launch_bounds__(IdxCfg<N, D_I>::kThreads, 1)
         constexpr int BATCH = NLD < 4 ? NLD : 4;
         const int q_per_grp = C::kGroupCols / H_I;
         const int q_lo = grp * q_per_grp;
-        float *ws = w_stage + ew * C::kGroupCols;
-        int *nvs = nv_stage + ew * C::kGroupCols;
+        constexpr int WREGS = (C::kGroupCols + 31) / 32;
+        constexpr int NVREGS = (C::kGroupCols / H_I + 31) / 32;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
@@ -241,21 +238,32 @@ __global__ void __launch_bounds__(IdxCfg<N, D_I>::kThreads, 1)
             decode_item(a, item, b, qt, kt);
             const int ext = tile_extent(a, b, qt, lane);
             if (kt * 128 >= ext) continue;
-            // stage this group's weights and row lengths while the MMA runs
+            // fetch this group's weights and row lengths into registers (lane
+            // i holds entry i, i+32, ...) before waiting, so the loads overlap
+            // with the TMA and MMA of this item
             const int t_base = qt * a.QT + q_lo;
             const int nq = max(0, min(q_per_grp, a.T - t_base));
             const int64_t row0 = (int64_t)b * a.T + t_base;
-            for (int i = lane; i < nq * H_I; i += 32)
-                ws[i] = __uint_as_float((uint32_t)a.w[row0 * H_I + i] << 16);
-            for (int i = lane; i < nq; i += 32) {
-                int nv = a.n_valid ? a.n_valid[row0 + i] : a.S - a.T + t_base + i + 1;
-                if (nv < 0 || nv > a.S) {   // never write outside the row
-                    report(a.dev_status, SA_DEV_INDEX);
-                    nv = nv < 0 ? 0 : a.S;
-                }
-                nvs[i] = nv;
+            float wr[WREGS];
+            int nvr[NVREGS];
+#pragma unroll
+            for (int k = 0; k < WREGS; ++k) {
+                const int i = lane + 32 * k;
+                wr[k] = (i < nq * H_I) ? __uint_as_float((uint32_t)__ldg(a.w + row0 * H_I + i) << 16) : 0.f;
             }
-            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < NVREGS; ++k) {
+                const int i = lane + 32 * k;
+                int nv = 0;
+                if (i < nq) {
+                    nv = a.n_valid ? __ldg(a.n_valid + row0 + i) : a.S - a.T + t_base + i + 1;
+                    if (nv < 0 || nv > a.S) {   // never write outside the row
+                        report(a.dev_status, SA_DEV_INDEX);
+                        nv = nv < 0 ? 0 : a.S;
+                    }
+                }
+                nvr[k] = nv;
+            }
             const bool ok = mbar_wait(&tfull_bar[acc], acc_phase, abort_flag);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
@@ -276,9 +284,13 @@ __global__ void __launch_bounds__(IdxCfg<N, D_I>::kThreads, 1)
                         if (q < nq) {
                             float sc = 0.f;
 #pragma unroll
-                            for (int j = 0; j < H_I; ++j)
-                                sc = fmaf(ws[q * H_I + j], fmaxf(__uint_as_float(v[bb][qq * H_I + j]), 0.f), sc);
-                            if (s < nvs[q]) out[(int64_t)q * a.ld] = sc;
+                            for (int j = 0; j < H_I; ++j) {
+                                const int e = q * H_I + j;
+                                const float wj = __shfl_sync(0xffffffffu, wr[e >> 5], e & 31);
+                                sc = fmaf(wj, fmaxf(__uint_as_float(v[bb][qq * H_I + j]), 0.f), sc);
+                            }
+                            const int nv = __shfl_sync(0xffffffffu, nvr[q >> 5], q & 31);
+                            if (s < nv) out[(int64_t)q * a.ld] = sc;
                         }
                     }
                 }
@@ -347,8 +359,7 @@ static sa_status launch_tc(const IndexerArgs &a, cudaStream_t st) {
     if (!make_map(&mq, a.qI, (uint64_t)a.B * a.T * H_I, D_I, N)) return SA_ERR_CUDA;
 
     auto kern = indexer_tc_kernel<N, D_I, H_I>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem) != cudaSuccess)
-        return SA_ERR_CUDA;
+    if (prepare_kernel<indexer_tc_kernel<N, D_I, H_I>>(C::kSmem, false) != cudaSuccess) return SA_ERR_CUDA;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

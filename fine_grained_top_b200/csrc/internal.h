@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/sa.h"
 
 namespace sa {
@@ -70,6 +72,7 @@ struct DecodeArgs {
     float *lse;
     void *workspace;
     int *dev_status;
+    bool force_split_k = false;   // always take the split-K path through `workspace`
 };
 size_t decode_workspace_bytes(int B, int Hq, int d, int K, int W);
 sa_status launch_decode(const DecodeArgs &a, cudaStream_t st);
@@ -80,5 +83,35 @@ sa_status launch_expand(const int32_t *blocks, int T, int S, int keep, int block
                         int64_t ld_cand, int32_t *n_cand, int *dev_status, cudaStream_t st);
 
 inline sa_status cuda_ok(cudaError_t e) { return e == cudaSuccess ? SA_OK : SA_ERR_CUDA; }
+
+// Raise a kernel's dynamic shared-memory limit (and allow clusters wider than
+// 8 CTAs) on the current device.  The attributes are set once per device and
+// kernel; later launches skip the runtime calls.  Concurrent first calls may
+// both set the same attributes, which is harmless.
+template <auto Kern>
+cudaError_t prepare_kernel(size_t smem, bool wide_cluster) {
+    static std::atomic<unsigned> done[64];   // per device: bit 31 wide clusters, low bits smem bytes
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned st = (dev >= 0 && dev < 64) ? done[dev].load(std::memory_order_relaxed) : 0u;
+    const unsigned have_smem = st & 0x7fffffffu;
+    const bool have_wide = (st >> 31) != 0;
+    if (have_smem >= smem && (!wide_cluster || have_wide)) return cudaSuccess;
+    if (smem > have_smem) {
+        e = cudaFuncSetAttribute(Kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    if (wide_cluster && !have_wide) {
+        e = cudaFuncSetAttribute(Kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
+    if (dev >= 0 && dev < 64) {
+        const unsigned ns = (unsigned)(smem > have_smem ? smem : have_smem) |
+                            ((wide_cluster || have_wide) ? 0x80000000u : 0u);
+        done[dev].store(ns, std::memory_order_relaxed);
+    }
+    return cudaSuccess;
+}
 
 }  // namespace sa

@@ -113,6 +113,7 @@ sa_status sa_sparse_attn_prefill(const sa_bf16 *q, const sa_bf16 *k, const sa_bf
                                  int *dev_status, sa_stream stream) {
     if (K < 0 || W < 0 || T < 0 || S < 0 || T > S) return SA_ERR_INVALID_ARG;
     if (!head_dim_ok(d) || Hq < 1 || Hq > 64) return SA_ERR_UNSUPPORTED;
+    if ((int64_t)K + W > 32768) return SA_ERR_UNSUPPORTED;   // the per-query key list lives in shared memory
     if (T == 0) return SA_OK;
     if (!q || !k || !v || !out || (K > 0 && !topk)) return SA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return SA_ERR_INVALID_ARG;
@@ -142,6 +143,9 @@ sa_status sa_sparse_attn_decode(const sa_bf16 *q, const sa_bf16 *k_cache, const 
     if (page_table) {
         if (page_size != 64) return SA_ERR_UNSUPPORTED;
         if (max_pages <= 0 || pool_pages <= 0) return SA_ERR_INVALID_ARG;
+        if ((int64_t)pool_pages * 64 > INT32_MAX) return SA_ERR_UNSUPPORTED;
+    } else if ((int64_t)B * S_max > INT32_MAX) {
+        return SA_ERR_UNSUPPORTED;
     }
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SA_ERR_INVALID_ARG;
     if (workspace_bytes < decode_workspace_bytes(B, Hq, d, K, W)) return SA_ERR_WORKSPACE;

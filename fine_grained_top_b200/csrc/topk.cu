@@ -27,7 +27,10 @@ namespace sa {
 
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
-constexpr int kTopkChunkTarget = 16384;   // columns per CTA before adding CTAs
+#ifndef SA_TOPK_CHUNK
+#define SA_TOPK_CHUNK 8192
+#endif
+constexpr int kTopkChunkTarget = SA_TOPK_CHUNK;   // columns per CTA before adding CTAs
 constexpr int kTopkMaxChunk = 32768;      // 128 KB of keys per CTA
 constexpr int kTopkMaxCluster = 16;
 constexpr int kBinsA = 4096;              // first pass: top 12 bits
@@ -36,21 +39,31 @@ int topk_max_row_len() { return kTopkMaxChunk * kTopkMaxCluster; }
 
 // Sum the CTAs' histograms (G > 1) and find the bin holding the need-th
 // largest key.  Every thread returns (digit, count above it, count in it).
+// The cluster sum is a reduce-scatter plus all-gather over distributed shared
+// memory: CTA r adds up bin slice r from every CTA (all G loads in flight at
+// once) and stores the sums into slice r of every CTA's `hsum`.
 template <int G, int BINS>
-__device__ __forceinline__ void find_threshold(const uint32_t *hl, uint32_t *hsum, uint32_t need,
+__device__ __forceinline__ void find_threshold(uint32_t *hl, uint32_t *hsum, uint32_t need,
                                                uint32_t *scan_tmp, uint32_t *sel, int tid) {
     constexpr int PER = BINS / kTopkThreads;   // bins per thread (8 or 2)
     const int lane = tid & 31, warp = tid >> 5;
     const uint32_t *h = hl;
     if (G > 1) {
+        constexpr int SLICE = BINS / G;
+        const uint32_t rank = cluster_rank();
         cluster_sync();   // every CTA's histogram is complete
-        for (int i = tid; i < BINS; i += kTopkThreads) {
+        for (int i = tid; i < SLICE; i += kTopkThreads) {
+            const int bin = (int)rank * SLICE + i;
+            uint32_t v[G];
+#pragma unroll
+            for (int c = 0; c < G; ++c) v[c] = dsmem_ld_u32(&hl[bin], (uint32_t)c);
             uint32_t s = 0;
 #pragma unroll
-            for (int c = 0; c < G; ++c) s += dsmem_ld_u32(&hl[i], (uint32_t)c);
-            hsum[i] = s;
+            for (int c = 0; c < G; ++c) s += v[c];
+#pragma unroll
+            for (int c = 0; c < G; ++c) dsmem_st_u32(&hsum[bin], (uint32_t)c, s);
         }
-        __syncthreads();
+        cluster_sync();   // every slice has reached every CTA
         h = hsum;
     }
     // thread i owns bins BINS-1-PER*i .. BINS-PER*i (scanned from the top down)
@@ -94,12 +107,13 @@ __device__ __forceinline__ void find_threshold(const uint32_t *hl, uint32_t *hsu
 
 template <int G>
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
-    // dynamic smem: keys[chunk] | hist_local[G > 1 ? 2 : 1][4096] | (G > 1) hist_sum[4096]
+    // dynamic smem: keys[chunk] | hist_local[4096] | (G > 1) hist_sum[4096]
+    // (peers read this CTA's histogram of a pass only between that pass's two
+    // cluster barriers, so one local buffer serves every pass)
     extern __shared__ __align__(16) uint32_t dsm[];
     uint32_t *keys = dsm;
     uint32_t *hist0 = dsm + a.chunk;
-    uint32_t *hist1 = (G > 1) ? hist0 + kBinsA : hist0;
-    uint32_t *hsum = (G > 1) ? hist1 + kBinsA : nullptr;
+    uint32_t *hsum = (G > 1) ? hist0 + kBinsA : nullptr;
     __shared__ uint32_t scan_tmp[64];
     __shared__ uint32_t sel[3];
     __shared__ uint32_t warp_gt[kTopkWarps], warp_eq[kTopkWarps];
@@ -149,15 +163,28 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     {
         const int len4 = len >> 2;   // c0 and ld are multiples of 4, base 16-byte aligned
         const float4 *src4 = reinterpret_cast<const float4 *>(row + c0);
-        for (int i = tid; i < len4; i += kTopkThreads) {
-            const float4 f = src4[i];
-            uint4 k;
-            k.x = order_key(f.x); k.y = order_key(f.y); k.z = order_key(f.z); k.w = order_key(f.w);
-            reinterpret_cast<uint4 *>(keys)[i] = k;
-            atomicAdd(&hist0[k.x >> 20], 1u);
-            atomicAdd(&hist0[k.y >> 20], 1u);
-            atomicAdd(&hist0[k.z >> 20], 1u);
-            atomicAdd(&hist0[k.w >> 20], 1u);
+        constexpr int U = 4;         // loads in flight per thread
+        for (int base = 0; base < len4; base += U * kTopkThreads) {
+            float4 f[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = base + u * kTopkThreads + tid;
+                if (i < len4) f[u] = __ldg(src4 + i);
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = base + u * kTopkThreads + tid;
+                if (i < len4) {
+                    uint4 k;
+                    k.x = order_key(f[u].x); k.y = order_key(f[u].y);
+                    k.z = order_key(f[u].z); k.w = order_key(f[u].w);
+                    reinterpret_cast<uint4 *>(keys)[i] = k;
+                    atomicAdd(&hist0[k.x >> 20], 1u);
+                    atomicAdd(&hist0[k.y >> 20], 1u);
+                    atomicAdd(&hist0[k.z >> 20], 1u);
+                    atomicAdd(&hist0[k.w >> 20], 1u);
+                }
+            }
         }
         for (int i = (len4 << 2) + tid; i < len; i += kTopkThreads) {
             const uint32_t k = order_key(row[c0 + i]);
@@ -176,9 +203,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
 #pragma unroll 1
     for (int pass = 1; pass < 3 && !whole; ++pass) {
         const int shift = pass == 1 ? 10 : 0;
-        // Peers read this CTA's histogram of pass p only before the cluster
-        // barrier of pass p+1, so the buffer of pass p-1 is free to reuse.
-        uint32_t *hl = (pass & 1) ? hist1 : hist0;
+        uint32_t *hl = hist0;
         for (int i = tid; i < 1024; i += kTopkThreads) hl[i] = 0u;
         __syncthreads();
         for (int i = tid; i < len; i += kTopkThreads) {
@@ -246,10 +271,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
 template <int G>
 static sa_status launch_topk_g(const TopkArgs &a, size_t smem, cudaStream_t st) {
     auto kern = topk_kernel<G>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return SA_ERR_CUDA;
-    if (G > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
-        return SA_ERR_CUDA;
+    if (prepare_kernel<topk_kernel<G>>(smem, G > 8) != cudaSuccess) return SA_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.rows * G));
     cfg.blockDim = dim3(kTopkThreads);
@@ -272,7 +294,7 @@ sa_status launch_topk(TopkArgs a, cudaStream_t st) {
     chunk = (chunk + 3) & ~3;
     if (chunk > kTopkMaxChunk) return SA_ERR_UNSUPPORTED;
     a.chunk = chunk;
-    const size_t hist_words = (g > 1) ? 3 * kBinsA : kBinsA;
+    const size_t hist_words = (g > 1) ? 2 * kBinsA : kBinsA;
     const size_t smem = ((size_t)chunk + hist_words) * 4;
     switch (g) {
         case 1: return launch_topk_g<1>(a, smem, st);

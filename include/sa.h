@@ -164,6 +164,7 @@ sa_status sa_topk_select(const float *scores, int64_t ld_scores, int rows,
  *   the P.V product; out is rounded to bf16 (nearest even).
  *   Device errors: a top-K entry > p sets SA_DEV_INDEX and is skipped; a row
  *   that is not strictly ascending sets SA_DEV_ORDER.
+ *   Limit: K + W <= 32768 (each query's key list is held in shared memory). 
  * ---------------------------------------------------------------------- */
 sa_status sa_sparse_attn_prefill(const sa_bf16 *q, const sa_bf16 *k,
                                  const sa_bf16 *v, const int32_t *topk, int K,
@@ -183,8 +184,10 @@ sa_status sa_sparse_attn_prefill(const sa_bf16 *q, const sa_bf16 *k,
  *   (log-sum-exp).  workspace: device memory of at least
  *   sa_decode_workspace_bytes(B, Hq, d, K, W) bytes, 256-byte aligned, owned
  *   by the caller; contents on entry do not matter.
- *   Errors: SA_ERR_WORKSPACE if too small; device SA_DEV_INDEX for a bad
- *   top-K entry or page id (skipped), SA_DEV_ORDER for a non-ascending row.
+ *   Errors: SA_ERR_WORKSPACE if too small; SA_ERR_UNSUPPORTED if B * S_max
+ *   (contiguous) or pool_pages * 64 (paged) exceeds INT32_MAX rows; device
+ *   SA_DEV_INDEX for a bad top-K entry or page id (skipped), SA_DEV_ORDER for
+ *   a non-ascending row.
  * ---------------------------------------------------------------------- */
 size_t sa_decode_workspace_bytes(int B, int Hq, int d, int K, int W);
 
