@@ -20,7 +20,12 @@
 // Warp roles (persistent CTAs, one per SM):
 //   warp 0     TMA producer (one elected lane) + TMEM allocator
 //   warp 1     MMA issuer (one elected lane): tcgen05.mma kind::f16
-//   warps 2..  epilogue, two TMEM accumulators in flight (double buffer)
+//   warps 2..  epilogue teams: 2 column groups x 2 TMEM accumulators for the
+//              256-column prefill tile; 4 item groups x 8 accumulators for the
+//              16-column decode tile (several items drain at once)
+// All roles classify the CTA's items 32 at a time (one item per lane) and
+// walk the same sequence of non-empty items; the producer resolves the page
+// ids of 32 items in parallel, off the TMA issue path.
 // Shared-memory ring of STAGES {A = 128 keys, B = N query-head rows} tiles,
 // filled by TMA with the 128B (D_I = 64) or 64B (D_I = 32) swizzle that the
 // UMMA K-major descriptors expect.
@@ -51,37 +56,54 @@ struct IdxCfg {
     static constexpr int kBBytes = N * D_I * 2;
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kStages = (N == 256) ? 4 : 8;
-    static constexpr int kEpiWarps = (N == 256) ? 8 : 4;
+    // Epilogue teams: CG column groups split one item's queries; IG item
+    // groups take alternate items so that several accumulators drain at once.
+    static constexpr int kCG = (N == 256) ? 2 : 1;
+    static constexpr int kIG = (N == 256) ? 1 : 4;
+    static constexpr int kAcc = (N == 256) ? 2 : 8;           // TMEM accumulators (multiple of kIG)
+    static constexpr int kEpiWarps = 4 * kCG * kIG;
     static constexpr int kThreads = (2 + kEpiWarps) * 32;
-    static constexpr uint32_t kTmemCols = (2 * N < 32) ? 32 : 2 * N;
+    static constexpr uint32_t kTmemCols = (kAcc * N <= 32) ? 32 : (kAcc * N <= 64) ? 64 : (kAcc * N <= 128) ? 128
+                                        : (kAcc * N <= 256) ? 256 : 512;
     static constexpr uint32_t kSwizzleBytes = D_I * 2;         // 128 or 64
     static constexpr uint32_t kSbo = 8 * kSwizzleBytes;        // 8-row core group stride
     static constexpr uint32_t kLayout = (D_I == 64) ? 2 : 4;   // UMMA layout: 128B / 64B swizzle
-    static constexpr int kEpiGroups = kEpiWarps / 4;
+    static constexpr int kGroupCols = N / kCG;                 // TMEM columns per epilogue warp
+    static constexpr size_t kWStage = (size_t)kEpiWarps * kGroupCols * 8;   // w (fp32) + n_valid per warp
+    static constexpr size_t kSmemUsed = 1024 + (size_t)kStages * kStageBytes + 1024 + kWStage;
     // at least 116 KB so that exactly one persistent CTA (and one TMEM
     // allocation) lands on each SM
-    static constexpr int kGroupCols = N / kEpiGroups;                 // TMEM columns per epilogue warp
-    static constexpr size_t kSmemUsed = 1024 + (size_t)kStages * kStageBytes + 1024;
     static constexpr size_t kSmem = kSmemUsed > 118784 ? kSmemUsed : 118784;
+    static_assert(kAcc % kIG == 0, "item groups must own whole accumulators");
 };
 
-// Largest n_valid among the tile's queries (the tile's key extent).  Called
-// by a full warp; every role evaluates it identically to skip empty tiles.
-__device__ __forceinline__ int tile_extent(const IdxKernelArgs &a, int b, int qt, int lane) {
-    const int t0 = qt * a.QT, t1 = min(t0 + a.QT, a.T);
-    if (a.n_valid == nullptr) return a.S - a.T + t1;   // causal: last query's count
-    int m = 0;
-    for (int t = t0 + lane; t < t1; t += 32) m = max(m, a.n_valid[(int64_t)b * a.T + t]);
-    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-    return min(m, a.S);
-}
+// One work item: query tile qt of batch b against key tile kt (128 keys).
+struct ItemInfo {
+    int b, qt, kt, ext;   // ext: the tile's key extent (largest n_valid of its queries)
+};
 
-__device__ __forceinline__ void decode_item(const IdxKernelArgs &a, int item, int &b, int &qt, int &kt) {
+// Work of the CTA's item `i` (rectangle item blockIdx.x + i * gridDim.x),
+// evaluated by one lane.  Every role classifies items the same way, 32 at a
+// time, so all roles walk the same sequence of non-empty items.
+__device__ __forceinline__ bool item_at(const IdxKernelArgs &a, int i, ItemInfo &it) {
+    const long long item = (long long)blockIdx.x + (long long)i * gridDim.x;
+    if (item >= a.n_items) return false;
     const int per_b = a.QTN * a.KT;
-    b = item / per_b;
-    const int rem = item - b * per_b;
-    qt = rem / a.KT;
-    kt = rem - qt * a.KT;
+    it.b = (int)(item / per_b);
+    const int rem = (int)(item - (long long)it.b * per_b);
+    it.qt = rem / a.KT;
+    it.kt = rem - it.qt * a.KT;
+    const int t0 = it.qt * a.QT, t1 = min(t0 + a.QT, a.T);
+    int ext;
+    if (a.n_valid == nullptr) {
+        ext = a.S - a.T + t1;   // causal: the tile's last query
+    } else {
+        ext = 0;
+        for (int t = t0; t < t1; ++t) ext = max(ext, __ldg(a.n_valid + (int64_t)it.b * a.T + t));
+        ext = min(ext, a.S);
+    }
+    it.ext = ext;
+    return true;
 }
 
 template <int N, int D_I, int H_I>
@@ -94,17 +116,19 @@ __global__ void __launch_bounds__(IdxCfg<N, D_I>::kThreads, 1)
     uint8_t *stage_base = smem;
     uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + C::kStages * C::kStageBytes);
     uint64_t *empty_bar = full_bar + C::kStages;
-    uint64_t *tfull_bar = empty_bar + C::kStages;   // [2]
-    uint64_t *tempty_bar = tfull_bar + 2;           // [2]
-    uint64_t *drain_bar = tempty_bar + 2;           // [1]
+    uint64_t *tfull_bar = empty_bar + C::kStages;   // [kAcc]
+    uint64_t *tempty_bar = tfull_bar + C::kAcc;     // [kAcc]
+    uint64_t *drain_bar = tempty_bar + C::kAcc;     // [1]
     uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(drain_bar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_base_slot + 1);
+    float *w_stage = reinterpret_cast<float *>(smem + C::kStages * C::kStageBytes + 1024);
+    int *nv_stage = reinterpret_cast<int *>(w_stage + C::kEpiWarps * C::kGroupCols);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::kStages; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
-        for (int i = 0; i < 2; ++i) { mbar_init(&tfull_bar[i], 1); mbar_init(&tempty_bar[i], C::kEpiWarps); }
+        for (int i = 0; i < C::kAcc; ++i) { mbar_init(&tfull_bar[i], 1); mbar_init(&tempty_bar[i], 4 * C::kCG); }
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -125,44 +149,53 @@ __global__ void __launch_bounds__(IdxCfg<N, D_I>::kThreads, 1)
         int stage = 0;
         uint32_t phase = 0;
         int issued = 0;
-        for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
-            int b, qt, kt;
-            decode_item(a, item, b, qt, kt);
-            const int ext = tile_extent(a, b, qt, lane);
-            if (kt * 128 >= ext) continue;
-            bool ok = true;
-            if (lane == 0) {
-                ok = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag);
-                if (ok) {
-                    uint8_t *sa_ = stage_base + stage * C::kStageBytes;
-                    uint8_t *sb_ = sa_ + C::kABytes;
-                    int boxes[2] = {0, 0};
-                    int nbox = 0;
-                    for (int i = 0; i < 2; ++i) {
-                        const int s0 = kt * 128 + i * C::kBoxRows;
-                        if (s0 >= ext) break;
+        bool ok = true;
+        for (int base = 0; ok; base += 32) {
+            ItemInfo it;
+            const bool in = item_at(a, base + lane, it);
+            const bool valid = in && it.kt * 128 < it.ext;
+            // the two 64-key boxes of this lane's item: cache rows, or -1 (skip)
+            int row0 = -1, row1 = -1;
+            if (valid) {
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int s0 = it.kt * 128 + i * C::kBoxRows;
+                    int row = -1;
+                    if (s0 < it.ext) {
                         if (a.page_table) {
-                            const int pid = a.page_table[(int64_t)b * a.max_pages + (s0 >> 6)];
-                            if (pid < 0 || pid >= a.pool_pages) { report(a.dev_status, SA_DEV_INDEX); continue; }
-                            boxes[i] = pid * 64;
+                            const int pid = __ldg(a.page_table + (int64_t)it.b * a.max_pages + (s0 >> 6));
+                            if (pid < 0 || pid >= a.pool_pages) report(a.dev_status, SA_DEV_INDEX);
+                            else row = pid * 64;
                         } else {
-                            boxes[i] = b * a.S + s0;
+                            row = it.b * a.S + s0;
                         }
-                        nbox |= 1 << i;
                     }
-                    const uint32_t bytes = C::kBBytes + (uint32_t)__popc(nbox) * (C::kABytes / 2);
-                    mbar_arrive_expect_tx(&full_bar[stage], bytes);
-                    tma_load_2d(sb_, &map_q, 0, (b * a.T + qt * a.QT) * H_I, &full_bar[stage]);
-                    for (int i = 0; i < 2; ++i)
-                        if (nbox & (1 << i))
-                            tma_load_2d(sa_ + i * (C::kABytes / 2), &map_k, 0, boxes[i], &full_bar[stage]);
-                    ++issued;
+                    (i == 0 ? row0 : row1) = row;
                 }
             }
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
-            __syncwarp();
-            if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+            if (__ballot_sync(0xffffffffu, in) == 0) break;
+            uint32_t vmask = __ballot_sync(0xffffffffu, valid);
+            while (vmask) {
+                const int j = __ffs(vmask) - 1;
+                vmask &= vmask - 1;
+                const int qrow = __shfl_sync(0xffffffffu, (it.b * a.T + it.qt * a.QT) * H_I, j);
+                const int r0 = __shfl_sync(0xffffffffu, row0, j), r1 = __shfl_sync(0xffffffffu, row1, j);
+                if (lane == 0) {
+                    ok = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag);
+                    if (ok) {
+                        uint8_t *sa_ = stage_base + stage * C::kStageBytes;
+                        const uint32_t bytes = C::kBBytes + (uint32_t)((r0 >= 0) + (r1 >= 0)) * (C::kABytes / 2);
+                        mbar_arrive_expect_tx(&full_bar[stage], bytes);
+                        tma_load_2d(sa_ + C::kABytes, &map_q, 0, qrow, &full_bar[stage]);
+                        if (r0 >= 0) tma_load_2d(sa_, &map_k, 0, r0, &full_bar[stage]);
+                        if (r1 >= 0) tma_load_2d(sa_ + C::kABytes / 2, &map_k, 0, r1, &full_bar[stage]);
+                        ++issued;
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
+            }
         }
         // drain: wait (bounded) for this CTA's last loads to land before teardown
         if (lane == 0 && *abort_flag) {
@@ -179,38 +212,40 @@ __global__ void __launch_bounds__(IdxCfg<N, D_I>::kThreads, 1)
         constexpr uint32_t idesc = idesc_bf16_f32(128, N);
         int stage = 0;
         uint32_t phase = 0;
-        int acc = 0;
-        uint32_t acc_phase = 0;
-        bool any = false;
-        for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
-            int b, qt, kt;
-            decode_item(a, item, b, qt, kt);
-            const int ext = tile_extent(a, b, qt, lane);
-            if (kt * 128 >= ext) continue;
-            bool ok = true;
-            if (lane == 0) {
-                ok = mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag) &&
-                     mbar_wait(&full_bar[stage], phase, abort_flag);
-                if (ok) {
-                    tc_fence_after();
-                    const uint32_t a_addr = smem_u32(stage_base + stage * C::kStageBytes);
-                    const uint32_t b_addr = a_addr + C::kABytes;
-                    const uint32_t d_tmem = tmem_base + (uint32_t)(acc * N);
+        int c = 0;   // non-empty items so far
+        bool ok = true, any = false;
+        for (int base = 0; ok; base += 32) {
+            ItemInfo it;
+            const bool in = item_at(a, base + lane, it);
+            const bool valid = in && it.kt * 128 < it.ext;
+            if (__ballot_sync(0xffffffffu, in) == 0) break;
+            const int nvalid = __popc(__ballot_sync(0xffffffffu, valid));
+            for (int k = 0; k < nvalid; ++k, ++c) {
+                const int acc = c % C::kAcc;
+                const uint32_t acc_phase = (uint32_t)(c / C::kAcc) & 1u;
+                if (lane == 0) {
+                    ok = mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag) &&
+                         mbar_wait(&full_bar[stage], phase, abort_flag);
+                    if (ok) {
+                        tc_fence_after();
+                        const uint32_t a_addr = smem_u32(stage_base + stage * C::kStageBytes);
+                        const uint32_t b_addr = a_addr + C::kABytes;
+                        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * N);
 #pragma unroll
-                    for (int k = 0; k < D_I / 16; ++k) {
-                        const uint64_t da = smem_desc(a_addr + k * 32, C::kSbo, C::kLayout);
-                        const uint64_t db = smem_desc(b_addr + k * 32, C::kSbo, C::kLayout);
-                        tc_mma_f16(d_tmem, da, db, idesc, k > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < D_I / 16; ++kk) {
+                            const uint64_t da = smem_desc(a_addr + kk * 32, C::kSbo, C::kLayout);
+                            const uint64_t db = smem_desc(b_addr + kk * 32, C::kSbo, C::kLayout);
+                            tc_mma_f16(d_tmem, da, db, idesc, kk > 0 ? 1u : 0u);
+                        }
+                        tc_commit(&empty_bar[stage]);
+                        tc_commit(&tfull_bar[acc]);
+                        any = true;
                     }
-                    tc_commit(&empty_bar[stage]);
-                    tc_commit(&tfull_bar[acc]);
-                    any = true;
                 }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
             }
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
-            if (++stage == C::kStages) { stage = 0; phase ^= 1u; }
-            if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
         }
         if (lane == 0 && any) {   // all issued MMAs complete before TMEM is released
             tc_commit(drain_bar);
@@ -219,86 +254,113 @@ __global__ void __launch_bounds__(IdxCfg<N, D_I>::kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        // Warp (quad, grp) owns TMEM lanes quad*32.. (keys) and the tile's
-        // query group grp (C::kGroupCols columns = q_per_grp queries x H_I).
+        // Warp ew = (item group ig, column group cg, lane quadrant quad): it
+        // owns TMEM lanes quad*32.. (keys) and the columns of query group cg
+        // (kGroupCols = q_per_grp queries x H_I heads) of every kIG-th item.
         const int ew = warp - 2;
-        const int quad = warp & 3;
-        const int grp = ew >> 2;
-        constexpr int QPL = 16 / H_I;                        // queries per 16-column TMEM load
-        constexpr int NLD = C::kGroupCols / 16;             // TMEM loads per item
+        const int quad = warp & 3;               // the TMEM lane quadrant a warp may access is warp % 4
+        const int cg = (ew >> 2) % C::kCG, ig = (ew >> 2) / C::kCG;
+        constexpr int QPL = 16 / H_I;            // queries per 16-column TMEM load
+        constexpr int NLD = C::kGroupCols / 16;  // TMEM loads per item
         constexpr int BATCH = NLD < 4 ? NLD : 4;
-        const int q_per_grp = C::kGroupCols / H_I;
-        const int q_lo = grp * q_per_grp;
+        constexpr int QPG = C::kGroupCols / H_I; // queries per group
         constexpr int WREGS = (C::kGroupCols + 31) / 32;
-        constexpr int NVREGS = (C::kGroupCols / H_I + 31) / 32;
-        int acc = 0;
-        uint32_t acc_phase = 0;
-        for (int item = blockIdx.x; item < a.n_items; item += gridDim.x) {
-            int b, qt, kt;
-            decode_item(a, item, b, qt, kt);
-            const int ext = tile_extent(a, b, qt, lane);
-            if (kt * 128 >= ext) continue;
-            // fetch this group's weights and row lengths into registers (lane
-            // i holds entry i, i+32, ...) before waiting, so the loads overlap
-            // with the TMA and MMA of this item
-            const int t_base = qt * a.QT + q_lo;
-            const int nq = max(0, min(q_per_grp, a.T - t_base));
-            const int64_t row0 = (int64_t)b * a.T + t_base;
-            float wr[WREGS];
-            int nvr[NVREGS];
+        constexpr int NVREGS = (QPG + 31) / 32;
+        const int q_lo = cg * QPG;
+        float *ws = w_stage + ew * C::kGroupCols;
+        int *nvs = nv_stage + ew * C::kGroupCols;
+        int c = 0;
+        bool ok = true;
+        for (int base = 0; ok; base += 32) {
+            ItemInfo mine;
+            const bool in = item_at(a, base + lane, mine);
+            const bool valid = in && mine.kt * 128 < mine.ext;
+            if (__ballot_sync(0xffffffffu, in) == 0) break;
+            uint32_t vmask = __ballot_sync(0xffffffffu, valid);
+            for (; vmask; ++c) {
+                const int j = __ffs(vmask) - 1;
+                vmask &= vmask - 1;
+                if (c % C::kIG != ig) continue;
+                const int b = __shfl_sync(0xffffffffu, mine.b, j);
+                const int qt = __shfl_sync(0xffffffffu, mine.qt, j);
+                const int kt = __shfl_sync(0xffffffffu, mine.kt, j);
+                const int acc = c % C::kAcc;
+                const uint32_t acc_phase = (uint32_t)(c / C::kAcc) & 1u;
+                // this group's weights and row lengths, fetched before the wait
+                const int t_base = qt * a.QT + q_lo;
+                const int nq = max(0, min(QPG, a.T - t_base));
+                const int64_t row0 = (int64_t)b * a.T + t_base;
+                float wr[WREGS];
+                int nvr[NVREGS];
 #pragma unroll
-            for (int k = 0; k < WREGS; ++k) {
-                const int i = lane + 32 * k;
-                wr[k] = (i < nq * H_I) ? __uint_as_float((uint32_t)__ldg(a.w + row0 * H_I + i) << 16) : 0.f;
-            }
-#pragma unroll
-            for (int k = 0; k < NVREGS; ++k) {
-                const int i = lane + 32 * k;
-                int nv = 0;
-                if (i < nq) {
-                    nv = a.n_valid ? __ldg(a.n_valid + row0 + i) : a.S - a.T + t_base + i + 1;
-                    if (nv < 0 || nv > a.S) {   // never write outside the row
-                        report(a.dev_status, SA_DEV_INDEX);
-                        nv = nv < 0 ? 0 : a.S;
-                    }
+                for (int k = 0; k < WREGS; ++k) {
+                    const int i = lane + 32 * k;
+                    wr[k] = (i < nq * H_I) ? __uint_as_float((uint32_t)__ldg(a.w + row0 * H_I + i) << 16) : 0.f;
                 }
-                nvr[k] = nv;
-            }
-            const bool ok = mbar_wait(&tfull_bar[acc], acc_phase, abort_flag);
-            if (!__all_sync(0xffffffffu, ok)) break;
-            tc_fence_after();
-            const int s = kt * 128 + quad * 32 + lane;
-            const uint32_t t_cols = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * N + grp * C::kGroupCols);
-            float *out = a.scores + row0 * a.ld + s;
 #pragma unroll
-            for (int l0 = 0; l0 < NLD; l0 += BATCH) {
-                uint32_t v[BATCH][16];
+                for (int k = 0; k < NVREGS; ++k) {
+                    const int i = lane + 32 * k;
+                    int nv = 0;
+                    if (i < nq) {
+                        nv = a.n_valid ? __ldg(a.n_valid + row0 + i) : a.S - a.T + t_base + i + 1;
+                        if (nv < 0 || nv > a.S) {   // never write outside the row
+                            report(a.dev_status, SA_DEV_INDEX);
+                            nv = nv < 0 ? 0 : a.S;
+                        }
+                    }
+                    nvr[k] = nv;
+                }
+                ok = __all_sync(0xffffffffu, mbar_wait(&tfull_bar[acc], acc_phase, abort_flag));
+                if (!ok) break;
+                tc_fence_after();
 #pragma unroll
-                for (int bb = 0; bb < BATCH; ++bb) tmem_ld_x16(t_cols + (uint32_t)((l0 + bb) * 16), v[bb]);
-                tmem_ld_wait();
+                for (int k = 0; k < WREGS; ++k)
+                    if (lane + 32 * k < C::kGroupCols) ws[lane + 32 * k] = wr[k];
 #pragma unroll
-                for (int bb = 0; bb < BATCH; ++bb) {
+                for (int k = 0; k < NVREGS; ++k)
+                    if (lane + 32 * k < QPG) nvs[lane + 32 * k] = nvr[k];
+                __syncwarp();
+                const int s = kt * 128 + quad * 32 + lane;
+                const uint32_t t_cols = tmem_base + ((uint32_t)(quad * 32) << 16) +
+                                        (uint32_t)(acc * N + cg * C::kGroupCols);
+                float *op = a.scores + row0 * a.ld + s;
 #pragma unroll
-                    for (int qq = 0; qq < QPL; ++qq) {
-                        const int q = (l0 + bb) * QPL + qq;
-                        if (q < nq) {
-                            float sc = 0.f;
+                for (int l0 = 0; l0 < NLD; l0 += BATCH) {
+                    uint32_t v[BATCH][16];
 #pragma unroll
-                            for (int j = 0; j < H_I; ++j) {
-                                const int e = q * H_I + j;
-                                const float wj = __shfl_sync(0xffffffffu, wr[e >> 5], e & 31);
-                                sc = fmaf(wj, fmaxf(__uint_as_float(v[bb][qq * H_I + j]), 0.f), sc);
+                    for (int bb = 0; bb < BATCH; ++bb) tmem_ld_x16(t_cols + (uint32_t)((l0 + bb) * 16), v[bb]);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int bb = 0; bb < BATCH; ++bb) {
+#pragma unroll
+                        for (int qq = 0; qq < QPL; ++qq) {
+                            const int q = (l0 + bb) * QPL + qq;
+                            if (q < nq) {
+                                float wv[H_I];
+                                if constexpr (H_I >= 4) {
+#pragma unroll
+                                    for (int j4 = 0; j4 < H_I; j4 += 4) {
+                                        const float4 w4 = *reinterpret_cast<const float4 *>(ws + q * H_I + j4);
+                                        wv[j4] = w4.x; wv[j4 + 1] = w4.y; wv[j4 + 2] = w4.z; wv[j4 + 3] = w4.w;
+                                    }
+                                } else {
+#pragma unroll
+                                    for (int j1 = 0; j1 < H_I; ++j1) wv[j1] = ws[q * H_I + j1];
+                                }
+                                float sc = 0.f;
+#pragma unroll
+                                for (int j1 = 0; j1 < H_I; ++j1)
+                                    sc = fmaf(wv[j1], fmaxf(__uint_as_float(v[bb][qq * H_I + j1]), 0.f), sc);
+                                if (s < nvs[q]) *op = sc;
                             }
-                            const int nv = __shfl_sync(0xffffffffu, nvr[q >> 5], q & 31);
-                            if (s < nv) out[(int64_t)q * a.ld] = sc;
+                            op += a.ld;
                         }
                     }
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty_bar[acc]);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty_bar[acc]);
-            if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
         }
     }
 
