@@ -33,6 +33,9 @@ SIGNATURES = {
                                  _vp, _vp, _i64, _vp, _vp]),
     "sa_indexer_scores_candidates": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp,
                                             _i64, _vp, _vp]),
+    "sa_block_scores_workspace_bytes": (_sz, [_i32, _i32, _i32]),
+    "sa_indexer_scores_blocks": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _i32, _i32, _vp, _i64,
+                                        _vp, _sz, _vp, _vp]),
     "sa_topk_select": (_i32, [_vp, _i64, _i32, _i32, _vp, _vp, _i64, _i32, _vp, _vp, _vp]),
     "sa_sparse_attn_prefill": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp,
                                       _vp, _vp, _vp]),
@@ -101,6 +104,17 @@ def sa_indexer_scores_candidates(qI, w, kI, T, S, H_I, D_I, cand, ld_cand, n_can
                                              ld_cand, _ptr(n_cand), _ptr(scores), ld_scores,
                                              _ptr(dev_status), _stream(stream)),
            "sa_indexer_scores_candidates")
+
+
+def sa_block_scores_workspace_bytes(T, S, keep) -> int:
+    return int(_lib.sa_block_scores_workspace_bytes(T, S, keep))
+
+
+def sa_indexer_scores_blocks(qI, w, kI, T, S, H_I, D_I, blocks, keep, block, scores, ld_scores, workspace,
+                             workspace_bytes, dev_status=None, stream=None):
+    _check(_lib.sa_indexer_scores_blocks(_ptr(qI), _ptr(w), _ptr(kI), T, S, H_I, D_I, _ptr(blocks), keep, block,
+                                         _ptr(scores), ld_scores, _ptr(workspace), workspace_bytes,
+                                         _ptr(dev_status), _stream(stream)), "sa_indexer_scores_blocks")
 
 
 def sa_topk_select(scores, ld_scores, rows, row_len, n_valid, cand_map, ld_cand, K, topk,

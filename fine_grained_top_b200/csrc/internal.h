@@ -50,6 +50,19 @@ struct CandArgs {
 };
 sa_status launch_indexer_candidates(const CandArgs &a, cudaStream_t st);
 
+struct BlockScoreArgs {
+    const uint16_t *qI, *w, *kI;
+    int T, S, H_I, D_I;
+    const int32_t *blocks;
+    int keep;
+    float *scores;
+    int64_t ld;
+    void *workspace;
+    int *dev_status;
+};
+size_t block_scores_workspace_bytes(int T, int S, int keep);
+sa_status launch_block_scores(const BlockScoreArgs &a, cudaStream_t st);
+
 struct PrefillArgs {
     const uint16_t *q, *k, *v;
     const int32_t *topk;

@@ -92,6 +92,32 @@ sa_status sa_indexer_scores_candidates(const sa_bf16 *qI, const sa_bf16 *w, cons
     });
 }
 
+size_t sa_block_scores_workspace_bytes(int T, int S, int keep) {
+    if (T < 0 || S < 0 || keep < 0) return 0;
+    return block_scores_workspace_bytes(T, S, keep);
+}
+
+sa_status sa_indexer_scores_blocks(const sa_bf16 *qI, const sa_bf16 *w, const sa_bf16 *kI, int T, int S, int H_I,
+                                   int D_I, const int32_t *blocks, int keep, int block, float *scores,
+                                   int64_t ld_scores, void *workspace, size_t workspace_bytes, int *dev_status,
+                                   sa_stream stream) {
+    if (T < 0 || S < T || keep < 0 || block <= 0) return SA_ERR_INVALID_ARG;
+    if (!index_heads_ok(H_I) || !index_dim_ok(D_I) || block != 64 || keep > 255 || T >= (1 << 24))
+        return SA_ERR_UNSUPPORTED;
+    if (ld_scores < (int64_t)keep * block + block) return SA_ERR_INVALID_ARG;
+    if (T == 0) return SA_OK;
+    if (!qI || !w || !kI || !scores || (keep > 0 && !blocks) || !aligned16(qI) || !aligned16(kI))
+        return SA_ERR_INVALID_ARG;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SA_ERR_INVALID_ARG;
+    if (workspace_bytes < block_scores_workspace_bytes(T, S, keep)) return SA_ERR_WORKSPACE;
+    return guarded([&] {
+        BlockScoreArgs a;
+        a.qI = qI; a.w = w; a.kI = kI; a.T = T; a.S = S; a.H_I = H_I; a.D_I = D_I; a.blocks = blocks;
+        a.keep = keep; a.scores = scores; a.ld = ld_scores; a.workspace = workspace; a.dev_status = dev_status;
+        return launch_block_scores(a, cs(stream));
+    });
+}
+
 sa_status sa_topk_select(const float *scores, int64_t ld_scores, int rows, int row_len, const int32_t *n_valid,
                          const int32_t *cand_map, int64_t ld_cand, int K, int32_t *topk, int *dev_status,
                          sa_stream stream) {

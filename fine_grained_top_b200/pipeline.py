@@ -18,9 +18,9 @@ import math
 
 import torch
 
-from . import (sa_coarse_block_counts, sa_decode_workspace_bytes, sa_expand_blocks, sa_indexer_scores,
-               sa_indexer_scores_candidates, sa_pool_index_keys, sa_sparse_attn_decode,
-               sa_sparse_attn_prefill, sa_topk_select)
+from . import (sa_block_scores_workspace_bytes, sa_coarse_block_counts, sa_decode_workspace_bytes,
+               sa_expand_blocks, sa_indexer_scores, sa_indexer_scores_blocks, sa_pool_index_keys,
+               sa_sparse_attn_decode, sa_sparse_attn_prefill, sa_topk_select)
 
 
 def _ld(n: int) -> int:
@@ -55,6 +55,8 @@ class PrefillPlan:
             self.cand = torch.empty((N, self.ld_cand), dtype=i32, device=dev)
             self.n_cand = torch.empty(N, dtype=i32, device=dev)
             self.fine = torch.empty((N, self.ld_cand), dtype=f32, device=dev)
+            self.ws_bytes = sa_block_scores_workspace_bytes(N, N, keep)
+            self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=dev)
 
     def stages(self, x, stream=None):
         N, K, ds, H, D = self.N, self.K, self.dev_status, self.H_I, self.D_I
@@ -79,9 +81,9 @@ class PrefillPlan:
                                                    0, keep, self.blocks, ds, stream)),
             ("expand", lambda: sa_expand_blocks(self.blocks, N, N, keep, blk, self.cand, self.ld_cand,
                                                 self.n_cand, ds, stream)),
-            ("fine_indexer", lambda: sa_indexer_scores_candidates(x["qI"], x["w"], x["kI"], N, N, H, D,
-                                                                  self.cand, self.ld_cand, self.n_cand,
-                                                                  self.fine, self.ld_cand, ds, stream)),
+            ("fine_indexer", lambda: sa_indexer_scores_blocks(x["qI"], x["w"], x["kI"], N, N, H, D, self.blocks,
+                                                              keep, blk, self.fine, self.ld_cand, self.workspace,
+                                                              self.ws_bytes, ds, stream)),
             ("fine_topk", lambda: sa_topk_select(self.fine, self.ld_cand, N, self.ld_cand, self.n_cand,
                                                  self.cand, self.ld_cand, K, self.topk, ds, stream)),
             attn]
@@ -93,7 +95,7 @@ class PrefillPlan:
 
     def launches(self) -> int:
         """Kernels one run() enqueues."""
-        return 3 if self.block is None else 8
+        return 3 if self.block is None else 12   # fine scores: memset-free count, scan, scatter, score
 
 
 class DecodePlan:

@@ -123,6 +123,37 @@ sa_status sa_indexer_scores_candidates(const sa_bf16 *qI, const sa_bf16 *w,
                                        float *scores, int64_t ld_scores,
                                        int *dev_status, sa_stream stream);
 
+/* Fine-pass scores of the two-stage selection, computed block by block on
+ * the tensor cores: the same values and layout as sa_indexer_scores_candidates
+ * applied to the candidates that sa_expand_blocks writes for the same
+ * `blocks`, i.e. for query t at position p = S - T + t:
+ *   scores[t*ld_scores + i*block + j] = I[t, blocks[t,i']*block + j] for the
+ *   i-th valid kept block i' (j < block), then
+ *   scores[t*ld_scores + n_kept*block + j] = I[t, (p/block)*block + j] for the
+ *   query's own block, j <= p - (p/block)*block; other entries are not written.
+ * ("What Fine-Grained Means": the fine pass scores tokens inside the coarse
+ * candidates; "Sparse Attention in 2026", "The designs that shipped": the
+ * loop runs over KV blocks and gathers the queries that chose each one.)
+ * Each 64-token block's keys are read once and multiplied (tcgen05, TMEM)
+ * against the gathered indexer queries of every query that kept it.
+ *   qI [T, H_I, D_I], w [T, H_I], kI [S, D_I], blocks [T, keep] (ascending,
+ *   -1 padded, ids < p/block), block = 64, keep <= 255, T < 2^24,
+ *   ld_scores >= keep*block + block.
+ *   workspace: device memory of at least sa_block_scores_workspace_bytes(T,
+ *   S, keep) bytes, 256-byte aligned, caller-owned; it holds the per-block
+ *   query lists (contents on entry do not matter).
+ *   Errors: SA_ERR_WORKSPACE, SA_ERR_UNSUPPORTED (block != 64 ...); device
+ *   SA_DEV_INDEX for a block id >= p/block (skipped), SA_DEV_TIMEOUT. */
+size_t sa_block_scores_workspace_bytes(int T, int S, int keep);
+
+sa_status sa_indexer_scores_blocks(const sa_bf16 *qI, const sa_bf16 *w,
+                                   const sa_bf16 *kI, int T, int S, int H_I,
+                                   int D_I, const int32_t *blocks, int keep,
+                                   int block, float *scores,
+                                   int64_t ld_scores, void *workspace,
+                                   size_t workspace_bytes, int *dev_status,
+                                   sa_stream stream);
+
 /* ------------------------------------------------------------------------
  * Stage 2 -- top-K select ("Where Sparse Attention Is Actually Sparse": Top-K
  * caps how many history positions take part in exact attention)

@@ -139,6 +139,31 @@ def test_indexer_decode_contiguous_and_paged(sa):
             assert np.array_equal(got[b, :L], want[0]), (paged, b)
 
 
+@pytest.mark.parametrize("N,keep,H_I,D_I,rows", [(1000, 4, 4, 64, None), (4096, 16, 8, 64, 200),
+                                                   (700, 3, 2, 32, None), (333, 8, 1, 32, None),
+                                                   (65, 2, 4, 64, None), (4160, 64, 4, 64, 150)])
+def test_block_scores_match_oracle(sa, N, keep, H_I, D_I, rows):
+    inp = gen_prefill(N=N, Hq=1, d=64, H_I=H_I, D_I=D_I, seed=N + keep)
+    allr = np.arange(N)
+    _, blocks = oracle.two_stage(allr, inp["qI"], inp["w"], inp["kI"], 64, keep, 1)   # the oracle's kept blocks
+    ld = (keep * 64 + 64 + 3) // 4 * 4
+    sc = torch.full((N, ld), float("nan"), device="cuda")
+    nbytes = sa.sa_block_scores_workspace_bytes(N, N, keep)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    ds = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t = _to_dev(inp, ("qI", "w", "kI"))
+    sa.sa_indexer_scores_blocks(t["qI"], t["w"], t["kI"], N, N, H_I, D_I, dev(blocks.astype(np.int32)), keep, 64,
+                                sc, ld, ws, nbytes, ds)
+    got = sc.cpu().numpy()
+    assert status(ds) == 0
+    r = allr if rows is None else np.unique(np.r_[np.linspace(0, N - 1, rows).astype(int), 63, 64, N - 1])
+    full = oracle.indexer(inp["qI"][r], inp["w"][r], inp["kI"], r)
+    for i, t_ in enumerate(r):
+        kept = [b for b in blocks[t_] if b >= 0]
+        cand = [b * 64 + j for b in kept for j in range(64)] + list(range((t_ // 64) * 64, t_ + 1))
+        assert np.array_equal(got[t_, :len(cand)], full[i, cand]), t_
+
+
 # ====================================================================== attention
 @pytest.mark.parametrize("N,Hq,d,K,W", [
     (512, 4, 64, 64, 32), (700, 16, 128, 100, 17), (300, 20, 64, 50, 0), (257, 64, 128, 64, 64),
