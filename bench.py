@@ -50,6 +50,37 @@ def load_peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, src="fallback")
 
 
+# --------------------------------------------------------------------------- ncu traffic
+STAGE_SOURCE = {"indexer": "indexer.cu", "coarse_indexer": "indexer.cu", "topk": "topk.cu",
+                "coarse_topk": "topk.cu", "fine_topk": "topk.cu", "attention": "attention.cu",
+                "fine_indexer": "block_scores.cu", "expand": "two_stage.cu", "pool": "two_stage.cu",
+                "block_counts": "two_stage.cu"}
+
+
+def source_hash(cu: str) -> str:
+    """SHA-1 (12 hex digits) over a kernel's .cu file, then ptx.cuh, then internal.h."""
+    import hashlib
+    csrc = os.path.join(ROOT, "fine_grained_top_b200", "csrc")
+    m = hashlib.sha1()
+    for f in (cu, "ptx.cuh", "internal.h"):
+        m.update(open(os.path.join(csrc, f), "rb").read())
+    return m.hexdigest()[:12]
+
+
+def ncu_traffic(workload: str, stage: str):
+    """DRAM read+write bytes per launch from profiles/dram_traffic.md, if that
+    capture was taken from the kernel source that is built now; else None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    if stage not in STAGE_SOURCE or not os.path.exists(path):
+        return None
+    want = source_hash(STAGE_SOURCE[stage])
+    for line in open(path):
+        f = [x.strip() for x in line.strip().strip("|").split("|")]
+        if len(f) == 5 and f[0] == workload and f[1] == stage and f[3] == want and f[4].isdigit():
+            return int(f[4])
+    return None
+
+
 # --------------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
@@ -360,7 +391,7 @@ def run_ours(args, rank, world, local_rank):
     w = work["stages"][dom]
     roof["kernel"] = dom
     roof["algorithmic"] = w["flops"] if roof["bound"] == "tensor" else w["bytes"]
-    roof["traffic"] = None
+    roof["traffic"] = ncu_traffic(args.workload, dom)   # per launch, from a capture of this exact source
     roof["peak_src"] = peaks["src"] + " (burst figure; kernel timed alone per step)"
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
