@@ -37,8 +37,9 @@ SIGNATURES = {
     "sa_indexer_scores_blocks": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _i32, _i32, _vp, _i64,
                                         _vp, _sz, _vp, _vp]),
     "sa_topk_select": (_i32, [_vp, _i64, _i32, _i32, _vp, _vp, _i64, _i32, _vp, _vp, _vp]),
+    "sa_prefill_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
     "sa_sparse_attn_prefill": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp,
-                                      _vp, _vp, _vp]),
+                                      _vp, _vp, _sz, _vp, _vp]),
     "sa_decode_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32]),
     "sa_sparse_attn_decode": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _vp, _i32, _i32,
                                      _i32, _i32, _i32, _f32, _vp, _vp, _vp, _sz, _vp, _vp]),
@@ -47,6 +48,7 @@ SIGNATURES = {
     "sa_pool_index_keys": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp]),
     "sa_coarse_block_counts": (_i32, [_i32, _i32, _i32, _vp, _vp]),
     "sa_expand_blocks": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp, _vp]),
+    "sa_selftest_wait_timeout": (_i32, [_i32, _vp, _vp]),
 }
 
 
@@ -123,11 +125,15 @@ def sa_topk_select(scores, ld_scores, rows, row_len, n_valid, cand_map, ld_cand,
                                ld_cand, K, _ptr(topk), _ptr(dev_status), _stream(stream)), "sa_topk_select")
 
 
-def sa_sparse_attn_prefill(q, k, v, topk, K, W, T, S, Hq, d, scale, out, lse=None, dev_status=None,
-                           stream=None):
+def sa_prefill_workspace_bytes(T, S, K, W, Hq, d) -> int:
+    return int(_lib.sa_prefill_workspace_bytes(T, S, K, W, Hq, d))
+
+
+def sa_sparse_attn_prefill(q, k, v, topk, K, W, T, S, Hq, d, scale, out, lse=None, workspace=None,
+                           workspace_bytes=0, dev_status=None, stream=None):
     _check(_lib.sa_sparse_attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(topk), K, W, T, S, Hq, d,
-                                       float(scale), _ptr(out), _ptr(lse), _ptr(dev_status),
-                                       _stream(stream)), "sa_sparse_attn_prefill")
+                                       float(scale), _ptr(out), _ptr(lse), _ptr(workspace), int(workspace_bytes),
+                                       _ptr(dev_status), _stream(stream)), "sa_sparse_attn_prefill")
 
 
 def sa_decode_workspace_bytes(B, Hq, d, K, W) -> int:
@@ -179,3 +185,8 @@ def sa_dev_status_decode(word: int) -> int:
 
 def sa_version() -> int:
     return int(_lib.sa_version())
+
+
+def sa_selftest_wait_timeout(limit_us, dev_status, stream=None):
+    _check(_lib.sa_selftest_wait_timeout(int(limit_us), _ptr(dev_status), _stream(stream)),
+           "sa_selftest_wait_timeout")

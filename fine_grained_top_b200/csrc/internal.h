@@ -70,9 +70,14 @@ struct PrefillArgs {
     float scale;
     uint16_t *out;
     float *lse;
+    void *workspace;          // selection bitmap for the masked tensor-core path, or NULL
+    size_t workspace_bytes;
     int *dev_status;
 };
 sa_status launch_prefill(const PrefillArgs &a, cudaStream_t st);
+bool prefill_tc_supported(const PrefillArgs &a);
+size_t prefill_tc_workspace_bytes(int T, int S);
+sa_status launch_prefill_tc(const PrefillArgs &a, cudaStream_t st);
 
 struct DecodeArgs {
     const uint16_t *q, *k, *v;

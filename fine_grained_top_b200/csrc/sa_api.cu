@@ -134,19 +134,29 @@ sa_status sa_topk_select(const float *scores, int64_t ld_scores, int rows, int r
     });
 }
 
+size_t sa_prefill_workspace_bytes(int T, int S, int K, int W, int Hq, int d) {
+    if (T < 0 || S < 0 || K < 0 || W < 0) return 0;
+    PrefillArgs a = {};
+    a.T = T; a.S = S; a.K = K; a.W = W; a.Hq = Hq; a.d = d;
+    return prefill_tc_supported(a) ? prefill_tc_workspace_bytes(T, S) : 0;
+}
+
 sa_status sa_sparse_attn_prefill(const sa_bf16 *q, const sa_bf16 *k, const sa_bf16 *v, const int32_t *topk, int K,
                                  int W, int T, int S, int Hq, int d, float scale, sa_bf16 *out, float *lse,
-                                 int *dev_status, sa_stream stream) {
+                                 void *workspace, size_t workspace_bytes, int *dev_status, sa_stream stream) {
     if (K < 0 || W < 0 || T < 0 || S < 0 || T > S) return SA_ERR_INVALID_ARG;
     if (!head_dim_ok(d) || Hq < 1 || Hq > 64) return SA_ERR_UNSUPPORTED;
     if ((int64_t)K + W > 32768) return SA_ERR_UNSUPPORTED;   // the per-query key list lives in shared memory
     if (T == 0) return SA_OK;
     if (!q || !k || !v || !out || (K > 0 && !topk)) return SA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return SA_ERR_INVALID_ARG;
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SA_ERR_INVALID_ARG;
     return guarded([&] {
         PrefillArgs a;
         a.q = q; a.k = k; a.v = v; a.topk = topk; a.K = K; a.W = W; a.T = T; a.S = S; a.Hq = Hq; a.d = d;
         a.scale = scale; a.out = out; a.lse = lse; a.dev_status = dev_status;
+        a.workspace = workspace;
+        a.workspace_bytes = workspace_bytes;
         return launch_prefill(a, cs(stream));
     });
 }

@@ -20,7 +20,7 @@ import torch
 
 from . import (sa_block_scores_workspace_bytes, sa_coarse_block_counts, sa_decode_workspace_bytes,
                sa_expand_blocks, sa_indexer_scores, sa_indexer_scores_blocks, sa_pool_index_keys,
-               sa_sparse_attn_decode, sa_sparse_attn_prefill, sa_topk_select)
+               sa_prefill_workspace_bytes, sa_sparse_attn_decode, sa_sparse_attn_prefill, sa_topk_select)
 
 
 def _ld(n: int) -> int:
@@ -41,6 +41,9 @@ class PrefillPlan:
         self.out = torch.empty((N, Hq, d), dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty((N, Hq), dtype=f32, device=dev)
         self.dev_status = torch.zeros(1, dtype=i32, device=dev)
+        self.attn_ws_bytes = sa_prefill_workspace_bytes(N, N, K, W, Hq, d)
+        self.attn_ws = (torch.empty(self.attn_ws_bytes, dtype=torch.uint8, device=dev)
+                        if self.attn_ws_bytes else None)
         if block is None:
             self.ld = _ld(N)
             self.scores = torch.empty((N, self.ld), dtype=f32, device=dev)
@@ -62,7 +65,7 @@ class PrefillPlan:
         N, K, ds, H, D = self.N, self.K, self.dev_status, self.H_I, self.D_I
         attn = ("attention", lambda: sa_sparse_attn_prefill(
             x["q"], x["k"], x["v"], self.topk, K, self.W, N, N, self.Hq, self.d, self.scale, self.out,
-            self.lse, ds, stream))
+            self.lse, self.attn_ws, self.attn_ws_bytes, ds, stream))
         if self.block is None:
             return [
                 ("indexer", lambda: sa_indexer_scores(x["qI"], x["w"], x["kI"], None, 0, 0, 64, 1, N, N, H, D,
@@ -95,7 +98,8 @@ class PrefillPlan:
 
     def launches(self) -> int:
         """Kernels one run() enqueues."""
-        return 3 if self.block is None else 12   # fine scores: memset-free count, scan, scatter, score
+        attn = 2 if self.attn_ws is not None else 1   # (selection bitmap +) attention
+        return (2 if self.block is None else 11) + attn
 
 
 class DecodePlan:

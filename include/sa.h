@@ -193,14 +193,28 @@ sa_status sa_topk_select(const float *scores, int64_t ld_scores, int rows,
  *   sa_topk_select writes it), out [T, Hq, d] bf16, lse [T, Hq] fp32.
  *   Softmax and accumulation are fp32; probabilities are rounded to bf16 for
  *   the P.V product; out is rounded to bf16 (nearest even).
+ *   Two kernels compute this.  Gathered: each query's selected K/V rows are
+ *   gathered into shared memory (any shape; the only one when workspace is
+ *   NULL).  Masked tensor-core tiles: when every query keeps a large share of
+ *   its causal keys (S * Hq <= 256 * (K + W), Hq in {4, 8, 16, 32}, d in
+ *   {64, 128}), groups of 128 / Hq queries stream the causal K/V once in
+ *   128-key tiles through tcgen05 MMAs, masked by a per-query selection
+ *   bitmap that is built in `workspace`.  Both give the same result within
+ *   rounding.
+ *   workspace: NULL, or device memory of at least
+ *   sa_prefill_workspace_bytes(T, S, K, W, Hq, d) bytes (0 when the masked
+ *   path does not apply), 256-byte aligned, caller-owned, contents ignored.
  *   Device errors: a top-K entry > p sets SA_DEV_INDEX and is skipped; a row
  *   that is not strictly ascending sets SA_DEV_ORDER.
  *   Limit: K + W <= 32768 (each query's key list is held in shared memory). 
  * ---------------------------------------------------------------------- */
+size_t sa_prefill_workspace_bytes(int T, int S, int K, int W, int Hq, int d);
+
 sa_status sa_sparse_attn_prefill(const sa_bf16 *q, const sa_bf16 *k,
                                  const sa_bf16 *v, const int32_t *topk, int K,
                                  int W, int T, int S, int Hq, int d,
                                  float scale, sa_bf16 *out, float *lse,
+                                 void *workspace, size_t workspace_bytes,
                                  int *dev_status, sa_stream stream);
 
 /* ------------------------------------------------------------------------
@@ -296,6 +310,15 @@ sa_status sa_coarse_block_counts(int T, int S, int block, int32_t *n_blocks,
 sa_status sa_expand_blocks(const int32_t *blocks, int T, int S, int keep,
                            int block, int32_t *cand, int64_t ld_cand,
                            int32_t *n_cand, int *dev_status, sa_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Health check (no counterpart on the pages): one thread waits on a barrier
+ * that nothing arrives at, giving up after limit_us microseconds (1 .. 10^6)
+ * exactly as every pipeline wait in this library does; *dev_status then holds
+ * SA_DEV_TIMEOUT and the CUDA context stays usable.
+ * ---------------------------------------------------------------------- */
+sa_status sa_selftest_wait_timeout(int limit_us, int *dev_status,
+                                   sa_stream stream);
 
 #ifdef __cplusplus
 }

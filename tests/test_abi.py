@@ -85,12 +85,15 @@ def test_indexer_argument_checks(sa):
 
 def test_attention_argument_checks(sa):
     f = sa._lib.sa_sparse_attn_prefill
-    assert f(P, P, P, P, 4, 2, 8, 8, 16, 96, 0.1, P, N0, N0, N0) == sa.SA_ERR_UNSUPPORTED   # d = 96
-    assert f(P, P, P, P, 4, 2, 8, 8, 65, 128, 0.1, P, N0, N0, N0) == sa.SA_ERR_UNSUPPORTED  # Hq > 64
-    assert f(P, P, P, P, 4, 2, 9, 8, 16, 128, 0.1, P, N0, N0, N0) == sa.SA_ERR_INVALID_ARG  # T > S
-    assert f(P, P, P, N0, 4, 2, 8, 8, 16, 128, 0.1, P, N0, N0, N0) == sa.SA_ERR_INVALID_ARG  # NULL topk
-    assert f(P, P, P, P, -1, 2, 8, 8, 16, 128, 0.1, P, N0, N0, N0) == sa.SA_ERR_INVALID_ARG
-    assert f(P, P, P, P, 4, 2, 0, 8, 16, 128, 0.1, P, N0, N0, N0) == sa.SA_OK
+    assert f(P, P, P, P, 4, 2, 8, 8, 16, 96, 0.1, P, N0, N0, 0, N0, N0) == sa.SA_ERR_UNSUPPORTED   # d = 96
+    assert f(P, P, P, P, 4, 2, 8, 8, 65, 128, 0.1, P, N0, N0, 0, N0, N0) == sa.SA_ERR_UNSUPPORTED  # Hq > 64
+    assert f(P, P, P, P, 4, 2, 9, 8, 16, 128, 0.1, P, N0, N0, 0, N0, N0) == sa.SA_ERR_INVALID_ARG  # T > S
+    assert f(P, P, P, N0, 4, 2, 8, 8, 16, 128, 0.1, P, N0, N0, 0, N0, N0) == sa.SA_ERR_INVALID_ARG  # NULL topk
+    assert f(P, P, P, P, -1, 2, 8, 8, 16, 128, 0.1, P, N0, N0, 0, N0, N0) == sa.SA_ERR_INVALID_ARG
+    assert f(P, P, P, P, 4, 2, 8, 8, 16, 128, 0.1, P, N0, P, 1024, N0, N0) == sa.SA_ERR_INVALID_ARG  # ws align
+    assert sa.sa_prefill_workspace_bytes(8192, 8192, 1024, 128, 16, 128) == 8192 * 256 * 4
+    assert sa.sa_prefill_workspace_bytes(65536, 65536, 2048, 512, 16, 128) == 0       # sparse: gathered path
+    assert f(P, P, P, P, 4, 2, 0, 8, 16, 128, 0.1, P, N0, N0, 0, N0, N0) == sa.SA_OK
     g = sa._lib.sa_sparse_attn_decode
     need = sa.sa_decode_workspace_bytes(8, 64, 128, 2048, 512)
     assert need > 8 * 64 * 128 * 4
@@ -109,3 +112,9 @@ def test_two_stage_helper_checks(sa):
     assert lib.sa_pool_index_keys(P, 128, 48, 64, P, N0) == sa.SA_ERR_UNSUPPORTED
     assert lib.sa_pool_index_keys(P, 63, 64, 64, P, N0) == sa.SA_OK                         # no full block
     assert lib.sa_coarse_block_counts(9, 8, 64, P, N0) == sa.SA_ERR_INVALID_ARG
+
+
+def test_selftest_argument_checks(sa):
+    lib = sa._lib
+    assert lib.sa_selftest_wait_timeout(0, P, N0) == sa.SA_ERR_INVALID_ARG
+    assert lib.sa_selftest_wait_timeout(100, N0, N0) == sa.SA_ERR_INVALID_ARG

@@ -165,11 +165,15 @@ def test_block_scores_match_oracle(sa, N, keep, H_I, D_I, rows):
 
 
 # ====================================================================== attention
+@pytest.mark.parametrize("use_ws", [False, True])
 @pytest.mark.parametrize("N,Hq,d,K,W", [
     (512, 4, 64, 64, 32), (700, 16, 128, 100, 17), (300, 20, 64, 50, 0), (257, 64, 128, 64, 64),
-    (90, 16, 128, 200, 8), (1, 16, 128, 4, 4), (200, 32, 64, 0, 5),
+    (90, 16, 128, 200, 8), (1, 16, 128, 4, 4), (200, 32, 64, 0, 5), (1000, 8, 128, 300, 40),
+    (130, 32, 64, 64, 0), (2048, 16, 128, 256, 64), (1500, 4, 128, 64, 1),
 ])
-def test_prefill_attention_given_oracle_topk(sa, N, Hq, d, K, W):
+def test_prefill_attention_given_oracle_topk(sa, N, Hq, d, K, W, use_ws):
+    # use_ws=False: the gathered kernel; True: the masked tensor-core kernel
+    # whenever the shape qualifies (sa_prefill_workspace_bytes > 0)
     inp = gen_prefill(N=N, Hq=Hq, d=d, H_I=2, D_I=32, seed=N + Hq)
     t = _to_dev(inp, ("q", "k", "v"))
     if K > 0:
@@ -181,7 +185,10 @@ def test_prefill_attention_given_oracle_topk(sa, N, Hq, d, K, W):
     out = torch.empty((N, Hq, d), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((N, Hq), dtype=torch.float32, device="cuda")
     ds = torch.zeros(1, dtype=torch.int32, device="cuda")
-    sa.sa_sparse_attn_prefill(t["q"], t["k"], t["v"], top_d, K, W, N, N, Hq, d, 1 / math.sqrt(d), out, lse, ds)
+    nb = sa.sa_prefill_workspace_bytes(N, N, K, W, Hq, d) if use_ws else 0
+    ws = torch.empty(max(nb, 1), dtype=torch.uint8, device="cuda") if nb else None
+    sa.sa_sparse_attn_prefill(t["q"], t["k"], t["v"], top_d, K, W, N, N, Hq, d, 1 / math.sqrt(d), out, lse,
+                              ws, nb, ds)
     ptr, idx = oracle.selection(top, W, np.arange(N))
     o, l = oracle.sparse_attention(inp["q"], inp["k"], inp["v"], ptr, idx, 1 / math.sqrt(d))
     assert status(ds) == 0
@@ -280,21 +287,25 @@ def test_decode_edge_lengths(sa, lengths, K, W):
 
 
 # ====================================================================== device errors
-def test_planted_bad_index_and_order_are_reported(sa):
+@pytest.mark.parametrize("use_ws", [False, True])
+def test_planted_bad_index_and_order_are_reported(sa, use_ws):
     N, Hq, d, K, W = 100, 16, 128, 8, 4
     inp = gen_prefill(N=N, Hq=Hq, d=d, H_I=2, D_I=32, seed=1)
     t = _to_dev(inp, ("q", "k", "v"))
+    nb = sa.sa_prefill_workspace_bytes(N, N, K, W, Hq, d) if use_ws else 0
+    assert nb > 0 or not use_ws
+    ws = torch.empty(max(nb, 1), dtype=torch.uint8, device="cuda") if nb else None
     top = np.tile(np.arange(K, dtype=np.int32), (N, 1))
     top[50, 3] = 99            # beyond position 50
     out = torch.empty((N, Hq, d), dtype=torch.bfloat16, device="cuda")
     ds = torch.zeros(1, dtype=torch.int32, device="cuda")
-    sa.sa_sparse_attn_prefill(t["q"], t["k"], t["v"], dev(top), K, W, N, N, Hq, d, 0.1, out, None, ds)
+    sa.sa_sparse_attn_prefill(t["q"], t["k"], t["v"], dev(top), K, W, N, N, Hq, d, 0.1, out, None, ws, nb, ds)
     assert status(ds) & sa.SA_DEV_INDEX
     assert torch.isfinite(out.float()).all()
     top2 = np.tile(np.arange(K, dtype=np.int32), (N, 1))
     top2[60, 2], top2[60, 3] = 5, 4   # not ascending
     ds.zero_()
-    sa.sa_sparse_attn_prefill(t["q"], t["k"], t["v"], dev(top2), K, W, N, N, Hq, d, 0.1, out, None, ds)
+    sa.sa_sparse_attn_prefill(t["q"], t["k"], t["v"], dev(top2), K, W, N, N, Hq, d, 0.1, out, None, ws, nb, ds)
     assert status(ds) & sa.SA_DEV_ORDER
 
 
@@ -308,3 +319,16 @@ def test_planted_bad_page_is_reported(sa):
     plan.run(t["q"], t["k"], t["v"], t["qI"], t["w"], t["kI"], dev(inp["lengths"]), dev(inp["page_table"]))
     assert status(plan.dev_status) & sa.SA_DEV_INDEX
     assert torch.isfinite(plan.out.float()).all()
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(sa):
+    # a wait on a barrier that nothing arrives at gives up after 20 ms and
+    # reports SA_DEV_TIMEOUT; the context keeps working afterwards
+    ds = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sa.sa_selftest_wait_timeout(20000, ds)
+    assert status(ds) == sa.SA_DEV_TIMEOUT
+    assert sa.sa_dev_status_decode(status(ds)) == sa.SA_ERR_TIMEOUT
+    sc = torch.arange(64, dtype=torch.float32, device="cuda").reshape(1, 64)
+    out = torch.empty((1, 4), dtype=torch.int32, device="cuda")
+    sa.sa_topk_select(sc, 64, 1, 64, None, None, 0, 4, out)
+    assert out.cpu().tolist() == [[60, 61, 62, 63]]
