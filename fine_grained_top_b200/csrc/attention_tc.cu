@@ -11,22 +11,26 @@
 // for a group of queries.  This kernel takes GQ = 128 / Hq consecutive queries
 // (M = GQ x Hq = 128 query-head rows) and walks the causal key range in
 // contiguous 128-key tiles:
-//   S = Q K^T         tcgen05.mma M=128, N=128, K=d  -> TMEM (double buffer)
-//   P = masked softmax of S, one thread per row (the row's query's selection
-//       as a 128-bit mask per tile), written to shared memory as bf16
-//   O += P V          tcgen05.mma M=128, N=d, K=128 (V as an MN-major operand)
-//                     -> TMEM
-// The running maximum is only raised when a tile exceeds it by more than 2^8
-// (then O is rescaled in TMEM), so P stays below 256.
+//   S = Q K^T         tcgen05.mma M=128, N=128, K=d  -> TMEM (two buffers)
+//   P = masked softmax of S (the row's query's selection as a 128-bit mask
+//       per tile), bf16, written back into the TMEM columns of its own S
+//   O += P V          tcgen05.mma M=128, N=d, K=128, A (= P) read from TMEM,
+//                     V as an MN-major shared-memory operand -> TMEM
+// P aliases S, so with two S buffers the softmax of tile kt+1 runs while the
+// tensor core computes P V of tile kt and Q K^T of tile kt+2.  The running
+// maximum is only raised when a tile exceeds it by more than 2^8 (then O is
+// rescaled in TMEM), so P stays below 256.
 //
 // The selection of each query is first expanded into a bitmap (one bit per
 // key; selection_bitmap_kernel, which also validates the top-K rows), so that
 // the TMA producer can fetch each tile's [GQ x 128-bit] mask with the K and V
 // tiles and no warp waits on index loads.
 //
-// Warp roles: 0 TMA producer (Q once; K, V and mask rings of 2) and TMEM
-// allocator; 1 MMA issuer; 2..5 softmax (TMEM lane quadrant = warp % 4).
-// Every wait is bounded.
+// Warp roles: 0 TMA producer (Q once; K + mask ring of 3 running one tile
+// ahead of a V ring of 2) and TMEM allocator; 1 MMA issuer; 2..9 softmax, two
+// warps per TMEM lane quadrant (warp % 4), each taking 64 of a tile's 128
+// columns, exchanging the row maximum through shared memory.  Every wait is
+// bounded, and the two warps of a quadrant leave their loop together.
 #include <cudaTypedefs.h>
 #include <math_constants.h>
 
@@ -40,7 +44,8 @@ namespace sa {
 namespace {
 
 constexpr int kTile = 128;                  // keys per tile
-constexpr int kTcThreads = 6 * 32;
+constexpr int kSoftWarps = 8;               // two per TMEM lane quadrant
+constexpr int kTcThreads = (2 + kSoftWarps) * 32;
 constexpr int kBitmapThreads = 256;
 
 struct TcParams {
@@ -54,16 +59,16 @@ struct TcParams {
 
 template <int D>
 struct TcCfg {
+    static constexpr int kKS = 3, kVS = 2;                  // K (+ mask) ring, V ring
     static constexpr int kHalf = 128 * 128;                 // one 64-column SW128 half of a 128-row tile
     static constexpr int kQBytes = 128 * D * 2;             // 128 rows x D
     static constexpr int kKVBytes = kTile * D * 2;          // 128 keys x D
-    static constexpr int kPBytes = 128 * kTile * 2;         // 128 rows x 128 keys
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kQBytes;
-    static constexpr int kOffV = kOffK + 2 * kKVBytes;
-    static constexpr int kOffP = kOffV + 2 * kKVBytes;
-    static constexpr int kOffMask = kOffP + kPBytes;           // [2 slots of 512 B][GQ rows][4 words]
-    static constexpr int kOffBar = kOffMask + 2 * 512;
+    static constexpr int kOffV = kOffK + kKS * kKVBytes;
+    static constexpr int kOffMask = kOffV + kVS * kKVBytes;   // [kKS slots of 512 B][GQ rows][4 words]
+    static constexpr int kOffRed = kOffMask + kKS * 512;      // float [2][2 halves][128 rows], int [2][8]
+    static constexpr int kOffBar = kOffRed + 2 * 2 * 128 * 4 + 2 * 8 * 4;
     static constexpr size_t kSmem = 1024 + kOffBar + 256;
 };
 
@@ -81,7 +86,17 @@ __device__ __forceinline__ uint64_t desc_mn(uint32_t addr, uint32_t lbo) {
     return d;
 }
 
-__device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t (&r)[16]) {
+// D (TMEM) += A (TMEM: row i in lane i, two bf16 per 32-bit column) x B (smem descriptor).
+__device__ __forceinline__ void tc_mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                              uint32_t accumulate) {
+    asm volatile(
+        "{ .reg .pred p; setp.ne.b32 p, %4, 0;"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t *r) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
             taddr),
@@ -91,20 +106,19 @@ __device__ __forceinline__ void tmem_st_x16(uint32_t taddr, const uint32_t (&r)[
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// Set bits [a, b] (inclusive, tile-relative, clipped to [0, 127]) of m[4].
-__device__ __forceinline__ void set_range(uint32_t (&m)[4], int a, int b) {
-    a = max(a, 0);
-    b = min(b, kTile - 1);
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-        const int lo = max(a, 32 * w), hi = min(b, 32 * w + 31);
-        if (lo <= hi) {
-            const int n = hi - lo + 1;
-            const uint32_t bits = (n == 32) ? 0xffffffffu : (((1u << n) - 1u) << (lo - 32 * w));
-            m[w] |= bits;
-        }
-    }
+// 2^x with flush-to-zero (the ex2.approx.ftz PTX instruction); 2^-inf = 0.
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float y;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
+    return y;
+}
+// Named barrier for the `n` threads of the warps that share `id`.
+__device__ __forceinline__ void pair_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
 // Row t of the bitmap: bit s of word s / 32 is set iff s is in S(t) (for the
 // query at position p = S - T + t): the top-K entries <= p - W and the window
@@ -151,19 +165,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                           TcParams P) {
     using C = TcCfg<D>;
     constexpr int GQ = 128 / HQ;   // queries per CTA
+    constexpr int KS = C::kKS, VS = C::kVS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + C::kOffBar);
-    uint64_t *q_full = bar + 0;
-    uint64_t *k_full = bar + 1, *k_empty = bar + 3;      // [2]
-    uint64_t *v_full = bar + 5, *v_empty = bar + 7;      // [2]
-    uint64_t *s_full = bar + 9, *s_empty = bar + 11;     // [2]
-    uint64_t *p_full = bar + 13, *o_done = bar + 14;
-    uint64_t *m_full = bar + 15, *m_empty = bar + 17;    // [2]
-    uint64_t *drain = bar + 19;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 20);
+    uint64_t *q_full = bar;
+    uint64_t *k_full = bar + 1, *k_empty = k_full + KS;      // [KS]
+    uint64_t *m_full = k_empty + KS, *m_empty = m_full + KS;  // [KS]
+    uint64_t *v_full = m_empty + KS, *v_empty = v_full + VS;  // [VS]
+    uint64_t *s_full = v_empty + VS;                          // [2] S(kt) in TMEM buffer kt % 2
+    uint64_t *p_full = s_full + 2;                            // [2] P(kt) written over it
+    uint64_t *o_done = p_full + 2;                            // [2] P V of tile kt done (kt % 2)
+    uint64_t *drain = o_done + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    uint32_t *masks = reinterpret_cast<uint32_t *>(sm + C::kOffMask);   // [2][GQ][4]
+    uint32_t *masks = reinterpret_cast<uint32_t *>(sm + C::kOffMask);   // [KS][128 words]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = P.n_groups - 1 - blockIdx.x;                  // heavy (late) groups first
@@ -174,14 +190,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < KS; ++i) {
             mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1);
-            mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1);
-            mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 4);
-            mbar_init(&m_full[i], 1); mbar_init(&m_empty[i], 4);
+            mbar_init(&m_full[i], 1); mbar_init(&m_empty[i], kSoftWarps);
         }
-        mbar_init(p_full, 4);
-        mbar_init(o_done, 1);
+        for (int i = 0; i < VS; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1); mbar_init(&p_full[i], kSoftWarps); mbar_init(&o_done[i], 1);
+        }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -198,7 +214,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t t_s = tmem, t_o = tmem + 256;                // S buffers at columns 0, 128; O at 256
+    const uint32_t t_s = tmem, t_o = tmem + 256;                // S/P buffers at columns 0, 128; O at 256
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -207,23 +223,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_arrive_expect_tx(q_full, C::kQBytes);
             for (int h = 0; h < D / 64; ++h)
                 tma_load_2d(sm + C::kOffQ + h * C::kHalf, &map_q, h * 64, t0 * HQ, q_full);
-            for (int kt = 0; kt < n_tiles && ok; ++kt) {
-                const int s = kt & 1;
-                const uint32_t par = ((uint32_t)(kt >> 1) & 1u) ^ 1u;
-                ok = mbar_wait(&k_empty[s], par, abort_flag);
-                if (!ok) break;
-                mbar_arrive_expect_tx(&k_full[s], C::kKVBytes);
-                for (int h = 0; h < D / 64; ++h)
-                    tma_load_2d(sm + C::kOffK + s * C::kKVBytes + h * C::kHalf, &map_k, h * 64, kt * kTile, &k_full[s]);
-                ok = mbar_wait(&m_empty[s], par, abort_flag);
-                if (!ok) break;
-                mbar_arrive_expect_tx(&m_full[s], GQ * 16);
-                tma_load_2d(masks + s * 128, &map_m, kt * 4, t0, &m_full[s]);
-                ok = mbar_wait(&v_empty[s], par, abort_flag);
-                if (!ok) break;
-                mbar_arrive_expect_tx(&v_full[s], C::kKVBytes);
-                for (int h = 0; h < D / 64; ++h)
-                    tma_load_2d(sm + C::kOffV + s * C::kKVBytes + h * C::kHalf, &map_v, h * 64, kt * kTile, &v_full[s]);
+            // K and the mask of tile i go out together with V of tile i - 1
+            for (int i = 0; i <= n_tiles && ok; ++i) {
+                if (i < n_tiles) {
+                    const int ks = i % KS;
+                    const uint32_t par = ((uint32_t)(i / KS) & 1u) ^ 1u;
+                    ok = mbar_wait(&k_empty[ks], par, abort_flag);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&k_full[ks], C::kKVBytes);
+                    for (int h = 0; h < D / 64; ++h)
+                        tma_load_2d(sm + C::kOffK + ks * C::kKVBytes + h * C::kHalf, &map_k, h * 64, i * kTile,
+                                    &k_full[ks]);
+                    ok = mbar_wait(&m_empty[ks], par, abort_flag);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&m_full[ks], GQ * 16);
+                    tma_load_2d(masks + ks * 128, &map_m, i * 4, t0, &m_full[ks]);
+                }
+                if (i >= 1) {
+                    const int j = i - 1, vs = j % VS;
+                    ok = mbar_wait(&v_empty[vs], ((uint32_t)(j / VS) & 1u) ^ 1u, abort_flag);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&v_full[vs], C::kKVBytes);
+                    for (int h = 0; h < D / 64; ++h)
+                        tma_load_2d(sm + C::kOffV + vs * C::kKVBytes + h * C::kHalf, &map_v, h * 64, j * kTile,
+                                    &v_full[vs]);
+                }
             }
         }
         __syncwarp();
@@ -233,41 +257,43 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, kTile);
             constexpr uint32_t idesc_o = idesc_bf16_f32(128, D) | (1u << 16);   // B (V) MN-major
             const uint32_t qa = smem_u32(sm + C::kOffQ);
-            const uint32_t pa = smem_u32(sm + C::kOffP);
             bool ok = mbar_wait(q_full, 0, abort_flag);
+            // S(kt) into buffer kt % 2.  The buffer last held P(kt - 2), read by
+            // P V of tile kt - 2, which this thread issued earlier (the tensor
+            // core runs one thread's MMAs in order).
             auto issue_s = [&](int kt) -> bool {
-                const int s = kt & 1;
-                const uint32_t use = (uint32_t)(kt >> 1) & 1u;
-                if (!mbar_wait(&k_full[s], use, abort_flag) || !mbar_wait(&s_empty[s], use ^ 1u, abort_flag))
-                    return false;
+                const int ks = kt % KS;
+                if (!mbar_wait(&k_full[ks], (uint32_t)(kt / KS) & 1u, abort_flag)) return false;
                 tc_fence_after();
-                const uint32_t ka = smem_u32(sm + C::kOffK + s * C::kKVBytes);
+                const uint32_t ka = smem_u32(sm + C::kOffK + ks * C::kKVBytes);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (uint32_t)((kk >> 2) * C::kHalf + (kk & 3) * 32);
-                    tc_mma_f16(t_s + (uint32_t)(s * kTile), desc_k(qa + off), desc_k(ka + off), idesc_s, kk > 0);
+                    tc_mma_f16(t_s + (uint32_t)((kt & 1) * kTile), desc_k(qa + off), desc_k(ka + off), idesc_s,
+                               kk > 0);
                 }
-                tc_commit(&k_empty[s]);
-                tc_commit(&s_full[s]);
+                tc_commit(&k_empty[ks]);
+                tc_commit(&s_full[kt & 1]);
                 return true;
             };
             if (ok) ok = issue_s(0);
             if (ok && n_tiles > 1) ok = issue_s(1);
             for (int kt = 0; kt < n_tiles && ok; ++kt) {
-                const int s = kt & 1;
-                ok = mbar_wait(p_full, (uint32_t)kt & 1u, abort_flag) &&
-                     mbar_wait(&v_full[s], (uint32_t)(kt >> 1) & 1u, abort_flag);
+                const int s = kt & 1, vs = kt % VS;
+                ok = mbar_wait(&p_full[s], (uint32_t)(kt >> 1) & 1u, abort_flag) &&
+                     mbar_wait(&v_full[vs], (uint32_t)(kt / VS) & 1u, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t va = smem_u32(sm + C::kOffV + s * C::kKVBytes);
+                const uint32_t va = smem_u32(sm + C::kOffV + vs * C::kKVBytes);
+                // P of keys 0..63 sits in columns 0..31 of the buffer, keys 64..127 in 64..95
 #pragma unroll
                 for (int kk = 0; kk < kTile / 16; ++kk) {
-                    const uint32_t poff = (uint32_t)((kk >> 2) * C::kHalf + (kk & 3) * 32);
-                    tc_mma_f16(t_o, desc_k(pa + poff), desc_mn(va + (uint32_t)kk * 2048u, C::kHalf), idesc_o,
-                               (kt > 0 || kk > 0) ? 1u : 0u);
+                    const uint32_t pa = t_s + (uint32_t)(s * kTile + (kk >> 2) * 64 + (kk & 3) * 8);
+                    tc_mma_f16_ts(t_o, pa, desc_mn(va + (uint32_t)kk * 2048u, C::kHalf), idesc_o,
+                                  (kt > 0 || kk > 0) ? 1u : 0u);
                 }
-                tc_commit(&v_empty[s]);
-                tc_commit(o_done);
+                tc_commit(&v_empty[vs]);
+                tc_commit(&o_done[s]);
                 if (kt + 2 < n_tiles) ok = issue_s(kt + 2);
             }
             tc_commit(drain);
@@ -276,117 +302,146 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ softmax (one thread per row)
-        const int quad = warp & 3;
+        // ------------------------------------------------------------ softmax (half a row per thread)
+        const int sw = warp - 2;                   // 0..7
+        const int quad = warp & 3, half = sw >> 2;
+        const int partner = sw ^ 4;                // the warp holding the other 64 columns of these rows
         const int r = quad * 32 + lane;            // TMEM lane = row = (query, head)
         const int q = r / HQ, h = r % HQ;
         const bool act = q < nq;
-        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        uint8_t *prow = sm + C::kOffP + r * 128;   // this row in each 64-key half of P
-        float m_used = -CUDART_INF_F, l = 0.f;
+        const uint32_t lane_t = tmem + ((uint32_t)(quad * 32) << 16);
+        float *red = reinterpret_cast<float *>(sm + C::kOffRed);               // [2][2][128]
+        int *okx = reinterpret_cast<int *>(sm + C::kOffRed + 2 * 2 * 128 * 4);  // [2][8]
+        const float sl2 = P.scale_log2;
+        float m_used = -CUDART_INF_F, l = 0.f;     // m_used in log2 units (score x scale x log2 e)
         bool ok = true;
-        for (int kt = 0; kt < n_tiles && ok; ++kt) {
-            const int s = kt & 1;
-            const uint32_t use = (uint32_t)(kt >> 1) & 1u;
-            ok = __all_sync(0xffffffffu, mbar_wait(&m_full[s], use, abort_flag) && mbar_wait(&s_full[s], use, abort_flag));
-            if (!ok) break;
-            tc_fence_after();
-            uint32_t mk[4];
-            {
-                const uint32_t *src = masks + s * 128 + (act ? q : 0) * 4;
-                mk[0] = act ? src[0] : 0u; mk[1] = act ? src[1] : 0u;
-                mk[2] = act ? src[2] : 0u; mk[3] = act ? src[3] : 0u;
-            }
-            // the row's 128 scores, masked and scaled in place (one register array)
-            float x[kTile];
+        int xchg = -1;                             // last tile whose exchange both warps took
+        for (int kt = 0; kt < n_tiles; ++kt) {
+            const int s = kt & 1, ks = kt % KS;
+            const bool mine = ok && __all_sync(0xffffffffu, mbar_wait(&m_full[ks], (uint32_t)(kt / KS) & 1u,
+                                                                      abort_flag) &&
+                                                                mbar_wait(&s_full[s], (uint32_t)(kt >> 1) & 1u,
+                                                                          abort_flag));
+            float x[64];
+            float pmax = -CUDART_INF_F;
+            if (mine) {
+                tc_fence_after();
+                uint32_t mk0 = 0u, mk1 = 0u;
+                if (act) {
+                    const uint32_t *src = masks + ks * 128 + q * 4 + half * 2;
+                    mk0 = src[0];
+                    mk1 = src[1];
+                }
+                uint32_t raw[64];
 #pragma unroll
-            for (int c = 0; c < kTile; c += 16) {
-                uint32_t tmp[16];
-                tmem_ld_x16(t_s + lane_off + (uint32_t)(s * kTile + c), tmp);
+                for (int c = 0; c < 64; c += 16)
+                    tmem_ld_x16(lane_t + (uint32_t)(s * kTile + half * 64 + c),
+                                *reinterpret_cast<uint32_t(*)[16]>(&raw[c]));
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) x[c + i] = __uint_as_float(tmp[i]);
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) { mbar_arrive(&s_empty[s]); mbar_arrive(&m_empty[s]); }
-            float tmax = -CUDART_INF_F;
+                for (int c = 0; c < 64; ++c) asm volatile("" : "+r"(raw[c]));   // keep uses after the wait
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&m_empty[ks]);
+                float m4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
 #pragma unroll
-            for (int c = 0; c < kTile; ++c) {
-                const bool on = (mk[c >> 5] >> (c & 31)) & 1u;
-                x[c] = on ? x[c] * P.scale_log2 : -CUDART_INF_F;
-                tmax = fmaxf(tmax, x[c]);
-            }
-            // PV of the previous tile must be done before O is rescaled or P rewritten
-            if (kt > 0) {
-                ok = __all_sync(0xffffffffu, mbar_wait(o_done, (uint32_t)(kt - 1) & 1u, abort_flag));
-                if (!ok) break;
-                tc_fence_after();
-            }
-            const bool raise = tmax > m_used + 8.f;
-            if (__any_sync(0xffffffffu, raise && l > 0.f)) {
-                // rescale this warp's O rows whose maximum rose (rare)
-                const float f = (raise && l > 0.f) ? exp2f(m_used - tmax) : 1.f;
-#pragma unroll
-                for (int c = 0; c < D; c += 16) {
-                    uint32_t o[16];
-                    tmem_ld_x16(t_o + lane_off + (uint32_t)c, o);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-                    tmem_st_x16(t_o + lane_off + (uint32_t)c, o);
+                for (int c = 0; c < 64; ++c) {
+                    const uint32_t wbits = c < 32 ? mk0 : mk1;
+                    x[c] = ((wbits >> (c & 31)) & 1u) ? __uint_as_float(raw[c]) : -CUDART_INF_F;
                 }
-                tmem_st_wait();
+#pragma unroll
+                for (int c = 0; c < 64; c += 8) {
+                    const int a = (c >> 3) & 3;
+                    m4[a] = max3(m4[a], x[c], x[c + 1]);
+                    m4[a] = max3(m4[a], x[c + 2], x[c + 3]);
+                    m4[a] = max3(m4[a], x[c + 4], x[c + 5]);
+                    m4[a] = max3(m4[a], x[c + 6], x[c + 7]);
+                }
+                pmax = fmaxf(max3(m4[0], m4[1], m4[2]), m4[3]);
             }
+            // exchange the partial maxima (and whether both warps got this far)
+            red[(s * 2 + half) * 128 + r] = pmax;
+            if (lane == 0) okx[s * 8 + sw] = mine ? 1 : 0;
+            pair_sync(1 + quad, 64);
+            xchg = kt;
+            ok = mine && okx[s * 8 + partner] != 0;
+            if (!ok) break;   // both warps of the pair take the same decision
+            const float tmax = fmaxf(pmax, red[(s * 2 + (half ^ 1)) * 128 + r]) * sl2;
+            const bool raise = tmax > m_used + 8.f;
+            const bool resc = raise && m_used != -CUDART_INF_F;   // O holds earlier tiles (kt >= 1)
+            if (__any_sync(0xffffffffu, resc)) {
+                // P V of tile kt - 1 must be done before O is rescaled
+                ok = __all_sync(0xffffffffu, mbar_wait(&o_done[(kt - 1) & 1], (uint32_t)((kt - 1) >> 1) & 1u,
+                                                       abort_flag));
+                if (ok) {
+                    tc_fence_after();
+                    const float f = resc ? ex2(m_used - tmax) : 1.f;
+#pragma unroll
+                    for (int c = 0; c < D / 2; c += 16) {
+                        uint32_t o[16];
+                        const uint32_t ta = t_o + (uint32_t)(half * (D / 2) + c) + ((uint32_t)(quad * 32) << 16);
+                        tmem_ld_x16(ta, o);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+                        tmem_st_x16(ta, o);
+                    }
+                    tmem_st_wait();
+                }
+            }
+            if (!ok) continue;   // the next exchange ends the loop for both warps
             if (raise) {
-                if (l > 0.f) l *= exp2f(m_used - tmax);
+                l = resc ? l * ex2(m_used - tmax) : 0.f;
                 m_used = tmax;
             }
-            const float base = (m_used == -CUDART_INF_F) ? 0.f : m_used;
-            float rs = 0.f;
+            const float nb = (m_used == -CUDART_INF_F) ? 0.f : -m_used;
+            uint32_t pk[32];
 #pragma unroll
-            for (int c = 0; c < kTile; c += 8) {
-                uint32_t pk[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float a = exp2f(x[c + 2 * i] - base), b2 = exp2f(x[c + 2 * i + 1] - base);
-                    rs += a + b2;
-                    pk[i] = pack_bf16(a, b2);
-                }
-                // chunk (c / 8) of the row: 64-key half c / 64, 16-byte chunk (c % 64) / 8, SW128
-                const int half = c >> 6, ch = (c & 63) >> 3;
-                *reinterpret_cast<uint4 *>(prow + half * C::kHalf + ((ch ^ (r & 7)) << 4)) =
-                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            for (int i = 0; i < 32; ++i) {
+                const float a = ex2(fmaf(x[2 * i], sl2, nb)), b = ex2(fmaf(x[2 * i + 1], sl2, nb));
+                l += a + b;
+                pk[i] = pack_bf16(a, b);
             }
-            l += rs;
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // P writes -> tensor core reads
+            // keys 64 * half .. + 63 -> columns 64 * half .. + 31 of the buffer (S columns this thread read)
+            tmem_st_x16(lane_t + (uint32_t)(s * kTile + half * 64), &pk[0]);
+            tmem_st_x16(lane_t + (uint32_t)(s * kTile + half * 64 + 16), &pk[16]);
+            tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
+            if (lane == 0) mbar_arrive(&p_full[s]);
         }
-        // ---- epilogue: O / l
-        if (ok && __all_sync(0xffffffffu, mbar_wait(o_done, (uint32_t)(n_tiles - 1) & 1u, abort_flag))) {
-            tc_fence_after();
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            const int t = t0 + q;
-            uint16_t *orow = P.out + ((int64_t)t * HQ + h) * D;
+        // ---- epilogue: combine the two halves' row sums, O / l
+        {
+            const int e = (xchg + 1) & 1;          // the buffer the partner read one exchange ago
+            red[(e * 2 + half) * 128 + r] = l;
+            if (lane == 0) okx[e * 8 + sw] = ok ? 1 : 0;
+            pair_sync(1 + quad, 64);
+            ok = ok && okx[e * 8 + partner] != 0 && xchg == n_tiles - 1;
+            const float lt = l + red[(e * 2 + (half ^ 1)) * 128 + r];
+            const int n1 = n_tiles - 1;
+            if (ok && __all_sync(0xffffffffu, mbar_wait(&o_done[n1 & 1], (uint32_t)(n1 >> 1) & 1u, abort_flag))) {
+                tc_fence_after();
+                const float inv = lt > 0.f ? 1.f / lt : 0.f;
+                const int t = t0 + q;
+                uint16_t *orow = P.out + ((int64_t)t * HQ + h) * D + half * (D / 2);
 #pragma unroll
-            for (int c = 0; c < D; c += 16) {
-                uint32_t o[16];
-                tmem_ld_x16(t_o + lane_off + (uint32_t)c, o);
-                tmem_ld_wait();
-                if (act) {
-                    uint32_t pk[8];
+                for (int c = 0; c < D / 2; c += 16) {
+                    uint32_t o[16];
+                    tmem_ld_x16(t_o + (uint32_t)(half * (D / 2) + c) + ((uint32_t)(quad * 32) << 16), o);
+                    tmem_ld_wait();
+                    if (act) {
+                        uint32_t pk[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        pk[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c);
-                    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                        for (int i = 0; i < 8; ++i)
+                            pk[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + c);
+                        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                    }
                 }
+                if (act && half == 0 && P.lse)
+                    P.lse[(int64_t)t * HQ + h] =
+                        (lt > 0.f ? m_used + __log2f(lt) : -CUDART_INF_F) * 0.69314718055994531f;
             }
-            if (act && P.lse)
-                P.lse[(int64_t)t * HQ + h] = (l > 0.f ? m_used + __log2f(l) : -CUDART_INF_F) * 0.69314718055994531f;
         }
     }
 

@@ -94,7 +94,7 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
 
 // 2-D tiled load of the box at (x = inner coordinate, y = row) into smem,
 // completing `bytes` of transaction on `bar`.  x * element size must be a
-// multiple of 16 bytes; callers only pass x = 0.
+// multiple of 16 bytes.
 __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *map, int x, int y,
                                             uint64_t *bar) {
     asm volatile(
