@@ -8,29 +8,28 @@
 //
 // When each query selects a large share of its causal keys, gathering the
 // selected rows per query costs more L2 traffic than streaming the keys once
-// for a group of queries.  This kernel takes GQ = 128 / Hq consecutive queries
-// (M = GQ x Hq = 128 query-head rows) and walks the causal key range in
-// contiguous 128-key tiles:
-//   S = Q K^T         tcgen05.mma M=128, N=128, K=d  -> TMEM (two buffers)
-//   P = masked softmax of S (the row's query's selection as a 128-bit mask
-//       per tile), bf16, written back into the TMEM columns of its own S
-//   O += P V          tcgen05.mma M=128, N=d, K=128, A (= P) read from TMEM,
-//                     V as an MN-major shared-memory operand -> TMEM
-// P aliases S, so with two S buffers the softmax of tile kt+1 runs while the
-// tensor core computes P V of tile kt and Q K^T of tile kt+2.  The running
-// maximum is only raised when a tile exceeds it by more than 2^8 (then O is
-// rescaled in TMEM), so P stays below 256.
+// for a group of queries.  A CTA takes 2 GQ consecutive queries, GQ = 128 / Hq,
+// as two 128-row tiles A and B (row = (query, head)), and walks the causal key
+// range in contiguous 128-key tiles, each K and V tile serving both:
+//   S_X = Q_X K^T       tcgen05.mma M=128, N=128, K=d -> TMEM
+//   P_X = masked softmax of S_X (the row's query's selection as a 128-bit
+//         mask per tile), bf16, written back over S_X in TMEM
+//   O_X += P_X V        tcgen05.mma M=128, N=d, K=128, A (= P_X) from TMEM,
+//                       V as an MN-major shared-memory operand -> TMEM
+// The tensor core alternates between the tiles (P V and the next S of A,
+// then of B), so the softmax of one tile runs while the other's matrix
+// products execute.  The running maximum is only raised when a tile exceeds
+// it by more than 2^8 (then O_X is rescaled in TMEM), so P stays below 256.
 //
 // The selection of each query is first expanded into a bitmap (one bit per
 // key; selection_bitmap_kernel, which also validates the top-K rows), so that
-// the TMA producer can fetch each tile's [GQ x 128-bit] mask with the K and V
-// tiles and no warp waits on index loads.
+// the TMA producer can fetch each tile's [2 GQ x 128-bit] mask with the K and
+// V tiles and no warp waits on index loads.
 //
-// Warp roles: 0 TMA producer (Q once; K + mask ring of 3 running one tile
-// ahead of a V ring of 2) and TMEM allocator; 1 MMA issuer; 2..9 softmax, two
-// warps per TMEM lane quadrant (warp % 4), each taking 64 of a tile's 128
-// columns, exchanging the row maximum through shared memory.  Every wait is
-// bounded, and the two warps of a quadrant leave their loop together.
+// Warp roles: 0 TMA producer (Q once; K + mask ring running one tile ahead of
+// a V ring of 2) and TMEM allocator; 1 MMA issuer; 2..5 softmax of tile A and
+// 6..9 of tile B, one thread per row (TMEM lane quadrant = warp % 4).  Every
+// wait is bounded.
 #include <cudaTypedefs.h>
 #include <math_constants.h>
 
@@ -44,9 +43,9 @@ namespace sa {
 namespace {
 
 constexpr int kTile = 128;                  // keys per tile
-constexpr int kSoftWarps = 8;               // two per TMEM lane quadrant
-constexpr int kTcThreads = (2 + kSoftWarps) * 32;
+constexpr int kTcThreads = 10 * 32;
 constexpr int kBitmapThreads = 256;
+constexpr size_t kSmemLimit = 232448;       // opt-in dynamic shared memory per CTA
 
 struct TcParams {
     int T, S, Hq;
@@ -57,19 +56,24 @@ struct TcParams {
     int n_groups;
 };
 
-template <int D>
+template <int D, int HQ>
 struct TcCfg {
-    static constexpr int kKS = 3, kVS = 2;                  // K (+ mask) ring, V ring
+    static constexpr int GQ = 128 / HQ;                     // queries per 128-row tile
     static constexpr int kHalf = 128 * 128;                 // one 64-column SW128 half of a 128-row tile
     static constexpr int kQBytes = 128 * D * 2;             // 128 rows x D
     static constexpr int kKVBytes = kTile * D * 2;          // 128 keys x D
-    static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + kQBytes;
+    static constexpr int kMaskBytes = 2 * GQ * 16;          // [2 GQ queries][4 words]
+    static constexpr int kVS = 2;
+    static constexpr size_t bytes(int ks) {
+        return 1024 + 2 * kQBytes + (size_t)(ks + kVS) * kKVBytes + (size_t)ks * kMaskBytes + 256;
+    }
+    static constexpr int kKS = bytes(3) <= kSmemLimit ? 3 : 2;   // K (+ mask) ring
+    static constexpr int kOffQ = 0;                         // [2 tiles]
+    static constexpr int kOffK = 2 * kQBytes;
     static constexpr int kOffV = kOffK + kKS * kKVBytes;
-    static constexpr int kOffMask = kOffV + kVS * kKVBytes;   // [kKS slots of 512 B][GQ rows][4 words]
-    static constexpr int kOffRed = kOffMask + kKS * 512;      // float [2][2 halves][128 rows], int [2][8]
-    static constexpr int kOffBar = kOffRed + 2 * 2 * 128 * 4 + 2 * 8 * 4;
-    static constexpr size_t kSmem = 1024 + kOffBar + 256;
+    static constexpr int kOffMask = kOffV + kVS * kKVBytes;
+    static constexpr int kOffBar = kOffMask + kKS * kMaskBytes;
+    static constexpr size_t kSmem = bytes(kKS);
 };
 
 __device__ __forceinline__ uint64_t desc_k(uint32_t addr) { return smem_desc(addr, 1024, 2); }
@@ -117,8 +121,25 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
     return y;
 }
-// Named barrier for the `n` threads of the warps that share `id`.
-__device__ __forceinline__ void pair_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+// Packed pairs of f32 (one 64-bit register pair) for the f32x2 instructions.
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float &lo, float &hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
 
 // Row t of the bitmap: bit s of word s / 32 is set iff s is in S(t) (for the
 // query at position p = S - T + t): the top-K entries <= p - W and the window
@@ -163,8 +184,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     masked_attn_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                           const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_m,
                           TcParams P) {
-    using C = TcCfg<D>;
-    constexpr int GQ = 128 / HQ;   // queries per CTA
+    using C = TcCfg<D, HQ>;
+    constexpr int GQ = C::GQ;
     constexpr int KS = C::kKS, VS = C::kVS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -173,31 +194,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint64_t *k_full = bar + 1, *k_empty = k_full + KS;      // [KS]
     uint64_t *m_full = k_empty + KS, *m_empty = m_full + KS;  // [KS]
     uint64_t *v_full = m_empty + KS, *v_empty = v_full + VS;  // [VS]
-    uint64_t *s_full = v_empty + VS;                          // [2] S(kt) in TMEM buffer kt % 2
-    uint64_t *p_full = s_full + 2;                            // [2] P(kt) written over it
-    uint64_t *o_done = p_full + 2;                            // [2] P V of tile kt done (kt % 2)
+    uint64_t *s_full = v_empty + VS;                          // [2 tiles] S_X(kt) in TMEM
+    uint64_t *p_full = s_full + 2;                            // [2 tiles] P_X(kt) written over it
+    uint64_t *o_done = p_full + 2;                            // [2 tiles] P_X V of tile kt done
     uint64_t *drain = o_done + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    uint32_t *masks = reinterpret_cast<uint32_t *>(sm + C::kOffMask);   // [KS][128 words]
+    uint32_t *masks = reinterpret_cast<uint32_t *>(sm + C::kOffMask);   // [KS][2 GQ][4]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = P.n_groups - 1 - blockIdx.x;                  // heavy (late) groups first
-    const int t0 = g * GQ;
-    const int nq = min(GQ, P.T - t0);
-    const int p_last = P.S - P.T + t0 + nq - 1;                 // position of the group's last query
+    const int t0 = g * 2 * GQ;
+    const int nq = min(2 * GQ, P.T - t0);
+    const int p_last = P.S - P.T + t0 + nq - 1;                 // position of the CTA's last query
     const int n_tiles = p_last / kTile + 1;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
         for (int i = 0; i < KS; ++i) {
             mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1);
-            mbar_init(&m_full[i], 1); mbar_init(&m_empty[i], kSoftWarps);
+            mbar_init(&m_full[i], 1); mbar_init(&m_empty[i], 8);
         }
         for (int i = 0; i < VS; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&s_full[i], 1); mbar_init(&p_full[i], kSoftWarps); mbar_init(&o_done[i], 1);
-        }
+        for (int i = 0; i < 2; ++i) { mbar_init(&s_full[i], 1); mbar_init(&p_full[i], 4); mbar_init(&o_done[i], 1); }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -213,16 +232,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const uint32_t t_s = tmem, t_o = tmem + 256;                // S/P buffers at columns 0, 128; O at 256
+    const uint32_t tmem = *tmem_slot;   // S_A, S_B at columns 0, 128; O_A, O_B at 256, 256 + D
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             bool ok = true;
-            mbar_arrive_expect_tx(q_full, C::kQBytes);
-            for (int h = 0; h < D / 64; ++h)
-                tma_load_2d(sm + C::kOffQ + h * C::kHalf, &map_q, h * 64, t0 * HQ, q_full);
+            mbar_arrive_expect_tx(q_full, 2 * C::kQBytes);
+            for (int x = 0; x < 2; ++x)
+                for (int h = 0; h < D / 64; ++h)
+                    tma_load_2d(sm + C::kOffQ + x * C::kQBytes + h * C::kHalf, &map_q, h * 64, (t0 + x * GQ) * HQ,
+                                q_full);
             // K and the mask of tile i go out together with V of tile i - 1
             for (int i = 0; i <= n_tiles && ok; ++i) {
                 if (i < n_tiles) {
@@ -236,8 +256,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                     &k_full[ks]);
                     ok = mbar_wait(&m_empty[ks], par, abort_flag);
                     if (!ok) break;
-                    mbar_arrive_expect_tx(&m_full[ks], GQ * 16);
-                    tma_load_2d(masks + ks * 128, &map_m, i * 4, t0, &m_full[ks]);
+                    mbar_arrive_expect_tx(&m_full[ks], C::kMaskBytes);
+                    tma_load_2d(sm + C::kOffMask + ks * C::kMaskBytes, &map_m, i * 4, t0, &m_full[ks]);
                 }
                 if (i >= 1) {
                     const int j = i - 1, vs = j % VS;
@@ -257,44 +277,57 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, kTile);
             constexpr uint32_t idesc_o = idesc_bf16_f32(128, D) | (1u << 16);   // B (V) MN-major
             const uint32_t qa = smem_u32(sm + C::kOffQ);
-            bool ok = mbar_wait(q_full, 0, abort_flag);
-            // S(kt) into buffer kt % 2.  The buffer last held P(kt - 2), read by
-            // P V of tile kt - 2, which this thread issued earlier (the tensor
-            // core runs one thread's MMAs in order).
-            auto issue_s = [&](int kt) -> bool {
-                const int ks = kt % KS;
-                if (!mbar_wait(&k_full[ks], (uint32_t)(kt / KS) & 1u, abort_flag)) return false;
-                tc_fence_after();
-                const uint32_t ka = smem_u32(sm + C::kOffK + ks * C::kKVBytes);
+            // S_X(kt) = Q_X K(kt)^T over the columns of S_X, which last held
+            // P_X(kt - 1), read by P V of tile kt - 1 that this thread issued
+            // earlier (the tensor core runs one thread's MMAs in order).
+            auto s_mma = [&](int x, int kt) {
+                const uint32_t ka = smem_u32(sm + C::kOffK + (kt % KS) * C::kKVBytes);
+                const uint32_t qx = qa + (uint32_t)(x * C::kQBytes);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (uint32_t)((kk >> 2) * C::kHalf + (kk & 3) * 32);
-                    tc_mma_f16(t_s + (uint32_t)((kt & 1) * kTile), desc_k(qa + off), desc_k(ka + off), idesc_s,
-                               kk > 0);
+                    tc_mma_f16(tmem + (uint32_t)(x * kTile), desc_k(qx + off), desc_k(ka + off), idesc_s, kk > 0);
                 }
-                tc_commit(&k_empty[ks]);
-                tc_commit(&s_full[kt & 1]);
-                return true;
+                tc_commit(&s_full[x]);
             };
-            if (ok) ok = issue_s(0);
-            if (ok && n_tiles > 1) ok = issue_s(1);
+            auto pv_mma = [&](int x, int kt, uint32_t va) {
+#pragma unroll
+                for (int kk = 0; kk < kTile / 16; ++kk)
+                    tc_mma_f16_ts(tmem + 256u + (uint32_t)(x * D), tmem + (uint32_t)(x * kTile + kk * 8),
+                                  desc_mn(va + (uint32_t)kk * 2048u, C::kHalf), idesc_o, (kt > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(&o_done[x]);
+            };
+            bool ok = mbar_wait(q_full, 0, abort_flag) && mbar_wait(&k_full[0], 0, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                s_mma(0, 0);
+                s_mma(1, 0);
+                tc_commit(&k_empty[0]);
+            }
             for (int kt = 0; kt < n_tiles && ok; ++kt) {
-                const int s = kt & 1, vs = kt % VS;
-                ok = mbar_wait(&p_full[s], (uint32_t)(kt >> 1) & 1u, abort_flag) &&
-                     mbar_wait(&v_full[vs], (uint32_t)(kt / VS) & 1u, abort_flag);
+                const int vs = kt % VS, kn = kt + 1, ks = kn % KS;
+                const uint32_t par = (uint32_t)kt & 1u;
+                ok = mbar_wait(&v_full[vs], (uint32_t)(kt / VS) & 1u, abort_flag) &&
+                     mbar_wait(&p_full[0], par, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t va = smem_u32(sm + C::kOffV + vs * C::kKVBytes);
-                // P of keys 0..63 sits in columns 0..31 of the buffer, keys 64..127 in 64..95
-#pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk) {
-                    const uint32_t pa = t_s + (uint32_t)(s * kTile + (kk >> 2) * 64 + (kk & 3) * 8);
-                    tc_mma_f16_ts(t_o, pa, desc_mn(va + (uint32_t)kk * 2048u, C::kHalf), idesc_o,
-                                  (kt > 0 || kk > 0) ? 1u : 0u);
+                pv_mma(0, kt, va);
+                if (kn < n_tiles) {
+                    ok = mbar_wait(&k_full[ks], (uint32_t)(kn / KS) & 1u, abort_flag);
+                    if (!ok) break;
+                    tc_fence_after();
+                    s_mma(0, kn);
                 }
+                ok = mbar_wait(&p_full[1], par, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                pv_mma(1, kt, va);
                 tc_commit(&v_empty[vs]);
-                tc_commit(&o_done[s]);
-                if (kt + 2 < n_tiles) ok = issue_s(kt + 2);
+                if (kn < n_tiles) {
+                    s_mma(1, kn);
+                    tc_commit(&k_empty[ks]);
+                }
             }
             tc_commit(drain);
             volatile int no_abort = 0;
@@ -302,146 +335,139 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ softmax (half a row per thread)
-        const int sw = warp - 2;                   // 0..7
-        const int quad = warp & 3, half = sw >> 2;
-        const int partner = sw ^ 4;                // the warp holding the other 64 columns of these rows
+        // ------------------------------------------------------------ softmax (one thread per row)
+        const int x = (warp - 2) >> 2;             // tile A (0) or B (1)
+        const int quad = warp & 3;
         const int r = quad * 32 + lane;            // TMEM lane = row = (query, head)
-        const int q = r / HQ, h = r % HQ;
-        const bool act = q < nq;
+        const int qi = x * GQ + r / HQ, h = r % HQ;
+        const bool act = qi < nq;
         const uint32_t lane_t = tmem + ((uint32_t)(quad * 32) << 16);
-        float *red = reinterpret_cast<float *>(sm + C::kOffRed);               // [2][2][128]
-        int *okx = reinterpret_cast<int *>(sm + C::kOffRed + 2 * 2 * 128 * 4);  // [2][8]
+        const uint32_t s_t = lane_t + (uint32_t)(x * kTile);
+        const uint32_t o_t = lane_t + 256u + (uint32_t)(x * D);
         const float sl2 = P.scale_log2;
-        float m_used = -CUDART_INF_F, l = 0.f;     // m_used in log2 units (score x scale x log2 e)
+        const uint64_t sl2x2 = f2(sl2, sl2);
+        float m_used = -CUDART_INF_F;              // log2 units: score x scale x log2 e
+        uint64_t l2 = f2(0.f, 0.f);                // row sum, as two partial sums
         bool ok = true;
-        int xchg = -1;                             // last tile whose exchange both warps took
         for (int kt = 0; kt < n_tiles; ++kt) {
-            const int s = kt & 1, ks = kt % KS;
-            const bool mine = ok && __all_sync(0xffffffffu, mbar_wait(&m_full[ks], (uint32_t)(kt / KS) & 1u,
-                                                                      abort_flag) &&
-                                                                mbar_wait(&s_full[s], (uint32_t)(kt >> 1) & 1u,
-                                                                          abort_flag));
-            float x[64];
-            float pmax = -CUDART_INF_F;
-            if (mine) {
-                tc_fence_after();
-                uint32_t mk0 = 0u, mk1 = 0u;
-                if (act) {
-                    const uint32_t *src = masks + ks * 128 + q * 4 + half * 2;
-                    mk0 = src[0];
-                    mk1 = src[1];
-                }
-                uint32_t raw[64];
+            const int ks = kt % KS;
+            ok = __all_sync(0xffffffffu, mbar_wait(&m_full[ks], (uint32_t)(kt / KS) & 1u, abort_flag) &&
+                                             mbar_wait(&s_full[x], (uint32_t)kt & 1u, abort_flag));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t mk[4] = {0u, 0u, 0u, 0u};
+            if (act) {
+                const uint4 m4 = *reinterpret_cast<const uint4 *>(masks + ks * (C::kMaskBytes / 4) + qi * 4);
+                mk[0] = m4.x; mk[1] = m4.y; mk[2] = m4.z; mk[3] = m4.w;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&m_empty[ks]);
+            // pass 1: masked scores (-inf outside the selection) back into S_X, and their maximum
+            float mx[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t v[64];
 #pragma unroll
                 for (int c = 0; c < 64; c += 16)
-                    tmem_ld_x16(lane_t + (uint32_t)(s * kTile + half * 64 + c),
-                                *reinterpret_cast<uint32_t(*)[16]>(&raw[c]));
+                    tmem_ld_x16(s_t + (uint32_t)(hh * 64 + c), *reinterpret_cast<uint32_t(*)[16]>(&v[c]));
                 tmem_ld_wait();
 #pragma unroll
-                for (int c = 0; c < 64; ++c) asm volatile("" : "+r"(raw[c]));   // keep uses after the wait
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&m_empty[ks]);
-                float m4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+                for (int c = 0; c < 64; ++c) asm volatile("" : "+r"(v[c]));   // keep uses after the wait
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    const uint32_t wbits = c < 32 ? mk0 : mk1;
-                    x[c] = ((wbits >> (c & 31)) & 1u) ? __uint_as_float(raw[c]) : -CUDART_INF_F;
+                for (int c = 0; c < 64; ++c)
+                    if (!((mk[hh * 2 + (c >> 5)] >> (c & 31)) & 1u)) v[c] = 0xff800000u;   // -inf
+#pragma unroll
+                for (int c = 0; c < 64; c += 2) {
+                    const int a = (c >> 1) & 3;
+                    mx[a] = max3(mx[a], __uint_as_float(v[c]), __uint_as_float(v[c + 1]));
                 }
 #pragma unroll
-                for (int c = 0; c < 64; c += 8) {
-                    const int a = (c >> 3) & 3;
-                    m4[a] = max3(m4[a], x[c], x[c + 1]);
-                    m4[a] = max3(m4[a], x[c + 2], x[c + 3]);
-                    m4[a] = max3(m4[a], x[c + 4], x[c + 5]);
-                    m4[a] = max3(m4[a], x[c + 6], x[c + 7]);
-                }
-                pmax = fmaxf(max3(m4[0], m4[1], m4[2]), m4[3]);
+                for (int c = 0; c < 64; c += 16) tmem_st_x16(s_t + (uint32_t)(hh * 64 + c), &v[c]);
             }
-            // exchange the partial maxima (and whether both warps got this far)
-            red[(s * 2 + half) * 128 + r] = pmax;
-            if (lane == 0) okx[s * 8 + sw] = mine ? 1 : 0;
-            pair_sync(1 + quad, 64);
-            xchg = kt;
-            ok = mine && okx[s * 8 + partner] != 0;
-            if (!ok) break;   // both warps of the pair take the same decision
-            const float tmax = fmaxf(pmax, red[(s * 2 + (half ^ 1)) * 128 + r]) * sl2;
+            const float tmax = fmaxf(max3(mx[0], mx[1], mx[2]), mx[3]) * sl2;
             const bool raise = tmax > m_used + 8.f;
-            const bool resc = raise && m_used != -CUDART_INF_F;   // O holds earlier tiles (kt >= 1)
+            const bool resc = raise && m_used != -CUDART_INF_F;   // O_X holds earlier tiles
             if (__any_sync(0xffffffffu, resc)) {
-                // P V of tile kt - 1 must be done before O is rescaled
-                ok = __all_sync(0xffffffffu, mbar_wait(&o_done[(kt - 1) & 1], (uint32_t)((kt - 1) >> 1) & 1u,
-                                                       abort_flag));
-                if (ok) {
-                    tc_fence_after();
-                    const float f = resc ? ex2(m_used - tmax) : 1.f;
+                // P_X V of tile kt - 1 is done: this thread saw S_X(kt), issued after it
+                const float f = resc ? ex2(m_used - tmax) : 1.f;
 #pragma unroll
-                    for (int c = 0; c < D / 2; c += 16) {
-                        uint32_t o[16];
-                        const uint32_t ta = t_o + (uint32_t)(half * (D / 2) + c) + ((uint32_t)(quad * 32) << 16);
-                        tmem_ld_x16(ta, o);
-                        tmem_ld_wait();
+                for (int c = 0; c < D; c += 16) {
+                    uint32_t o[16];
+                    tmem_ld_x16(o_t + (uint32_t)c, o);
+                    tmem_ld_wait();
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-                        tmem_st_x16(ta, o);
-                    }
-                    tmem_st_wait();
+                    for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+                    tmem_st_x16(o_t + (uint32_t)c, o);
                 }
             }
-            if (!ok) continue;   // the next exchange ends the loop for both warps
             if (raise) {
-                l = resc ? l * ex2(m_used - tmax) : 0.f;
+                if (resc) {
+                    const float f = ex2(m_used - tmax);
+                    l2 = fma2(l2, f2(f, f), f2(0.f, 0.f));
+                } else {
+                    l2 = f2(0.f, 0.f);
+                }
                 m_used = tmax;
             }
+            tmem_st_wait();   // masked scores (and rescaled O) are in TMEM
             const float nb = (m_used == -CUDART_INF_F) ? 0.f : -m_used;
-            uint32_t pk[32];
+            const uint64_t nbx2 = f2(nb, nb);
+            // pass 2: P = 2^(x scale log2 e - m_used) over the columns of S_X
+            // (keys 64 hh .. 64 hh + 63 -> columns 32 hh .. 32 hh + 31, all read by now)
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float a = ex2(fmaf(x[2 * i], sl2, nb)), b = ex2(fmaf(x[2 * i + 1], sl2, nb));
-                l += a + b;
-                pk[i] = pack_bf16(a, b);
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t v[64];
+#pragma unroll
+                for (int c = 0; c < 64; c += 16)
+                    tmem_ld_x16(s_t + (uint32_t)(hh * 64 + c), *reinterpret_cast<uint32_t(*)[16]>(&v[c]));
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < 64; ++c) asm volatile("" : "+r"(v[c]));
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    float a, b;
+                    f2_split(fma2(f2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), sl2x2, nbx2), a, b);
+                    a = ex2(a);
+                    b = ex2(b);
+                    l2 = add2(l2, f2(a, b));
+                    pk[i] = pack_bf16(a, b);
+                }
+                tmem_st_x16(s_t + (uint32_t)(hh * 32), &pk[0]);
+                tmem_st_x16(s_t + (uint32_t)(hh * 32 + 16), &pk[16]);
             }
-            // keys 64 * half .. + 63 -> columns 64 * half .. + 31 of the buffer (S columns this thread read)
-            tmem_st_x16(lane_t + (uint32_t)(s * kTile + half * 64), &pk[0]);
-            tmem_st_x16(lane_t + (uint32_t)(s * kTile + half * 64 + 16), &pk[16]);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[s]);
+            if (lane == 0) mbar_arrive(&p_full[x]);
         }
-        // ---- epilogue: combine the two halves' row sums, O / l
-        {
-            const int e = (xchg + 1) & 1;          // the buffer the partner read one exchange ago
-            red[(e * 2 + half) * 128 + r] = l;
-            if (lane == 0) okx[e * 8 + sw] = ok ? 1 : 0;
-            pair_sync(1 + quad, 64);
-            ok = ok && okx[e * 8 + partner] != 0 && xchg == n_tiles - 1;
-            const float lt = l + red[(e * 2 + (half ^ 1)) * 128 + r];
-            const int n1 = n_tiles - 1;
-            if (ok && __all_sync(0xffffffffu, mbar_wait(&o_done[n1 & 1], (uint32_t)(n1 >> 1) & 1u, abort_flag))) {
-                tc_fence_after();
-                const float inv = lt > 0.f ? 1.f / lt : 0.f;
-                const int t = t0 + q;
-                uint16_t *orow = P.out + ((int64_t)t * HQ + h) * D + half * (D / 2);
+        // ---- epilogue: O_X / l
+        const int n1 = n_tiles - 1;
+        if (ok && __all_sync(0xffffffffu, mbar_wait(&o_done[x], (uint32_t)n1 & 1u, abort_flag))) {
+            tc_fence_after();
+            float la, lb;
+            f2_split(l2, la, lb);
+            const float l = la + lb;
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const int t = t0 + qi;
+            uint16_t *orow = P.out + ((int64_t)t * HQ + h) * D;
 #pragma unroll
-                for (int c = 0; c < D / 2; c += 16) {
-                    uint32_t o[16];
-                    tmem_ld_x16(t_o + (uint32_t)(half * (D / 2) + c) + ((uint32_t)(quad * 32) << 16), o);
-                    tmem_ld_wait();
-                    if (act) {
-                        uint32_t pk[8];
+            for (int c = 0; c < D; c += 16) {
+                uint32_t o[16];
+                tmem_ld_x16(o_t + (uint32_t)c, o);
+                tmem_ld_wait();
+                if (act) {
+                    uint32_t pk[8];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            pk[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + c);
-                        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                    }
+                    for (int i = 0; i < 8; ++i)
+                        pk[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c);
+                    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                 }
-                if (act && half == 0 && P.lse)
-                    P.lse[(int64_t)t * HQ + h] =
-                        (lt > 0.f ? m_used + __log2f(lt) : -CUDART_INF_F) * 0.69314718055994531f;
             }
+            if (act && P.lse)
+                P.lse[(int64_t)t * HQ + h] = (l > 0.f ? m_used + __log2f(l) : -CUDART_INF_F) * 0.69314718055994531f;
         }
     }
 
@@ -479,13 +505,13 @@ bool map_rows(CUtensorMap *m, const void *base, uint64_t rows, int D) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// selection bitmap [T rows x words] uint32, box = GQ rows x 4 words (one 128-key tile)
-bool map_bitmap(CUtensorMap *m, const void *base, uint64_t rows, int words, int gq) {
+// selection bitmap [T rows x words] uint32, box = `rows_box` rows x 4 words (one 128-key tile)
+bool map_bitmap(CUtensorMap *m, const void *base, uint64_t rows, int words, int rows_box) {
     auto enc = encoder();
     if (!enc) return false;
     cuuint64_t dims[2] = {(cuuint64_t)words, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)words * 4};
-    cuuint32_t box[2] = {4, (cuuint32_t)gq};
+    cuuint32_t box[2] = {4, (cuuint32_t)rows_box};
     cuuint32_t estr[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void *>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
@@ -496,18 +522,19 @@ int bitmap_words(int S) { return (S + kTile - 1) / kTile * 4; }
 
 template <int D, int HQ>
 sa_status launch_tc(const PrefillArgs &a, cudaStream_t st) {
-    using C = TcCfg<D>;
-    constexpr int GQ = 128 / HQ;
+    using C = TcCfg<D, HQ>;
+    constexpr int GQ = C::GQ;
+    static_assert(C::kSmem <= kSmemLimit, "shared memory");
     TcParams p;
     p.T = a.T; p.S = a.S; p.Hq = a.Hq;
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.out = a.out; p.lse = a.lse; p.dev_status = a.dev_status;
-    p.n_groups = (a.T + GQ - 1) / GQ;
+    p.n_groups = (a.T + 2 * GQ - 1) / (2 * GQ);
     const int words = bitmap_words(a.S);
     uint32_t *bitmap = reinterpret_cast<uint32_t *>(a.workspace);
     CUtensorMap mq, mk, mv, mm;
     if (!map_rows(&mq, a.q, (uint64_t)a.T * HQ, D) || !map_rows(&mk, a.k, (uint64_t)a.S, D) ||
-        !map_rows(&mv, a.v, (uint64_t)a.S, D) || !map_bitmap(&mm, bitmap, (uint64_t)a.T, words, GQ))
+        !map_rows(&mv, a.v, (uint64_t)a.S, D) || !map_bitmap(&mm, bitmap, (uint64_t)a.T, words, 2 * GQ))
         return SA_ERR_CUDA;
     const size_t bsmem = (size_t)words * 4;
     if (prepare_kernel<selection_bitmap_kernel>(bsmem, false) != cudaSuccess) return SA_ERR_CUDA;
