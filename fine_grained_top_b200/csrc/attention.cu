@@ -515,8 +515,10 @@ sa_status launch_prefill(const PrefillArgs &a, cudaStream_t st) {
     // Dense selections (each query keeps a large share of its causal keys):
     // stream contiguous K/V tiles once per group of queries through masked
     // tensor-core tiles instead of gathering every query's rows.
-    if (a.workspace && prefill_tc_supported(a) && a.workspace_bytes >= prefill_tc_workspace_bytes(a.T, a.S))
-        return launch_prefill_tc(a, st);
+    if (a.workspace && prefill_tc_supported(a) && a.workspace_bytes >= prefill_tc_workspace_bytes(a.T, a.S)) {
+        const sa_status s = launch_prefill_tc(a, st);
+        if (s != SA_ERR_UNSUPPORTED) return s;   // else the gathered path below
+    }
     AttnParams p = base_params(a.q, a.k, a.v, a.topk, a.K, a.W, a.Hq, a.d, a.scale, a.out, a.lse, a.dev_status);
     p.T = a.T;
     p.S = a.S;

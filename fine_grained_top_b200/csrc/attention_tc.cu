@@ -10,7 +10,8 @@
 // selected rows per query costs more L2 traffic than streaming the keys once
 // for a group of queries.  A CTA takes 2 GQ consecutive queries, GQ = 128 / Hq,
 // as two 128-row tiles A and B (row = (query, head)), and walks the causal key
-// range in contiguous 128-key tiles, each K and V tile serving both:
+// range in contiguous 128-key tiles (starting at a tile that differs between
+// neighbouring CTAs), each K and V tile serving both:
 //   S_X = Q_X K^T       tcgen05.mma M=128, N=128, K=d -> TMEM
 //   P_X = masked softmax of S_X (the row's query's selection as a 128-bit
 //         mask per tile), bf16, written back over S_X in TMEM
@@ -27,9 +28,10 @@
 // V tiles and no warp waits on index loads.
 //
 // Warp roles: 0 TMA producer (Q once; K + mask ring running one tile ahead of
-// a V ring of 2) and TMEM allocator; 1 MMA issuer; 2..5 softmax of tile A and
-// 6..9 of tile B, one thread per row (TMEM lane quadrant = warp % 4).  Every
-// wait is bounded.
+// a V ring of 2) and TMEM allocator; 1 MMA issuer; 2, 3 idle; 4..7 softmax of
+// tile A and 8..11 of tile B, one thread per row (TMEM lane quadrant =
+// warp % 4), which hold the row's 128 scores in registers (the first
+// warpgroup hands its registers over with setmaxnreg).  Every wait is bounded.
 #include <cudaTypedefs.h>
 #include <math_constants.h>
 
@@ -43,7 +45,9 @@ namespace sa {
 namespace {
 
 constexpr int kTile = 128;                  // keys per tile
-constexpr int kTcThreads = 10 * 32;
+constexpr int kTcThreads = 12 * 32;                // three warpgroups
+constexpr int kTcRegs = 168;                        // registers per thread at launch: 65536 / 384, rounded down to 8
+constexpr int kRegsLow = 80, kRegsHigh = 208;       // after the handover: producer / MMA group, softmax groups
 constexpr int kBitmapThreads = 256;
 constexpr size_t kSmemLimit = 232448;       // opt-in dynamic shared memory per CTA
 
@@ -208,6 +212,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int nq = min(2 * GQ, P.T - t0);
     const int p_last = P.S - P.T + t0 + nq - 1;                 // position of the CTA's last query
     const int n_tiles = p_last / kTile + 1;
+    // The CTA visits its key tiles starting from a different one than its
+    // neighbours (the softmax does not depend on the order), so that CTAs
+    // running at the same time read different K/V tiles from L2.
+    const int rot = (int)(blockIdx.x % (unsigned)n_tiles);
+    auto tile_of = [&](int i) { return i + rot < n_tiles ? i + rot : i + rot - n_tiles; };
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -233,7 +242,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;   // S_A, S_B at columns 0, 128; O_A, O_B at 256, 256 + D
+    // The first warpgroup (producer, MMA issuer, two idle warps) hands registers
+    // to the two softmax warpgroups; the sum stays within the launch's allocation.
+    static_assert(128 * kRegsLow + 256 * kRegsHigh <= kTcThreads * kTcRegs, "register split");
 
+    if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow) : "memory");
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
@@ -252,12 +266,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     if (!ok) break;
                     mbar_arrive_expect_tx(&k_full[ks], C::kKVBytes);
                     for (int h = 0; h < D / 64; ++h)
-                        tma_load_2d(sm + C::kOffK + ks * C::kKVBytes + h * C::kHalf, &map_k, h * 64, i * kTile,
-                                    &k_full[ks]);
+                        tma_load_2d(sm + C::kOffK + ks * C::kKVBytes + h * C::kHalf, &map_k, h * 64,
+                                    tile_of(i) * kTile, &k_full[ks]);
                     ok = mbar_wait(&m_empty[ks], par, abort_flag);
                     if (!ok) break;
                     mbar_arrive_expect_tx(&m_full[ks], C::kMaskBytes);
-                    tma_load_2d(sm + C::kOffMask + ks * C::kMaskBytes, &map_m, i * 4, t0, &m_full[ks]);
+                    tma_load_2d(sm + C::kOffMask + ks * C::kMaskBytes, &map_m, tile_of(i) * 4, t0, &m_full[ks]);
                 }
                 if (i >= 1) {
                     const int j = i - 1, vs = j % VS;
@@ -265,8 +279,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                     if (!ok) break;
                     mbar_arrive_expect_tx(&v_full[vs], C::kKVBytes);
                     for (int h = 0; h < D / 64; ++h)
-                        tma_load_2d(sm + C::kOffV + vs * C::kKVBytes + h * C::kHalf, &map_v, h * 64, j * kTile,
-                                    &v_full[vs]);
+                        tma_load_2d(sm + C::kOffV + vs * C::kKVBytes + h * C::kHalf, &map_v, h * 64,
+                                    tile_of(j) * kTile, &v_full[vs]);
                 }
             }
         }
@@ -334,9 +348,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_wait(drain, 0, &no_abort);
         }
         __syncwarp();
+    }
     } else {
         // ------------------------------------------------------------ softmax (one thread per row)
-        const int x = (warp - 2) >> 2;             // tile A (0) or B (1)
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh) : "memory");
+        const int x = (warp - 4) >> 2;             // tile A (0) or B (1)
         const int quad = warp & 3;
         const int r = quad * 32 + lane;            // TMEM lane = row = (query, head)
         const int qi = x * GQ + r / HQ, h = r % HQ;
@@ -362,27 +378,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&m_empty[ks]);
-            // pass 1: masked scores (-inf outside the selection) back into S_X, and their maximum
+            // the row's 128 scores, -inf outside the selection, and their maximum
+            uint32_t v[128];
+#pragma unroll
+            for (int c = 0; c < 128; c += 16)
+                tmem_ld_x16(s_t + (uint32_t)c, *reinterpret_cast<uint32_t(*)[16]>(&v[c]));
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 128; ++c) asm volatile("" : "+r"(v[c]));   // keep uses after the wait
             float mx[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                uint32_t v[64];
+            for (int c = 0; c < 128; ++c)
+                if (!((mk[c >> 5] >> (c & 31)) & 1u)) v[c] = 0xff800000u;   // -inf
 #pragma unroll
-                for (int c = 0; c < 64; c += 16)
-                    tmem_ld_x16(s_t + (uint32_t)(hh * 64 + c), *reinterpret_cast<uint32_t(*)[16]>(&v[c]));
-                tmem_ld_wait();
-#pragma unroll
-                for (int c = 0; c < 64; ++c) asm volatile("" : "+r"(v[c]));   // keep uses after the wait
-#pragma unroll
-                for (int c = 0; c < 64; ++c)
-                    if (!((mk[hh * 2 + (c >> 5)] >> (c & 31)) & 1u)) v[c] = 0xff800000u;   // -inf
-#pragma unroll
-                for (int c = 0; c < 64; c += 2) {
-                    const int a = (c >> 1) & 3;
-                    mx[a] = max3(mx[a], __uint_as_float(v[c]), __uint_as_float(v[c + 1]));
-                }
-#pragma unroll
-                for (int c = 0; c < 64; c += 16) tmem_st_x16(s_t + (uint32_t)(hh * 64 + c), &v[c]);
+            for (int c = 0; c < 128; c += 2) {
+                const int a = (c >> 1) & 3;
+                mx[a] = max3(mx[a], __uint_as_float(v[c]), __uint_as_float(v[c + 1]));
             }
             const float tmax = fmaxf(max3(mx[0], mx[1], mx[2]), mx[3]) * sl2;
             const bool raise = tmax > m_used + 8.f;
@@ -390,7 +401,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (__any_sync(0xffffffffu, resc)) {
                 // P_X V of tile kt - 1 is done: this thread saw S_X(kt), issued after it
                 const float f = resc ? ex2(m_used - tmax) : 1.f;
-#pragma unroll
+#pragma unroll 1
                 for (int c = 0; c < D; c += 16) {
                     uint32_t o[16];
                     tmem_ld_x16(o_t + (uint32_t)c, o);
@@ -409,32 +420,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 m_used = tmax;
             }
-            tmem_st_wait();   // masked scores (and rescaled O) are in TMEM
             const float nb = (m_used == -CUDART_INF_F) ? 0.f : -m_used;
             const uint64_t nbx2 = f2(nb, nb);
-            // pass 2: P = 2^(x scale log2 e - m_used) over the columns of S_X
-            // (keys 64 hh .. 64 hh + 63 -> columns 32 hh .. 32 hh + 31, all read by now)
+            // P = 2^(x scale log2 e - m_used), keys 2i, 2i + 1 -> column i of S_X
+            // (all of S_X has been read into registers)
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                uint32_t v[64];
+            for (int c = 0; c < 128; c += 32) {
+                uint32_t pk[16];
 #pragma unroll
-                for (int c = 0; c < 64; c += 16)
-                    tmem_ld_x16(s_t + (uint32_t)(hh * 64 + c), *reinterpret_cast<uint32_t(*)[16]>(&v[c]));
-                tmem_ld_wait();
-#pragma unroll
-                for (int c = 0; c < 64; ++c) asm volatile("" : "+r"(v[c]));
-                uint32_t pk[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
+                for (int i = 0; i < 16; ++i) {
                     float a, b;
-                    f2_split(fma2(f2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), sl2x2, nbx2), a, b);
+                    f2_split(fma2(f2(__uint_as_float(v[c + 2 * i]), __uint_as_float(v[c + 2 * i + 1])), sl2x2, nbx2),
+                             a, b);
                     a = ex2(a);
                     b = ex2(b);
                     l2 = add2(l2, f2(a, b));
                     pk[i] = pack_bf16(a, b);
                 }
-                tmem_st_x16(s_t + (uint32_t)(hh * 32), &pk[0]);
-                tmem_st_x16(s_t + (uint32_t)(hh * 32 + 16), &pk[16]);
+                tmem_st_x16(s_t + (uint32_t)(c / 2), pk);
             }
             tmem_st_wait();
             tc_fence_before();
@@ -525,6 +528,15 @@ sa_status launch_tc(const PrefillArgs &a, cudaStream_t st) {
     using C = TcCfg<D, HQ>;
     constexpr int GQ = C::GQ;
     static_assert(C::kSmem <= kSmemLimit, "shared memory");
+    // The register handover inside the kernel assumes the launch allocation
+    // of kTcRegs per thread; with any other count it is not run.
+    static int regs_ok = -1;
+    if (regs_ok < 0) {
+        cudaFuncAttributes fa;
+        regs_ok = (cudaFuncGetAttributes(&fa, masked_attn_tc_kernel<D, HQ>) == cudaSuccess && fa.numRegs == kTcRegs)
+                      ? 1 : 0;
+    }
+    if (!regs_ok) return SA_ERR_UNSUPPORTED;
     TcParams p;
     p.T = a.T; p.S = a.S; p.Hq = a.Hq;
     p.scale_log2 = a.scale * 1.4426950408889634f;
