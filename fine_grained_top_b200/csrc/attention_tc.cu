@@ -27,8 +27,8 @@
 // the TMA producer can fetch each tile's [2 GQ x 128-bit] mask with the K and
 // V tiles and no warp waits on index loads.
 //
-// Warp roles: 0 TMA producer (Q once; K + mask ring running one tile ahead of
-// a V ring of 2) and TMEM allocator; 1 MMA issuer; 2, 3 idle; 4..7 softmax of
+// Warp roles: 0 TMA producer (Q once; a ring whose step i carries K and the
+// mask of tile i with V of tile i - 1) and TMEM allocator; 1 MMA issuer; 2, 3 idle; 4..7 softmax of
 // tile A and 8..11 of tile B, one thread per row (TMEM lane quadrant =
 // warp % 4), which hold the row's 128 scores in registers (the first
 // warpgroup hands its registers over with setmaxnreg).  Every wait is bounded.
@@ -67,17 +67,17 @@ struct TcCfg {
     static constexpr int kQBytes = 128 * D * 2;             // 128 rows x D
     static constexpr int kKVBytes = kTile * D * 2;          // 128 keys x D
     static constexpr int kMaskBytes = 2 * GQ * 16;          // [2 GQ queries][4 words]
-    static constexpr int kVS = 2;
-    static constexpr size_t bytes(int ks) {
-        return 1024 + 2 * kQBytes + (size_t)(ks + kVS) * kKVBytes + (size_t)ks * kMaskBytes + 256;
+    // Step i of the ring carries K and the mask of tile i and V of tile i - 1.
+    static constexpr size_t bytes(int ns) {
+        return 1024 + 2 * kQBytes + (size_t)ns * (2 * kKVBytes + kMaskBytes) + 256;
     }
-    static constexpr int kKS = bytes(3) <= kSmemLimit ? 3 : 2;   // K (+ mask) ring
+    static constexpr int kNS = bytes(3) <= kSmemLimit ? 3 : 2;
     static constexpr int kOffQ = 0;                         // [2 tiles]
-    static constexpr int kOffK = 2 * kQBytes;
-    static constexpr int kOffV = kOffK + kKS * kKVBytes;
-    static constexpr int kOffMask = kOffV + kVS * kKVBytes;
-    static constexpr int kOffBar = kOffMask + kKS * kMaskBytes;
-    static constexpr size_t kSmem = bytes(kKS);
+    static constexpr int kOffK = 2 * kQBytes;               // [kNS]
+    static constexpr int kOffV = kOffK + kNS * kKVBytes;    // [kNS]
+    static constexpr int kOffMask = kOffV + kNS * kKVBytes;  // [kNS]
+    static constexpr int kOffBar = kOffMask + kNS * kMaskBytes;
+    static constexpr size_t kSmem = bytes(kNS);
 };
 
 __device__ __forceinline__ uint64_t desc_k(uint32_t addr) { return smem_desc(addr, 1024, 2); }
@@ -101,6 +101,22 @@ __device__ __forceinline__ void tc_mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, 
         "{ .reg .pred p; setp.ne.b32 p, %4, 0;"
         " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }" ::"r"(d_tmem),
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// The same two forms with the accumulator always read (no predicate register).
+__device__ __forceinline__ void tc_mma_ss_acc(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc) {
+    asm volatile(
+        "{ .reg .pred p; setp.eq.u32 p, 1, 1;"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc)
+        : "memory");
+}
+__device__ __forceinline__ void tc_mma_ts_acc(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc) {
+    asm volatile(
+        "{ .reg .pred p; setp.eq.u32 p, 1, 1;"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc)
         : "memory");
 }
 
@@ -190,21 +206,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                           TcParams P) {
     using C = TcCfg<D, HQ>;
     constexpr int GQ = C::GQ;
-    constexpr int KS = C::kKS, VS = C::kVS;
+    constexpr int NS = C::kNS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + C::kOffBar);
     uint64_t *q_full = bar;
-    uint64_t *k_full = bar + 1, *k_empty = k_full + KS;      // [KS]
-    uint64_t *m_full = k_empty + KS, *m_empty = m_full + KS;  // [KS]
-    uint64_t *v_full = m_empty + KS, *v_empty = v_full + VS;  // [VS]
-    uint64_t *s_full = v_empty + VS;                          // [2 tiles] S_X(kt) in TMEM
+    uint64_t *kv_full = bar + 1, *kv_empty = kv_full + NS;   // [NS] K(i), V(i - 1) of step i
+    uint64_t *m_full = kv_empty + NS, *m_empty = m_full + NS; // [NS] mask of tile i
+    uint64_t *s_full = m_empty + NS;                          // [2 tiles] S_X(kt) in TMEM
     uint64_t *p_full = s_full + 2;                            // [2 tiles] P_X(kt) written over it
-    uint64_t *o_done = p_full + 2;                            // [2 tiles] P_X V of tile kt done
+    uint64_t *o_done = p_full + 2;                            // [2 tiles] the last P_X V done
     uint64_t *drain = o_done + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    uint32_t *masks = reinterpret_cast<uint32_t *>(sm + C::kOffMask);   // [KS][2 GQ][4]
+    uint32_t *masks = reinterpret_cast<uint32_t *>(sm + C::kOffMask);   // [NS][2 GQ][4]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = P.n_groups - 1 - blockIdx.x;                  // heavy (late) groups first
@@ -220,11 +235,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int i = 0; i < KS; ++i) {
-            mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1);
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&kv_full[i], 1); mbar_init(&kv_empty[i], 1);
             mbar_init(&m_full[i], 1); mbar_init(&m_empty[i], 8);
         }
-        for (int i = 0; i < VS; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
         for (int i = 0; i < 2; ++i) { mbar_init(&s_full[i], 1); mbar_init(&p_full[i], 4); mbar_init(&o_done[i], 1); }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -257,30 +271,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 for (int h = 0; h < D / 64; ++h)
                     tma_load_2d(sm + C::kOffQ + x * C::kQBytes + h * C::kHalf, &map_q, h * 64, (t0 + x * GQ) * HQ,
                                 q_full);
-            // K and the mask of tile i go out together with V of tile i - 1
+            // step i: K and the mask of tile i, V of tile i - 1
             for (int i = 0; i <= n_tiles && ok; ++i) {
+                const int ns = i % NS;
+                const uint32_t par = ((uint32_t)(i / NS) & 1u) ^ 1u;
+                ok = mbar_wait(&kv_empty[ns], par, abort_flag);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&kv_full[ns], (i < n_tiles ? C::kKVBytes : 0) + (i >= 1 ? C::kKVBytes : 0));
+                if (i < n_tiles)
+                    for (int h = 0; h < D / 64; ++h)
+                        tma_load_2d(sm + C::kOffK + ns * C::kKVBytes + h * C::kHalf, &map_k, h * 64,
+                                    tile_of(i) * kTile, &kv_full[ns]);
+                if (i >= 1)
+                    for (int h = 0; h < D / 64; ++h)
+                        tma_load_2d(sm + C::kOffV + ns * C::kKVBytes + h * C::kHalf, &map_v, h * 64,
+                                    tile_of(i - 1) * kTile, &kv_full[ns]);
                 if (i < n_tiles) {
-                    const int ks = i % KS;
-                    const uint32_t par = ((uint32_t)(i / KS) & 1u) ^ 1u;
-                    ok = mbar_wait(&k_empty[ks], par, abort_flag);
+                    ok = mbar_wait(&m_empty[ns], par, abort_flag);
                     if (!ok) break;
-                    mbar_arrive_expect_tx(&k_full[ks], C::kKVBytes);
-                    for (int h = 0; h < D / 64; ++h)
-                        tma_load_2d(sm + C::kOffK + ks * C::kKVBytes + h * C::kHalf, &map_k, h * 64,
-                                    tile_of(i) * kTile, &k_full[ks]);
-                    ok = mbar_wait(&m_empty[ks], par, abort_flag);
-                    if (!ok) break;
-                    mbar_arrive_expect_tx(&m_full[ks], C::kMaskBytes);
-                    tma_load_2d(sm + C::kOffMask + ks * C::kMaskBytes, &map_m, tile_of(i) * 4, t0, &m_full[ks]);
-                }
-                if (i >= 1) {
-                    const int j = i - 1, vs = j % VS;
-                    ok = mbar_wait(&v_empty[vs], ((uint32_t)(j / VS) & 1u) ^ 1u, abort_flag);
-                    if (!ok) break;
-                    mbar_arrive_expect_tx(&v_full[vs], C::kKVBytes);
-                    for (int h = 0; h < D / 64; ++h)
-                        tma_load_2d(sm + C::kOffV + vs * C::kKVBytes + h * C::kHalf, &map_v, h * 64,
-                                    tile_of(j) * kTile, &v_full[vs]);
+                    mbar_arrive_expect_tx(&m_full[ns], C::kMaskBytes);
+                    tma_load_2d(sm + C::kOffMask + ns * C::kMaskBytes, &map_m, tile_of(i) * 4, t0, &m_full[ns]);
                 }
             }
         }
@@ -290,58 +300,59 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, kTile);
             constexpr uint32_t idesc_o = idesc_bf16_f32(128, D) | (1u << 16);   // B (V) MN-major
-            const uint32_t qa = smem_u32(sm + C::kOffQ);
+            // Descriptors are built once; an operand at byte offset o from a base
+            // is base + (o >> 4) (the 14-bit address field never carries over).
+            const uint64_t q_d = desc_k(smem_u32(sm + C::kOffQ));
+            const uint64_t k_d = desc_k(smem_u32(sm + C::kOffK));
+            const uint64_t v_d = desc_mn(smem_u32(sm + C::kOffV), C::kHalf);
             // S_X(kt) = Q_X K(kt)^T over the columns of S_X, which last held
             // P_X(kt - 1), read by P V of tile kt - 1 that this thread issued
             // earlier (the tensor core runs one thread's MMAs in order).
             auto s_mma = [&](int x, int kt) {
-                const uint32_t ka = smem_u32(sm + C::kOffK + (kt % KS) * C::kKVBytes);
-                const uint32_t qx = qa + (uint32_t)(x * C::kQBytes);
+                const uint64_t qd = q_d + (uint64_t)(x * (C::kQBytes >> 4));
+                const uint64_t kd = k_d + (uint64_t)((kt % NS) * (C::kKVBytes >> 4));
+                const uint32_t dt = tmem + (uint32_t)(x * kTile);
+                tc_mma_f16(dt, qd, kd, idesc_s, 0u);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (uint32_t)((kk >> 2) * C::kHalf + (kk & 3) * 32);
-                    tc_mma_f16(tmem + (uint32_t)(x * kTile), desc_k(qx + off), desc_k(ka + off), idesc_s, kk > 0);
+                for (int kk = 1; kk < D / 16; ++kk) {
+                    const uint64_t off = (uint64_t)(((kk >> 2) * C::kHalf + (kk & 3) * 32) >> 4);
+                    tc_mma_ss_acc(dt, qd + off, kd + off, idesc_s);
                 }
                 tc_commit(&s_full[x]);
             };
-            auto pv_mma = [&](int x, int kt, uint32_t va) {
+            // O_X += P_X V: P_X in the first 64 columns of S_X, V(kt) MN-major
+            auto pv_mma = [&](int x, int kt, uint64_t vd) {
+                const uint32_t dt = tmem + 256u + (uint32_t)(x * D), at = tmem + (uint32_t)(x * kTile);
+                tc_mma_f16_ts(dt, at, vd, idesc_o, kt > 0 ? 1u : 0u);
 #pragma unroll
-                for (int kk = 0; kk < kTile / 16; ++kk)
-                    tc_mma_f16_ts(tmem + 256u + (uint32_t)(x * D), tmem + (uint32_t)(x * kTile + kk * 8),
-                                  desc_mn(va + (uint32_t)kk * 2048u, C::kHalf), idesc_o, (kt > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(&o_done[x]);
+                for (int kk = 1; kk < kTile / 16; ++kk)
+                    tc_mma_ts_acc(dt, at + (uint32_t)(kk * 8), vd + (uint64_t)((kk * 2048) >> 4), idesc_o);
+                if (kt == n_tiles - 1) tc_commit(&o_done[x]);
             };
-            bool ok = mbar_wait(q_full, 0, abort_flag) && mbar_wait(&k_full[0], 0, abort_flag);
+            bool ok = mbar_wait(q_full, 0, abort_flag) && mbar_wait(&kv_full[0], 0, abort_flag);
             if (ok) {
                 tc_fence_after();
                 s_mma(0, 0);
                 s_mma(1, 0);
-                tc_commit(&k_empty[0]);
+                tc_commit(&kv_empty[0]);
             }
+            // step kt + 1 holds V(kt) and K(kt + 1); one commit releases both
             for (int kt = 0; kt < n_tiles && ok; ++kt) {
-                const int vs = kt % VS, kn = kt + 1, ks = kn % KS;
+                const int kn = kt + 1, ns = kn % NS;
                 const uint32_t par = (uint32_t)kt & 1u;
-                ok = mbar_wait(&v_full[vs], (uint32_t)(kt / VS) & 1u, abort_flag) &&
+                ok = mbar_wait(&kv_full[ns], (uint32_t)(kn / NS) & 1u, abort_flag) &&
                      mbar_wait(&p_full[0], par, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t va = smem_u32(sm + C::kOffV + vs * C::kKVBytes);
-                pv_mma(0, kt, va);
-                if (kn < n_tiles) {
-                    ok = mbar_wait(&k_full[ks], (uint32_t)(kn / KS) & 1u, abort_flag);
-                    if (!ok) break;
-                    tc_fence_after();
-                    s_mma(0, kn);
-                }
+                const uint64_t vd = v_d + (uint64_t)(ns * (C::kKVBytes >> 4));
+                pv_mma(0, kt, vd);
+                if (kn < n_tiles) s_mma(0, kn);
                 ok = mbar_wait(&p_full[1], par, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
-                pv_mma(1, kt, va);
-                tc_commit(&v_empty[vs]);
-                if (kn < n_tiles) {
-                    s_mma(1, kn);
-                    tc_commit(&k_empty[ks]);
-                }
+                pv_mma(1, kt, vd);
+                if (kn < n_tiles) s_mma(1, kn);
+                tc_commit(&kv_empty[ns]);
             }
             tc_commit(drain);
             volatile int no_abort = 0;
@@ -366,8 +377,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         uint64_t l2 = f2(0.f, 0.f);                // row sum, as two partial sums
         bool ok = true;
         for (int kt = 0; kt < n_tiles; ++kt) {
-            const int ks = kt % KS;
-            ok = __all_sync(0xffffffffu, mbar_wait(&m_full[ks], (uint32_t)(kt / KS) & 1u, abort_flag) &&
+            const int ks = kt % NS;
+            ok = __all_sync(0xffffffffu, mbar_wait(&m_full[ks], (uint32_t)(kt / NS) & 1u, abort_flag) &&
                                              mbar_wait(&s_full[x], (uint32_t)kt & 1u, abort_flag));
             if (!ok) break;
             tc_fence_after();
@@ -445,8 +456,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (lane == 0) mbar_arrive(&p_full[x]);
         }
         // ---- epilogue: O_X / l
-        const int n1 = n_tiles - 1;
-        if (ok && __all_sync(0xffffffffu, mbar_wait(&o_done[x], (uint32_t)n1 & 1u, abort_flag))) {
+        if (ok && __all_sync(0xffffffffu, mbar_wait(&o_done[x], 0u, abort_flag))) {
             tc_fence_after();
             float la, lb;
             f2_split(l2, la, lb);
