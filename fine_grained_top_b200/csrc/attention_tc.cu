@@ -28,10 +28,10 @@
 // V tiles and no warp waits on index loads.
 //
 // Warp roles: 0 TMA producer (Q once; a ring whose step i carries K and the
-// mask of tile i with V of tile i - 1) and TMEM allocator; 1 MMA issuer; 2, 3 idle; 4..7 softmax of
-// tile A and 8..11 of tile B, one thread per row (TMEM lane quadrant =
-// warp % 4), which hold the row's 128 scores in registers (the first
-// warpgroup hands its registers over with setmaxnreg).  Every wait is bounded.
+// mask of tile i with V of tile i - 1) and TMEM allocator; 1 MMA issuer;
+// 2..5 softmax of tile A and 6..9 of tile B, one thread per row (TMEM lane
+// quadrant = warp % 4) holding the row's 128 scores in registers.  Every wait
+// is bounded.
 #include <cudaTypedefs.h>
 #include <math_constants.h>
 
@@ -45,9 +45,7 @@ namespace sa {
 namespace {
 
 constexpr int kTile = 128;                  // keys per tile
-constexpr int kTcThreads = 12 * 32;                // three warpgroups
-constexpr int kTcRegs = 168;                        // registers per thread at launch: 65536 / 384, rounded down to 8
-constexpr int kRegsLow = 80, kRegsHigh = 208;       // after the handover: producer / MMA group, softmax groups
+constexpr int kTcThreads = 10 * 32;
 constexpr int kBitmapThreads = 256;
 constexpr size_t kSmemLimit = 232448;       // opt-in dynamic shared memory per CTA
 
@@ -141,6 +139,9 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     asm("max.f32 %0, %1, %2, %3;" : "=f"(y) : "f"(a), "f"(b), "f"(c));
     return y;
 }
+// Named barrier `id` over `n` threads (warps may reach it from different code).
+__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+
 // Packed pairs of f32 (one 64-bit register pair) for the f32x2 instructions.
 __device__ __forceinline__ uint64_t f2(float lo, float hi) {
     uint64_t r;
@@ -217,7 +218,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint64_t *p_full = s_full + 2;                            // [2 tiles] P_X(kt) written over it
     uint64_t *o_done = p_full + 2;                            // [2 tiles] the last P_X V done
     uint64_t *drain = o_done + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    constexpr int kSlotWord = 8 + 4 * NS;                     // tmem_slot, abort flag after the barriers
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + kSlotWord);
+    static_assert(kSlotWord * 8 + 8 <= 256, "barrier region");
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     uint32_t *masks = reinterpret_cast<uint32_t *>(sm + C::kOffMask);   // [NS][2 GQ][4]
 
@@ -256,12 +259,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;   // S_A, S_B at columns 0, 128; O_A, O_B at 256, 256 + D
-    // The first warpgroup (producer, MMA issuer, two idle warps) hands registers
-    // to the two softmax warpgroups; the sum stays within the launch's allocation.
-    static_assert(128 * kRegsLow + 256 * kRegsHigh <= kTcThreads * kTcRegs, "register split");
 
-    if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow) : "memory");
+    if (warp < 2) {
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
@@ -360,10 +359,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         __syncwarp();
     }
+    // Once all warps are past their last TMEM access, warp 0 frees TMEM.
+    tc_fence_before();
+    named_sync(1, kTcThreads);
+    if (warp == 0) {
+        uint8_t *smb = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+        uint32_t *slot = reinterpret_cast<uint32_t *>(reinterpret_cast<uint64_t *>(smb + C::kOffBar) + kSlotWord);
+        if (lane == 0 && *reinterpret_cast<volatile int *>(slot + 1)) report(P.dev_status, SA_DEV_TIMEOUT);
+        tc_fence_after();
+        tmem_dealloc(*slot, 512);
+    }
     } else {
         // ------------------------------------------------------------ softmax (one thread per row)
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh) : "memory");
-        const int x = (warp - 4) >> 2;             // tile A (0) or B (1)
+        const int x = (warp - 2) >> 2;             // tile A (0) or B (1)
         const int quad = warp & 3;
         const int r = quad * 32 + lane;            // TMEM lane = row = (query, head)
         const int qi = x * GQ + r / HQ, h = r % HQ;
@@ -482,14 +490,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             if (act && P.lse)
                 P.lse[(int64_t)t * HQ + h] = (l > 0.f ? m_used + __log2f(l) : -CUDART_INF_F) * 0.69314718055994531f;
         }
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    if (threadIdx.x == 0 && *abort_flag) report(P.dev_status, SA_DEV_TIMEOUT);
-    if (warp == 0) {
-        tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tc_fence_before();
+        named_sync(1, kTcThreads);   // TMEM is freed by warp 0 after this
     }
 }
 
@@ -538,15 +540,6 @@ sa_status launch_tc(const PrefillArgs &a, cudaStream_t st) {
     using C = TcCfg<D, HQ>;
     constexpr int GQ = C::GQ;
     static_assert(C::kSmem <= kSmemLimit, "shared memory");
-    // The register handover inside the kernel assumes the launch allocation
-    // of kTcRegs per thread; with any other count it is not run.
-    static int regs_ok = -1;
-    if (regs_ok < 0) {
-        cudaFuncAttributes fa;
-        regs_ok = (cudaFuncGetAttributes(&fa, masked_attn_tc_kernel<D, HQ>) == cudaSuccess && fa.numRegs == kTcRegs)
-                      ? 1 : 0;
-    }
-    if (!regs_ok) return SA_ERR_UNSUPPORTED;
     TcParams p;
     p.T = a.T; p.S = a.S; p.Hq = a.Hq;
     p.scale_log2 = a.scale * 1.4426950408889634f;
