@@ -52,17 +52,18 @@ def load_peaks():
 
 # --------------------------------------------------------------------------- ncu traffic
 STAGE_SOURCE = {"indexer": "indexer.cu", "coarse_indexer": "indexer.cu", "topk": "topk.cu",
-                "coarse_topk": "topk.cu", "fine_topk": "topk.cu", "attention": "attention.cu",
+                "coarse_topk": "topk.cu", "fine_topk": "topk.cu", "attention": "attention.cu+attention_tc.cu",
                 "fine_indexer": "block_scores.cu", "expand": "two_stage.cu", "pool": "two_stage.cu",
                 "block_counts": "two_stage.cu"}
 
 
 def source_hash(cu: str) -> str:
-    """SHA-1 (12 hex digits) over a kernel's .cu file, then ptx.cuh, then internal.h."""
+    """SHA-1 (12 hex digits) over a stage's .cu files ('+'-separated), then
+    ptx.cuh, then internal.h."""
     import hashlib
     csrc = os.path.join(ROOT, "fine_grained_top_b200", "csrc")
     m = hashlib.sha1()
-    for f in (cu, "ptx.cuh", "internal.h"):
+    for f in cu.split("+") + ["ptx.cuh", "internal.h"]:
         m.update(open(os.path.join(csrc, f), "rb").read())
     return m.hexdigest()[:12]
 

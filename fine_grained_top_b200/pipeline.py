@@ -41,7 +41,12 @@ class PrefillPlan:
         self.out = torch.empty((N, Hq, d), dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty((N, Hq), dtype=f32, device=dev)
         self.dev_status = torch.zeros(1, dtype=i32, device=dev)
-        self.attn_ws_bytes = sa_prefill_workspace_bytes(N, N, K, W, Hq, d)
+        # The masked tensor-core attention (selected by passing its bitmap
+        # workspace) runs one CTA per 256 query-head rows; below one CTA per SM
+        # the gathered kernel, one CTA per query, is faster.
+        groups = N * Hq // 256
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count if dev.type == "cuda" else 148
+        self.attn_ws_bytes = sa_prefill_workspace_bytes(N, N, K, W, Hq, d) if groups >= sms else 0
         self.attn_ws = (torch.empty(self.attn_ws_bytes, dtype=torch.uint8, device=dev)
                         if self.attn_ws_bytes else None)
         if block is None:
