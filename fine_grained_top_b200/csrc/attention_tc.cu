@@ -162,6 +162,34 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
     return r;
 }
 
+// 2^y for a pair, on the FMA pipe instead of the ex2 unit.  Range reduction:
+// adding 1.5 * 2^23 rounds y to the nearest integer r in the low mantissa bits
+// of t (exact for |y| < 2^22), f = y - r lies in [-1/2, 1/2], and 2^f is a
+// cubic fitted to it in relative error (max 7.5e-5, well below bf16's 2^-8
+// spacing).  r is added to the exponent field of 2^f: the shifter's own bits
+// shifted left by 23 vanish mod 2^32, so t_bits << 23 == r << 23.  y is first
+// raised to -126, where 2^y is below 2^-125 (masked keys, y = -inf, end there
+// rather than at 0; callers judge "nothing selected" by the running maximum).
+constexpr float kExpShift = 12582912.0f;   // 1.5 * 2^23
+constexpr float kExp2C0 = 9.999280572e-01f, kExp2C1 = 6.932609677e-01f, kExp2C2 = 2.426111400e-01f,
+                kExp2C3 = 5.517166853e-02f;
+__device__ __forceinline__ void exp2_pair_fma(uint64_t y, float &a, float &b) {
+    float y0, y1;
+    f2_split(y, y0, y1);
+    const uint64_t yc = f2(fmaxf(y0, -126.f), fmaxf(y1, -126.f));
+    const uint64_t t = add2(yc, f2(kExpShift, kExpShift));
+    const uint64_t r = add2(t, f2(-kExpShift, -kExpShift));
+    const uint64_t fr = fma2(r, f2(-1.f, -1.f), yc);
+    uint64_t p = fma2(f2(kExp2C3, kExp2C3), fr, f2(kExp2C2, kExp2C2));
+    p = fma2(p, fr, f2(kExp2C1, kExp2C1));
+    p = fma2(p, fr, f2(kExp2C0, kExp2C0));
+    float t0, t1, p0, p1;
+    f2_split(t, t0, t1);
+    f2_split(p, p0, p1);
+    a = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+    b = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
 // Row t of the bitmap: bit s of word s / 32 is set iff s is in S(t) (for the
 // query at position p = S - T + t): the top-K entries <= p - W and the window
 // {max(0, p-W+1) .. p}.  Built in shared memory, written whole (zeros past p).
@@ -449,10 +477,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     float a, b;
-                    f2_split(fma2(f2(__uint_as_float(v[c + 2 * i]), __uint_as_float(v[c + 2 * i + 1])), sl2x2, nbx2),
-                             a, b);
-                    a = ex2(a);
-                    b = ex2(b);
+                    const uint64_t y =
+                        fma2(f2(__uint_as_float(v[c + 2 * i]), __uint_as_float(v[c + 2 * i + 1])), sl2x2, nbx2);
+                    if ((i & 7) == 7) {   // one pair in eight on the FMA pipe, the rest on the ex2 unit
+                        exp2_pair_fma(y, a, b);
+                    } else {
+                        f2_split(y, a, b);
+                        a = ex2(a);
+                        b = ex2(b);
+                    }
                     l2 = add2(l2, f2(a, b));
                     pk[i] = pack_bf16(a, b);
                 }
@@ -469,7 +502,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             float la, lb;
             f2_split(l2, la, lb);
             const float l = la + lb;
-            const float inv = l > 0.f ? 1.f / l : 0.f;
+            // no selected key at all leaves the maximum at -inf (l then only holds
+            // the polynomial's floor values of masked keys)
+            const bool any = m_used != -CUDART_INF_F;
+            const float inv = any && l > 0.f ? 1.f / l : 0.f;
             const int t = t0 + qi;
             uint16_t *orow = P.out + ((int64_t)t * HQ + h) * D;
 #pragma unroll
@@ -488,7 +524,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
             }
             if (act && P.lse)
-                P.lse[(int64_t)t * HQ + h] = (l > 0.f ? m_used + __log2f(l) : -CUDART_INF_F) * 0.69314718055994531f;
+                P.lse[(int64_t)t * HQ + h] = (any && l > 0.f ? m_used + __log2f(l) : -CUDART_INF_F) * 0.69314718055994531f;
         }
         tc_fence_before();
         named_sync(1, kTcThreads);   // TMEM is freed by warp 0 after this
