@@ -17,8 +17,9 @@
 //     the remaining passes are skipped;
 //   * the K-th key tau (to the resolved precision) is then known, together
 //     with how many keys equal to it must be taken (the lowest-positioned);
-//   * ordered compaction: warp ballots count "> tau" and "== tau" keys in
-//     column order, a scan over warps and over the cluster's CTAs gives every
+//   * ordered compaction: each warp counts "> tau" and "== tau" keys of its
+//     span in column order (4 keys per lane per step, both counts packed in
+//     one word), a scan over lanes, warps and the cluster's CTAs gives every
 //     kept key its output slot, so the output comes out ascending.
 #include "internal.h"
 #include "ptx.cuh"
@@ -66,10 +67,22 @@ __device__ __forceinline__ void find_threshold(uint32_t *hl, uint32_t *hsum, uin
         cluster_sync();   // every slice has reached every CTA
         h = hsum;
     }
-    // thread i owns bins BINS-1-PER*i .. BINS-PER*i (scanned from the top down)
+    // thread i owns bins BINS-1-PER*i .. BINS-PER*i (scanned from the top down),
+    // read as PER/4 16-byte vectors
+    static_assert(PER % 4 == 0 || PER == 2, "bins per thread");
     uint32_t cnt[PER], lsum = 0;
+    if constexpr (PER % 4 == 0) {
 #pragma unroll
-    for (int k = 0; k < PER; ++k) { cnt[k] = h[BINS - 1 - PER * tid - k]; lsum += cnt[k]; }
+        for (int q4 = 0; q4 < PER / 4; ++q4) {
+            const uint4 b = reinterpret_cast<const uint4 *>(h + BINS - PER * (tid + 1))[PER / 4 - 1 - q4];
+            cnt[4 * q4 + 0] = b.w; cnt[4 * q4 + 1] = b.z; cnt[4 * q4 + 2] = b.y; cnt[4 * q4 + 3] = b.x;
+        }
+    } else {
+        const uint2 b = reinterpret_cast<const uint2 *>(h + BINS - PER * (tid + 1))[0];
+        cnt[0] = b.y; cnt[1] = b.x;
+    }
+#pragma unroll
+    for (int k = 0; k < PER; ++k) lsum += cnt[k];
     uint32_t incl = lsum;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -78,17 +91,9 @@ __device__ __forceinline__ void find_threshold(uint32_t *hl, uint32_t *hsum, uin
     }
     if (lane == 31) scan_tmp[warp] = incl;
     __syncthreads();
-    if (warp == 0) {
-        uint32_t t = lane < kTopkWarps ? scan_tmp[lane] : 0u, x = t;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t v = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += v;
-        }
-        if (lane < kTopkWarps) scan_tmp[32 + lane] = x - t;   // exclusive warp offsets
-    }
-    __syncthreads();
-    const uint32_t excl = scan_tmp[32 + warp] + incl - lsum;
+    // bins above this warp's: the totals of the warps before it
+    const uint32_t wexcl = __reduce_add_sync(0xffffffffu, lane < warp ? scan_tmp[lane] : 0u);
+    const uint32_t excl = wexcl + incl - lsum;
     if (excl < need && need <= excl + lsum) {
         uint32_t acc = excl;
 #pragma unroll
@@ -116,7 +121,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     uint32_t *hsum = (G > 1) ? hist0 + kBinsA : nullptr;
     __shared__ uint32_t scan_tmp[64];
     __shared__ uint32_t sel[3];
-    __shared__ uint32_t warp_gt[kTopkWarps], warp_eq[kTopkWarps];
+    __shared__ uint32_t warp_gt[kTopkWarps];   // packed per-warp counts
     __shared__ uint32_t cta_counts[2];
 
     const int r = blockIdx.x / G;
@@ -219,51 +224,81 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     }
     const uint32_t tau = prefix, tmask = mask;   // keep: (u&tmask) > tau, and `need` of (u&tmask) == tau
 
-    // ---- ordered compaction
-    const int sub = ((len + kTopkThreads - 1) / kTopkThreads) * 32;   // per-warp span, multiple of 32
+    // ---- ordered compaction.  Warp w owns keys [w0, w0 + sub) of the chunk and
+    // visits them 128 at a time, 4 consecutive keys per lane; per-lane counts
+    // of "> tau" (low 16 bits) and "== tau" (high 16 bits) are packed into one
+    // word, so one warp sum or scan handles both (a CTA holds < 65536 keys).
+    const int sub = ((len + 4 * kTopkThreads - 1) / (4 * kTopkThreads)) * 128;
     const int w0 = warp * sub, w1 = min(w0 + sub, len);
-    uint32_t gt = 0, eq = 0;
-    for (int i = w0 + lane; i < w0 + sub; i += 32) {
-        const bool valid = i < w1;
-        const uint32_t u = valid ? (keys[i] & tmask) : 0u;
-        gt += __popc(__ballot_sync(0xffffffffu, valid && u > tau));
-        eq += __popc(__ballot_sync(0xffffffffu, valid && u == tau));
-    }
-    if (lane == 0) { warp_gt[warp] = gt; warp_eq[warp] = eq; }
-    __syncthreads();
-    if (tid == 0) {
-        uint32_t g = 0, e = 0;
-        for (int w = 0; w < kTopkWarps; ++w) {
-            const uint32_t tg = warp_gt[w], te = warp_eq[w];
-            warp_gt[w] = g; warp_eq[w] = e;
-            g += tg; e += te;
+    auto load4 = [&](int p, uint32_t (&u)[4]) {
+        if (p + 3 < w1) {
+            const uint4 k = reinterpret_cast<const uint4 *>(keys)[p >> 2];
+            u[0] = k.x; u[1] = k.y; u[2] = k.z; u[3] = k.w;
+        } else {   // the ragged end of the span (or past it)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) u[e] = p + e < w1 ? keys[p + e] : 0u;
         }
-        cta_counts[0] = g; cta_counts[1] = e;
+    };
+    auto count4 = [&](int p, uint32_t (&u)[4]) -> uint32_t {
+        uint32_t c = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            u[e] &= tmask;
+            const bool valid = p + e < w1;
+            c += (valid && u[e] > tau) ? 1u : 0u;
+            c += (valid && u[e] == tau) ? 0x10000u : 0u;
+        }
+        return c;
+    };
+    uint32_t wtot = 0;
+    for (int j = w0; j < w0 + sub; j += 128) {
+        uint32_t u[4];
+        load4(j + 4 * lane, u);
+        wtot += __reduce_add_sync(0xffffffffu, count4(j + 4 * lane, u));
     }
+    if (lane == 0) warp_gt[warp] = wtot;
     __syncthreads();
+    const uint32_t wbase = __reduce_add_sync(0xffffffffu, lane < warp ? warp_gt[lane] : 0u);   // warps before
+    if (tid == kTopkThreads - 1) {
+        cta_counts[0] = (wbase + wtot) & 0xFFFFu;
+        cta_counts[1] = (wbase + wtot) >> 16;
+    }
     uint32_t base_gt = 0, base_eq = 0;
     if (G > 1) {
-        cluster_sync();
+        cluster_sync();   // every CTA's totals are written
         for (uint32_t c = 0; c < rank; ++c) {
             base_gt += dsmem_ld_u32(&cta_counts[0], c);
             base_eq += dsmem_ld_u32(&cta_counts[1], c);
         }
     }
-    uint32_t run_gt = base_gt + warp_gt[warp], run_eq = base_eq + warp_eq[warp];
-    const uint32_t lt = lanemask_lt();
-    for (int i = w0 + lane; i < w0 + sub; i += 32) {
-        const bool valid = i < w1;
-        const uint32_t u = valid ? (keys[i] & tmask) : 0u;
-        const bool is_gt = valid && u > tau, is_eq = valid && u == tau;
-        const uint32_t bg = __ballot_sync(0xffffffffu, is_gt), be = __ballot_sync(0xffffffffu, is_eq);
-        const uint32_t gt_before = run_gt + __popc(bg & lt), eq_before = run_eq + __popc(be & lt);
-        if (is_gt || (is_eq && eq_before < need)) {
-            const uint32_t slot = gt_before + min(eq_before, need);
-            const int col = c0 + i;
-            out[slot] = cand ? cand[col] : col;
+    uint32_t run = wbase;   // packed counts before the current 128-key group of this warp
+    for (int j = w0; j < w0 + sub; j += 128) {
+        uint32_t u[4];
+        const int p = j + 4 * lane;
+        load4(p, u);
+        const uint32_t c = count4(p, u);
+        uint32_t incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
         }
-        run_gt += __popc(bg);
-        run_eq += __popc(be);
+        if (c != 0u) {   // this lane keeps or ties at least one of its keys
+            const uint32_t before = run + incl - c;
+            uint32_t gt_before = base_gt + (before & 0xFFFFu), eq_before = base_eq + (before >> 16);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const bool valid = p + e < w1;
+                const bool is_gt = valid && u[e] > tau, is_eq = valid && u[e] == tau;
+                if (is_gt || (is_eq && eq_before < need)) {
+                    const int col = c0 + p + e;
+                    out[gt_before + min(eq_before, need)] = cand ? cand[col] : col;
+                }
+                gt_before += is_gt ? 1u : 0u;
+                eq_before += is_eq ? 1u : 0u;
+            }
+        }
+        run += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (G > 1) cluster_sync();   // peers may still read this CTA's counters
 }
