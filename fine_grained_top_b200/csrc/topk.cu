@@ -163,34 +163,28 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     }
 
     // ---- load the chunk as order-preserving keys, counting the top 12 bits
-    for (int i = tid; i < kBinsA; i += kTopkThreads) hist0[i] = 0u;
+    for (int i = tid; i < kBinsA / 4; i += kTopkThreads) reinterpret_cast<uint4 *>(hist0)[i] = make_uint4(0u, 0u, 0u, 0u);
     __syncthreads();
     {
         const int len4 = len >> 2;   // c0 and ld are multiples of 4, base 16-byte aligned
         const float4 *src4 = reinterpret_cast<const float4 *>(row + c0);
-        constexpr int U = 4;         // loads in flight per thread
-        for (int base = 0; base < len4; base += U * kTopkThreads) {
-            float4 f[U];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int i = base + u * kTopkThreads + tid;
-                if (i < len4) f[u] = __ldg(src4 + i);
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int i = base + u * kTopkThreads + tid;
-                if (i < len4) {
-                    uint4 k;
-                    k.x = order_key(f[u].x); k.y = order_key(f[u].y);
-                    k.z = order_key(f[u].z); k.w = order_key(f[u].w);
-                    reinterpret_cast<uint4 *>(keys)[i] = k;
-                    atomicAdd(&hist0[k.x >> 20], 1u);
-                    atomicAdd(&hist0[k.y >> 20], 1u);
-                    atomicAdd(&hist0[k.z >> 20], 1u);
-                    atomicAdd(&hist0[k.w >> 20], 1u);
-                }
-            }
+        auto put = [&](int i, const float4 &f) {
+            uint4 k;
+            k.x = order_key(f.x); k.y = order_key(f.y);
+            k.z = order_key(f.z); k.w = order_key(f.w);
+            reinterpret_cast<uint4 *>(keys)[i] = k;
+            atomicAdd(&hist0[k.x >> 20], 1u);
+            atomicAdd(&hist0[k.y >> 20], 1u);
+            atomicAdd(&hist0[k.z >> 20], 1u);
+            atomicAdd(&hist0[k.w >> 20], 1u);
+        };
+        int i = tid;
+        for (; i + kTopkThreads < len4; i += 2 * kTopkThreads) {   // two 16-byte loads in flight
+            const float4 f0 = __ldg(src4 + i), f1 = __ldg(src4 + i + kTopkThreads);
+            put(i, f0);
+            put(i + kTopkThreads, f1);
         }
+        if (i < len4) put(i, __ldg(src4 + i));
         for (int i = (len4 << 2) + tid; i < len; i += kTopkThreads) {
             const uint32_t k = order_key(row[c0 + i]);
             keys[i] = k;
@@ -209,9 +203,17 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     for (int pass = 1; pass < 3 && !whole; ++pass) {
         const int shift = pass == 1 ? 10 : 0;
         uint32_t *hl = hist0;
-        for (int i = tid; i < 1024; i += kTopkThreads) hl[i] = 0u;
+        if (tid < 256) reinterpret_cast<uint4 *>(hl)[tid] = make_uint4(0u, 0u, 0u, 0u);
         __syncthreads();
-        for (int i = tid; i < len; i += kTopkThreads) {
+        const int len4 = len >> 2;
+        for (int i = tid; i < len4; i += kTopkThreads) {
+            const uint4 k = reinterpret_cast<const uint4 *>(keys)[i];
+            if ((k.x & mask) == prefix) atomicAdd(&hl[(k.x >> shift) & 1023u], 1u);
+            if ((k.y & mask) == prefix) atomicAdd(&hl[(k.y >> shift) & 1023u], 1u);
+            if ((k.z & mask) == prefix) atomicAdd(&hl[(k.z >> shift) & 1023u], 1u);
+            if ((k.w & mask) == prefix) atomicAdd(&hl[(k.w >> shift) & 1023u], 1u);
+        }
+        for (int i = (len4 << 2) + tid; i < len; i += kTopkThreads) {
             const uint32_t u = keys[i];
             if ((u & mask) == prefix) atomicAdd(&hl[(u >> shift) & 1023u], 1u);
         }
