@@ -241,22 +241,27 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
             for (int e = 0; e < 4; ++e) u[e] = p + e < w1 ? keys[p + e] : 0u;
         }
     };
-    auto count4 = [&](int p, uint32_t (&u)[4]) -> uint32_t {
-        uint32_t c = 0;
+    // per lane and 128-key group: bits 0..3 "key e > tau", bits 4..7 "key e == tau",
+    // kept for the write sweep in the first histogram's storage (free by now)
+    uint32_t *flags = hist0 + warp * (sub / 4);   // sub / 128 groups x 32 lanes per warp
+    auto flags4 = [&](int p, uint32_t (&u)[4]) -> uint32_t {
+        uint32_t f = 0;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            u[e] &= tmask;
+            const uint32_t k = u[e] & tmask;
             const bool valid = p + e < w1;
-            c += (valid && u[e] > tau) ? 1u : 0u;
-            c += (valid && u[e] == tau) ? 0x10000u : 0u;
+            f |= (valid && k > tau) ? (1u << e) : 0u;
+            f |= (valid && k == tau) ? (16u << e) : 0u;
         }
-        return c;
+        return f;
     };
     uint32_t wtot = 0;
-    for (int j = w0; j < w0 + sub; j += 128) {
+    for (int j = w0, g = 0; j < w0 + sub; j += 128, ++g) {
         uint32_t u[4];
         load4(j + 4 * lane, u);
-        wtot += __reduce_add_sync(0xffffffffu, count4(j + 4 * lane, u));
+        const uint32_t f = flags4(j + 4 * lane, u);
+        flags[g * 32 + lane] = f;
+        wtot += __reduce_add_sync(0xffffffffu, (uint32_t)__popc(f & 15u) + ((uint32_t)__popc(f >> 4) << 16));
     }
     if (lane == 0) warp_gt[warp] = wtot;
     __syncthreads();
@@ -274,24 +279,22 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
         }
     }
     uint32_t run = wbase;   // packed counts before the current 128-key group of this warp
-    for (int j = w0; j < w0 + sub; j += 128) {
-        uint32_t u[4];
+    for (int j = w0, g = 0; j < w0 + sub; j += 128, ++g) {
         const int p = j + 4 * lane;
-        load4(p, u);
-        const uint32_t c = count4(p, u);
+        const uint32_t f = flags[g * 32 + lane];
+        const uint32_t c = (uint32_t)__popc(f & 15u) + ((uint32_t)__popc(f >> 4) << 16);
         uint32_t incl = c;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += t;
         }
-        if (c != 0u) {   // this lane keeps or ties at least one of its keys
+        if (f != 0u) {   // this lane keeps or ties at least one of its keys
             const uint32_t before = run + incl - c;
             uint32_t gt_before = base_gt + (before & 0xFFFFu), eq_before = base_eq + (before >> 16);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const bool valid = p + e < w1;
-                const bool is_gt = valid && u[e] > tau, is_eq = valid && u[e] == tau;
+                const bool is_gt = (f >> e) & 1u, is_eq = (f >> (4 + e)) & 1u;
                 if (is_gt || (is_eq && eq_before < need)) {
                     const int col = c0 + p + e;
                     out[gt_before + min(eq_before, need)] = cand ? cand[col] : col;
