@@ -20,9 +20,10 @@
 // Warp roles (persistent CTAs, one per SM):
 //   warp 0     TMA producer (one elected lane) + TMEM allocator
 //   warp 1     MMA issuer (one elected lane): tcgen05.mma kind::f16
-//   warps 2..  epilogue teams: 2 column groups x 2 TMEM accumulators for the
-//              256-column prefill tile; 4 item groups x 8 accumulators for the
-//              16-column decode tile (several items drain at once)
+//   warps 2..  epilogue teams: for the 256-column prefill tile, 2 item groups
+//              (alternate items, one TMEM accumulator each) x 2 column groups;
+//              for the 16-column decode tile, 4 item groups x 8 accumulators
+//              (several items drain at once)
 // All roles classify the CTA's items 32 at a time (one item per lane) and
 // walk the same sequence of non-empty items; the producer resolves the page
 // ids of 32 items in parallel, off the TMA issue path.
@@ -59,7 +60,7 @@ struct IdxCfg {
     // Epilogue teams: CG column groups split one item's queries; IG item
     // groups take alternate items so that several accumulators drain at once.
     static constexpr int kCG = (N == 256) ? 2 : 1;
-    static constexpr int kIG = (N == 256) ? 1 : 4;
+    static constexpr int kIG = (N == 256) ? 2 : 4;
     static constexpr int kAcc = (N == 256) ? 2 : 8;           // TMEM accumulators (multiple of kIG)
     static constexpr int kEpiWarps = 4 * kCG * kIG;
     static constexpr int kThreads = (2 + kEpiWarps) * 32;
