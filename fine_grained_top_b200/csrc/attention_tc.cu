@@ -46,7 +46,8 @@ namespace {
 
 constexpr int kTile = 128;                  // keys per tile
 constexpr int kTcThreads = 10 * 32;
-constexpr int kBitmapThreads = 256;
+constexpr int kBitmapThreads = 256;        // up to 4 rows of the selection bitmap per CTA
+constexpr int kBitmapRowThreads = 64;
 constexpr size_t kSmemLimit = 232448;       // opt-in dynamic shared memory per CTA
 
 struct TcParams {
@@ -194,38 +195,61 @@ __device__ __forceinline__ void exp2_pair_fma(uint64_t y, float &a, float &b) {
 // query at position p = S - T + t): the top-K entries <= p - W and the window
 // {max(0, p-W+1) .. p}.  Built in shared memory, written whole (zeros past p).
 // Entries beyond p are reported (SA_DEV_INDEX) and skipped; a row that is not
-// strictly ascending before its -1 padding sets SA_DEV_ORDER.
+// strictly ascending before its -1 padding sets SA_DEV_ORDER.  64 threads
+// build one row; a CTA holds blockDim.x / 64 rows.
 __global__ void __launch_bounds__(kBitmapThreads) selection_bitmap_kernel(const int32_t *topk, int K, int W, int T,
                                                                           int S, int words, uint32_t *bitmap,
                                                                           int *dev_status) {
-    extern __shared__ uint32_t rowbits[];   // [words]
-    const int t = blockIdx.x;
-    const int p = S - T + t;
-    for (int i = threadIdx.x; i < words; i += kBitmapThreads) rowbits[i] = 0u;
+    extern __shared__ uint4 bits4[];   // [rows per CTA][words / 4]
+    const int rows = (int)blockDim.x / kBitmapRowThreads;
+    const int sub = (int)threadIdx.x / kBitmapRowThreads, lt = (int)threadIdx.x % kBitmapRowThreads;
+    const int t = (int)blockIdx.x * rows + sub;
+    const bool live = t < T;
+    uint32_t *rowbits = reinterpret_cast<uint32_t *>(bits4) + (size_t)sub * words;
+    if (live)
+        for (int i = lt; i < words / 4; i += kBitmapRowThreads)
+            reinterpret_cast<uint4 *>(rowbits)[i] = make_uint4(0u, 0u, 0u, 0u);
     __syncthreads();
-    const int32_t *row = topk + (int64_t)t * K;
     bool bad_idx = false, bad_ord = false;
-    for (int i = threadIdx.x; i < K; i += kBitmapThreads) {
-        const int e = __ldg(row + i);
-        if (e < 0) continue;
-        if (i > 0) {
-            const int prev = __ldg(row + i - 1);
-            if (!(prev >= 0 && prev < e)) bad_ord = true;
+    if (live) {
+        const int p = S - T + t;
+        const int32_t *row = topk + (int64_t)t * K;
+        auto take = [&](int i, int e, int prev) {   // entry i holds e; prev is entry i - 1
+            if (e < 0) return;
+            if (i > 0 && !(prev >= 0 && prev < e)) bad_ord = true;
+            if (e > p) {
+                bad_idx = true;
+                return;
+            }
+            if (e <= p - W) atomicOr(&rowbits[e >> 5], 1u << (e & 31));
+        };
+        if ((K & 3) == 0 && (reinterpret_cast<uintptr_t>(topk) & 15u) == 0) {
+            const int4 *row4 = reinterpret_cast<const int4 *>(row);
+            for (int i4 = lt; i4 < K / 4; i4 += kBitmapRowThreads) {
+                const int4 v = __ldg(row4 + i4);
+                const int prev = i4 > 0 ? __ldg(row + 4 * i4 - 1) : 0;
+                take(4 * i4, v.x, prev);
+                take(4 * i4 + 1, v.y, v.x);
+                take(4 * i4 + 2, v.z, v.y);
+                take(4 * i4 + 3, v.w, v.z);
+            }
+        } else {
+            for (int i = lt; i < K; i += kBitmapRowThreads) take(i, __ldg(row + i), i > 0 ? __ldg(row + i - 1) : 0);
         }
-        if (e > p) { bad_idx = true; continue; }
-        if (e <= p - W) atomicOr(&rowbits[e >> 5], 1u << (e & 31));
+        const int w0 = max(0, p - W + 1);
+        for (int wi = (w0 >> 5) + lt; wi <= (p >> 5) && W > 0; wi += kBitmapRowThreads) {
+            const int lo = max(w0, wi * 32), hi = min(p, wi * 32 + 31);
+            const int n = hi - lo + 1;
+            atomicOr(&rowbits[wi], (n == 32) ? 0xffffffffu : (((1u << n) - 1u) << (lo - wi * 32)));
+        }
     }
     if (bad_idx) report(dev_status, SA_DEV_INDEX);
     if (bad_ord) report(dev_status, SA_DEV_ORDER);
-    const int w0 = max(0, p - W + 1);
-    for (int wi = (w0 >> 5) + (int)threadIdx.x; wi <= (p >> 5) && W > 0; wi += kBitmapThreads) {
-        const int a = max(w0, wi * 32), b = min(p, wi * 32 + 31);
-        const int n = b - a + 1;
-        atomicOr(&rowbits[wi], (n == 32) ? 0xffffffffu : (((1u << n) - 1u) << (a - wi * 32)));
-    }
     __syncthreads();
-    uint32_t *dst = bitmap + (int64_t)t * words;
-    for (int i = threadIdx.x; i < words; i += kBitmapThreads) dst[i] = rowbits[i];
+    if (live) {
+        uint4 *dst = reinterpret_cast<uint4 *>(bitmap + (int64_t)t * words);
+        for (int i = lt; i < words / 4; i += kBitmapRowThreads) dst[i] = reinterpret_cast<const uint4 *>(rowbits)[i];
+    }
 }
 
 template <int D, int HQ>
@@ -587,10 +611,12 @@ sa_status launch_tc(const PrefillArgs &a, cudaStream_t st) {
     if (!map_rows(&mq, a.q, (uint64_t)a.T * HQ, D) || !map_rows(&mk, a.k, (uint64_t)a.S, D) ||
         !map_rows(&mv, a.v, (uint64_t)a.S, D) || !map_bitmap(&mm, bitmap, (uint64_t)a.T, words, 2 * GQ))
         return SA_ERR_CUDA;
-    const size_t bsmem = (size_t)words * 4;
+    // 4 rows per CTA while their bitmap rows fit in 48 KB, else one
+    const int brows = (size_t)words * 4 * 4 <= 48 * 1024 ? 4 : 1;
+    const size_t bsmem = (size_t)words * 4 * brows;
     if (prepare_kernel<selection_bitmap_kernel>(bsmem, false) != cudaSuccess) return SA_ERR_CUDA;
-    selection_bitmap_kernel<<<a.T, kBitmapThreads, bsmem, st>>>(a.topk, a.K, a.W, a.T, a.S, words, bitmap,
-                                                               a.dev_status);
+    selection_bitmap_kernel<<<(a.T + brows - 1) / brows, kBitmapRowThreads * brows, bsmem, st>>>(
+        a.topk, a.K, a.W, a.T, a.S, words, bitmap, a.dev_status);
     if (prepare_kernel<masked_attn_tc_kernel<D, HQ>>(C::kSmem, false) != cudaSuccess) return SA_ERR_CUDA;
     masked_attn_tc_kernel<D, HQ><<<p.n_groups, kTcThreads, C::kSmem, st>>>(mq, mk, mv, mm, p);
     return cuda_ok(cudaGetLastError());

@@ -325,6 +325,8 @@ __global__ void __launch_bounds__(IdxCfg<N, D_I>::kThreads, 1)
                 const uint32_t t_cols = tmem_base + ((uint32_t)(quad * 32) << 16) +
                                         (uint32_t)(acc * N + cg * C::kGroupCols);
                 float *op = a.scores + row0 * a.ld + s;
+                const bool causal = a.n_valid == nullptr;
+                const int causal_end = a.S - a.T + t_base + 1;   // row length of query q: causal_end + q
 #pragma unroll
                 for (int l0 = 0; l0 < NLD; l0 += BATCH) {
                     uint32_t v[BATCH][16];
@@ -352,7 +354,8 @@ __global__ void __launch_bounds__(IdxCfg<N, D_I>::kThreads, 1)
 #pragma unroll
                                 for (int j1 = 0; j1 < H_I; ++j1)
                                     sc = fmaf(wv[j1], fmaxf(__uint_as_float(v[bb][qq * H_I + j1]), 0.f), sc);
-                                if (s < nvs[q]) *op = sc;
+                                // causal rows (no n_valid) end at their own position
+                                if (causal ? s < causal_end + q : s < nvs[q]) *op = sc;
                             }
                             op += a.ld;
                         }
