@@ -87,35 +87,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
-// Non-blocking test of the phase with the given parity (never suspends).
-__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{ .reg .pred p; mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-// mbar_wait for latency-critical hand-offs: polls with test_wait instead of
-// letting try_wait suspend the thread, so the phase is seen within a few
-// cycles of completing.  Same bound and abort protocol as mbar_wait.
-__device__ __forceinline__ bool mbar_wait_spin(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                               unsigned long long limit_ns = kWaitLimitNs) {
-    if (mbar_test_wait(bar, parity)) return true;
-    const unsigned long long t0 = globaltimer();
-    while (true) {
-        for (int i = 0; i < 64; ++i)
-            if (mbar_test_wait(bar, parity)) return true;
-        if (*abort) return false;
-        if (globaltimer() - t0 > limit_ns) {
-            *abort = 1;
-            return false;
-        }
-    }
-}
-
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
