@@ -7,6 +7,8 @@ library's kernels on one stream; the host does no arithmetic of the method.
                    sequence (optionally the two-stage coarse/fine selection)
     DecodePlan     one new query per sequence over a contiguous or paged
                    KV cache: indexer -> top-K -> split-K attention + merge
+    HostPipeline   steps fed from and read back to pinned host memory, the
+                   copies of neighbouring steps overlapped with the kernels
 
 ``stages(inputs)`` returns the step as a list of (name, launch) pairs, one
 per C-ABI call, so that callers can time each kernel; ``run`` executes them.
@@ -152,3 +154,67 @@ class DecodePlan:
 
     def launches(self) -> int:
         return 4   # indexer, top-K, split attention, merge
+
+
+class HostPipeline:
+    """Steps whose inputs come from pinned host memory and whose output goes
+    back to pinned host memory, with the copies running under the kernels.
+
+    Two plans (two sets of device buffers) alternate.  Step i uploads its
+    inputs into set i % 2 on an upload stream, runs the path on the compute
+    stream and downloads the plan's output on a download stream.  Its upload
+    waits only for step i - 2's compute (the set's previous reader), and its
+    compute waits for its own upload and for step i - 2's download (the set's
+    previous output).  So step i + 1's upload and step i - 1's download overlap
+    step i's kernels, and each step still moves all of its own bytes.
+
+    make_plan: () -> a PrefillPlan / DecodePlan (anything with .stages and .out)
+    host_inputs: name -> pinned host tensor, the shapes and dtypes of one step's inputs
+    resident: name -> device tensor that every step reads in place (e.g. a KV cache)
+    """
+
+    def __init__(self, make_plan, host_inputs, resident=None, device="cuda"):
+        dev = torch.device(device)
+        self.plans = [make_plan(), make_plan()]
+        self.inputs = []
+        for _ in range(2):
+            x = {k: torch.empty(v.shape, dtype=v.dtype, device=dev) for k, v in host_inputs.items()}
+            x.update(resident or {})
+            self.inputs.append(x)
+        self.up, self.comp, self.down = (torch.cuda.Stream(device=dev) for _ in range(3))
+        self.stages = [p.stages(x, self.comp) for p, x in zip(self.plans, self.inputs)]
+        ev = lambda: [torch.cuda.Event(), torch.cuda.Event()]
+        self.up_done, self.comp_done, self.down_done = ev(), ev(), ev()
+        self.used = [False, False]
+
+    def run(self, step_inputs, step_outputs, before_compute=None):
+        """step_inputs[i]: name -> pinned host tensor; step_outputs[i]: pinned host
+        tensor shaped like plan.out.  before_compute(i), if given, runs on the
+        compute stream ahead of step i's kernels.  Returns without waiting;
+        synchronize (or wait on self.down) before reading the outputs."""
+        for i, (hin, hout) in enumerate(zip(step_inputs, step_outputs)):
+            b = i % 2
+            with torch.cuda.stream(self.up):
+                if self.used[b]:
+                    self.up.wait_event(self.comp_done[b])
+                for k, t in hin.items():
+                    self.inputs[b][k].copy_(t, non_blocking=True)
+                self.up_done[b].record(self.up)
+            with torch.cuda.stream(self.comp):
+                self.comp.wait_event(self.up_done[b])
+                if self.used[b]:
+                    self.comp.wait_event(self.down_done[b])
+                if before_compute is not None:
+                    before_compute(i)
+                for _, fn in self.stages[b]:
+                    fn()
+                self.comp_done[b].record(self.comp)
+            with torch.cuda.stream(self.down):
+                self.down.wait_event(self.comp_done[b])
+                hout.copy_(self.plans[b].out, non_blocking=True)
+                self.down_done[b].record(self.down)
+            self.used[b] = True
+
+    def dev_status(self) -> int:
+        """OR of both plans' device status words (synchronizes)."""
+        return int(self.plans[0].dev_status.item()) | int(self.plans[1].dev_status.item())

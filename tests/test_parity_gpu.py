@@ -213,6 +213,29 @@ def _prefill_e2e(sa, inp, K, W, rows=None, block=None, keep=None):
     return plan, ref
 
 
+def test_host_pipeline_matches_direct_runs(sa):
+    # three steps with different inputs through the overlapped host-buffer
+    # runner: each downloaded output equals a direct run of the plan
+    from fine_grained_top_b200.pipeline import HostPipeline
+    PrefillPlan, _ = _pl()
+    c = CONFIGS["prefill_512"]
+    names = ("q", "k", "v", "qI", "w", "kI")
+    steps = [gen_prefill(seed=s, **c) for s in (0, 1, 2)]
+    hin = [{n: dev(st[n]).cpu().pin_memory() for n in names} for st in steps]
+    make = lambda: PrefillPlan(c["N"], c["Hq"], c["d"], c["H_I"], c["D_I"], c["K"], c["W"])
+    pipe = HostPipeline(make, hin[0])
+    outs = [torch.empty((c["N"], c["Hq"], c["d"]), dtype=torch.bfloat16).pin_memory() for _ in steps]
+    pipe.run(hin, outs)
+    torch.cuda.synchronize()
+    assert pipe.dev_status() == 0
+    for st, o in zip(steps, outs):
+        plan = make()
+        t = _to_dev(st)
+        plan.run(t["q"], t["k"], t["v"], t["qI"], t["w"], t["kI"])
+        assert torch.equal(o, plan.out.cpu())
+    assert not torch.equal(outs[0], outs[1])
+
+
 def test_e2e_prefill_512(sa):
     c = CONFIGS["prefill_512"]
     _prefill_e2e(sa, config_inputs("prefill_512"), c["K"], c["W"])
