@@ -123,6 +123,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     __shared__ uint32_t sel[3];
     __shared__ uint32_t warp_gt[kTopkWarps];   // packed per-warp counts
     __shared__ uint32_t cta_counts[2];
+    __shared__ uint32_t low_bits[2];   // OR, AND of the last digit over the first refinement's keys
 
     const int r = blockIdx.x / G;
     const uint32_t rank = (G > 1) ? cluster_rank() : 0u;
@@ -198,24 +199,45 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     uint32_t prefix = sel[0] << 20, mask = 0xFFF00000u;
     need -= sel[1];
     bool whole = sel[2] == need;        // the threshold bin is taken entirely
-    // two 10-bit refinements over the keys that match the prefix
+    // two 10-bit refinements over the keys that match the prefix.  A single-CTA
+    // row also takes, in the first, the OR and AND of the last digit (bits
+    // 9..0) over those keys: when they agree, every key of the bin shares its
+    // last digit and the second refinement is decided without a pass (keys with
+    // few mantissa bits, e.g. integer-valued or FP8-product scores).
 #pragma unroll 1
     for (int pass = 1; pass < 3 && !whole; ++pass) {
         const int shift = pass == 1 ? 10 : 0;
+        const bool track = G == 1 && pass == 1;
         uint32_t *hl = hist0;
         if (tid < 256) reinterpret_cast<uint4 *>(hl)[tid] = make_uint4(0u, 0u, 0u, 0u);
+        if (track && tid == 0) { low_bits[0] = 0u; low_bits[1] = 1023u; }
         __syncthreads();
+        uint32_t lor = 0u, land = 1023u;
+        auto count = [&](uint32_t u) {
+            if ((u & mask) == prefix) {
+                atomicAdd(&hl[(u >> shift) & 1023u], 1u);
+                if (track) {
+                    lor |= u & 1023u;
+                    land &= u & 1023u;
+                }
+            }
+        };
         const int len4 = len >> 2;
         for (int i = tid; i < len4; i += kTopkThreads) {
             const uint4 k = reinterpret_cast<const uint4 *>(keys)[i];
-            if ((k.x & mask) == prefix) atomicAdd(&hl[(k.x >> shift) & 1023u], 1u);
-            if ((k.y & mask) == prefix) atomicAdd(&hl[(k.y >> shift) & 1023u], 1u);
-            if ((k.z & mask) == prefix) atomicAdd(&hl[(k.z >> shift) & 1023u], 1u);
-            if ((k.w & mask) == prefix) atomicAdd(&hl[(k.w >> shift) & 1023u], 1u);
+            count(k.x);
+            count(k.y);
+            count(k.z);
+            count(k.w);
         }
-        for (int i = (len4 << 2) + tid; i < len; i += kTopkThreads) {
-            const uint32_t u = keys[i];
-            if ((u & mask) == prefix) atomicAdd(&hl[(u >> shift) & 1023u], 1u);
+        for (int i = (len4 << 2) + tid; i < len; i += kTopkThreads) count(keys[i]);
+        if (track) {
+            lor = __reduce_or_sync(0xffffffffu, lor);
+            land = __reduce_and_sync(0xffffffffu, land);
+            if (lane == 0) {
+                atomicOr(&low_bits[0], lor);
+                atomicAnd(&low_bits[1], land);
+            }
         }
         __syncthreads();
         find_threshold<G, 1024>(hl, hsum, need, scan_tmp, sel, tid);
@@ -223,6 +245,11 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
         mask |= 1023u << shift;
         need -= sel[1];
         whole = sel[2] == need;
+        if (track && !whole && low_bits[0] == low_bits[1]) {   // the last digit is the same for all
+            prefix |= low_bits[0];
+            mask = 0xFFFFFFFFu;
+            break;
+        }
     }
     const uint32_t tau = prefix, tmask = mask;   // keep: (u&tmask) > tau, and `need` of (u&tmask) == tau
 
