@@ -196,6 +196,33 @@ def test_prefill_attention_given_oracle_topk(sa, N, Hq, d, K, W, use_ws):
     assert np.max(np.abs(host_f64(lse) - l)) < 1e-3
 
 
+@pytest.mark.parametrize("use_ws", [False, True])
+def test_prefill_chunk_of_long_sequence(sa, use_ws):
+    # the last T queries of an S-token sequence (T < S); with use_ws the masked
+    # kernel runs and, at this S, its selection bitmap takes one row per CTA
+    S, T, Hq, d, K, W = 100000, 48, 4, 64, 2048, 64
+    inp = gen_prefill(N=S, Hq=Hq, d=d, H_I=2, D_I=32, seed=7)
+    pos = np.arange(S - T, S)
+    sc = oracle.indexer(inp["qI"][S - T:], inp["w"][S - T:], inp["kI"], pos)
+    top = oracle.topk(sc, pos + 1, K)
+    q = dev(np.ascontiguousarray(inp["q"][S - T:]))
+    t = _to_dev(inp, ("k", "v"))
+    out = torch.empty((T, Hq, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((T, Hq), dtype=torch.float32, device="cuda")
+    ds = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nb = sa.sa_prefill_workspace_bytes(T, S, K, W, Hq, d) if use_ws else 0
+    if use_ws:
+        assert nb > 0   # the shape qualifies for the masked kernel
+    ws = torch.empty(nb, dtype=torch.uint8, device="cuda") if nb else None
+    sa.sa_sparse_attn_prefill(q, t["k"], t["v"], dev(top.astype(np.int32)), K, W, T, S, Hq, d, 1 / math.sqrt(d),
+                              out, lse, ws, nb, ds)
+    ptr, idx = oracle.selection(top, W, pos)
+    o, l = oracle.sparse_attention(inp["q"][S - T:], inp["k"], inp["v"], ptr, idx, 1 / math.sqrt(d))
+    assert status(ds) == 0
+    assert_close_attention(host_f64(out), o, "out")
+    assert np.max(np.abs(host_f64(lse) - l)) < 1e-3
+
+
 # ====================================================================== end to end
 def _prefill_e2e(sa, inp, K, W, rows=None, block=None, keep=None):
     PrefillPlan, _ = _pl()
