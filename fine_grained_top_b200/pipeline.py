@@ -33,9 +33,12 @@ class PrefillPlan:
     """Buffers for one sequence of N tokens (queries at positions 0..N-1).
     Inputs: dict with q [N,Hq,d], k/v [N,d], qI [N,H_I,D_I], w [N,H_I], kI [N,D_I]."""
 
-    def __init__(self, N, Hq, d, H_I, D_I, K, W, block=None, keep=None, device="cuda"):
+    def __init__(self, N, Hq, d, H_I, D_I, K, W, block=None, keep=None, row_blocks=1, device="cuda"):
         self.N, self.Hq, self.d, self.H_I, self.D_I, self.K, self.W = N, Hq, d, H_I, D_I, K, W
         self.block, self.keep = block, keep
+        # single-stage only: score and select the queries in row_blocks blocks,
+        # so that a block's scores are still in L2 when top-K reads them
+        self.row_blocks = max(1, int(row_blocks)) if block is None else 1
         self.scale = 1.0 / math.sqrt(d)
         dev = torch.device(device)
         i32, f32 = torch.int32, torch.float32
@@ -73,6 +76,20 @@ class PrefillPlan:
         attn = ("attention", lambda: sa_sparse_attn_prefill(
             x["q"], x["k"], x["v"], self.topk, K, self.W, N, N, self.Hq, self.d, self.scale, self.out,
             self.lse, self.attn_ws, self.attn_ws_bytes, ds, stream))
+        if self.block is None and self.row_blocks > 1:
+            # queries t0..t1-1 are the last t1 - t0 of a t1-key causal sequence
+            bounds = [N * b // self.row_blocks for b in range(self.row_blocks + 1)]
+            out = []
+            for b in range(self.row_blocks):
+                t0, t1 = bounds[b], bounds[b + 1]
+                if t1 <= t0:
+                    continue
+                out.append(("indexer", lambda t0=t0, t1=t1: sa_indexer_scores(
+                    x["qI"][t0:t1], x["w"][t0:t1], x["kI"], None, 0, 0, 64, 1, t1 - t0, t1, H, D, None,
+                    self.scores[t0:t1], self.ld, ds, stream)))
+                out.append(("topk", lambda t0=t0, t1=t1: sa_topk_select(
+                    self.scores[t0:t1], self.ld, t1 - t0, t1, None, None, 0, K, self.topk[t0:t1], ds, stream)))
+            return out + [attn]
         if self.block is None:
             return [
                 ("indexer", lambda: sa_indexer_scores(x["qI"], x["w"], x["kI"], None, 0, 0, 64, 1, N, N, H, D,
@@ -106,7 +123,7 @@ class PrefillPlan:
     def launches(self) -> int:
         """Kernels one run() enqueues."""
         attn = 2 if self.attn_ws is not None else 1   # (selection bitmap +) attention
-        return (2 if self.block is None else 11) + attn
+        return (2 * self.row_blocks if self.block is None else 11) + attn
 
 
 class DecodePlan:

@@ -263,6 +263,22 @@ def test_host_pipeline_matches_direct_runs(sa):
     assert not torch.equal(outs[0], outs[1])
 
 
+def test_row_blocked_scoring_matches_whole(sa):
+    # scoring and selecting in row blocks gives the same step as one launch each
+    PrefillPlan, _ = _pl()
+    c = CONFIGS["prefill_512"]
+    inp = config_inputs("prefill_512")
+    t = _to_dev(inp)
+    plans = [PrefillPlan(c["N"], c["Hq"], c["d"], c["H_I"], c["D_I"], c["K"], c["W"], row_blocks=rb)
+             for rb in (1, 3)]
+    for p in plans:
+        p.run(t["q"], t["k"], t["v"], t["qI"], t["w"], t["kI"])
+        assert status(p.dev_status) == 0
+    assert torch.equal(plans[0].topk, plans[1].topk)
+    assert torch.equal(plans[0].out, plans[1].out)
+    assert plans[1].launches() == 2 * 3 + 1
+
+
 def test_e2e_prefill_512(sa):
     c = CONFIGS["prefill_512"]
     _prefill_e2e(sa, config_inputs("prefill_512"), c["K"], c["W"])
