@@ -9,6 +9,7 @@ package imports nothing from it; both take their inputs from ``workloads``.
 Functions (each cites the passage it follows in ``sa_oracle.c``):
 
 ``indexer``           I[t,s] = sum_j w[t,j] ReLU(qI[t,j].kI[s]), s <= lim[t]
+``e4m3_encode`` / ``e4m3_decode`` / ``indexer_fp8``  the FP8 operand format
 ``topk``              K best scores per row, ties -> lower position, ascending
 ``pool_mean``         mean of each complete block of index keys
 ``two_stage``         coarse block top-k, then fine top-K inside the blocks
@@ -58,6 +59,9 @@ def _load():
         lib = ctypes.CDLL(build())
         i64, i32 = ctypes.c_int64, ctypes.c_int
         lib.oracle_indexer.argtypes = [i64, i32, i32, i32, _f64p, _f64p, _f64p, _i64p, _f64p, i32]
+        _u8p = np.ctypeslib.ndpointer(dtype=np.uint8, flags="C_CONTIGUOUS")
+        lib.oracle_e4m3_encode.argtypes = [i64, _f64p, _u8p]
+        lib.oracle_e4m3_decode.argtypes = [i64, _u8p, _f64p]
         lib.oracle_topk.argtypes = [i64, i64, _f64p, _i64p, ctypes.c_void_p, i32, _i64p, i32]
         lib.oracle_pool_mean.argtypes = [i64, i32, i32, _f64p, _f64p]
         lib.oracle_two_stage.argtypes = [i64, _i64p, i32, i32, _f64p, _f64p, i64, _f64p,
@@ -99,6 +103,28 @@ def indexer(qI, w, kI, lim, S=None) -> np.ndarray:
     _load().oracle_indexer(R, S, H, D, qI.reshape(-1), w.reshape(-1),
                            np.ascontiguousarray(kI[:S]).reshape(-1), lim, out, threads())
     return out
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """Nearest OCP e4m3 code of each value (ties to even, +-448 saturation)."""
+    x = _f64(x)
+    out = np.empty(x.shape, dtype=np.uint8)
+    _load().oracle_e4m3_encode(x.size, np.ascontiguousarray(x).reshape(-1), out.reshape(-1))
+    return out
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Value of each e4m3 code (uint8) as a double."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(codes.shape, dtype=np.float64)
+    _load().oracle_e4m3_decode(codes.size, codes.reshape(-1), out.reshape(-1))
+    return out
+
+
+def indexer_fp8(qI_codes, w, kI_codes, lim, S=None) -> np.ndarray:
+    """The indexer over e4m3 operands: the same scores computed on the values
+    the codes hold (the FP8 indexer quantises its operands, nothing else)."""
+    return indexer(e4m3_decode(qI_codes), w, e4m3_decode(kI_codes), lim, S)
 
 
 # --------------------------------------------------------------------------

@@ -28,6 +28,12 @@
  *    "What Fine-Grained Means" (coarse block pass, then fine top-K inside the
  *    candidates) and section 2 "Learned Block Routing" (blocks mean-pooled
  *    over complete blocks, dot product, top-k).
+ *  - FP8 indexer operands: "Sparse Attention in 2026", "The designs that
+ *    shipped" (the lightning indexer is a small FP8 network).  The pages name
+ *    no FP8 layout; this file takes e4m3 as the OCP 8-bit float format defines
+ *    it (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, subnormals at
+ *    exponent field 0, no infinities, exponent 15 with mantissa 7 is NaN),
+ *    with round-to-nearest-even and saturation of finite overflow to +-448.
  *  - attention: "A Guide to Sparse Attention in Large Models" (Baidu),
  *    section 2: Attention = softmax(QK^T/sqrt(d)) V and its masked form
  *    softmax(QK^T * Mask + (1-Mask)(-inf)) V with Mask[i,j] = 1 iff j in S(i).
@@ -107,6 +113,48 @@ void oracle_indexer(int64_t R, int S, int H, int D, const double *qI,
                     double *out, int nthreads) {
     idx_ctx c = {S, H, D, qI, w, kI, lim, out};
     for_rows(R, nthreads, indexer_row, &c);
+}
+
+/* ------------------------------------------------------------------ */
+/* e4m3 (OCP FP8) values and codes                                     */
+/* ------------------------------------------------------------------ */
+/* The value of a code: (-1)^s * (1 + M/8) * 2^(E-7) for E > 0, and
+ * (-1)^s * (M/8) * 2^-6 for E = 0; E = 15, M = 7 is NaN. */
+static double e4m3_value(uint8_t c) {
+    const int s = c >> 7, E = (c >> 3) & 15, M = c & 7;
+    if (E == 15 && M == 7) return NAN;
+    const double v = (E == 0) ? ldexp((double)M, -9) : ldexp((double)(8 + M), E - 10);
+    return s ? -v : v;
+}
+
+/* The nearest code (ties to the even mantissa).  Within the binade
+ * [2^e, 2^(e+1)), e >= -6, the representable values are spaced 2^(e-3);
+ * below 2^-6 the subnormals keep the spacing 2^-9.  Counting the value in
+ * units of that spacing and rounding gives the code directly: a subnormal's
+ * code is its unit count, a normal's is (e+7)*8 + (units - 8), and a round-up
+ * to the next binade lands on that binade's first code. */
+static uint8_t e4m3_code(double x) {
+    if (isnan(x)) return signbit(x) ? 0xFF : 0x7F;
+    const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    const double a = fabs(x);
+    if (a >= 448.0) return sign | 0x7E;          /* largest finite value */
+    int e = -6;
+    if (a >= ldexp(1.0, -6)) {
+        int ex;
+        frexp(a, &ex);                           /* a = m 2^ex, m in [0.5, 1) */
+        e = ex - 1;
+    }
+    const double units = rint(ldexp(a, 3 - e));  /* exact scaling; rint: ties to even */
+    const int code = (e + 7) * 8 + (int)units - 8;
+    return sign | (uint8_t)code;
+}
+
+void oracle_e4m3_encode(int64_t n, const double *x, uint8_t *out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = e4m3_code(x[i]);
+}
+
+void oracle_e4m3_decode(int64_t n, const uint8_t *c, double *out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = e4m3_value(c[i]);
 }
 
 /* ------------------------------------------------------------------ */

@@ -110,6 +110,64 @@ def test_indexer_exact_integer_bound_on_workload_inputs():
     assert np.all(np.isneginf(sc[np.triu_indices(300, 1)]))
 
 
+# ---------------------------------------------------------------- e4m3 operands
+# The FP8 indexer reading: OCP e4m3, round to nearest even, +-448 saturation.
+def test_e4m3_decode_matches_torch_on_every_code():
+    torch = pytest.importorskip("torch")
+    codes = np.arange(256, dtype=np.uint8)
+    ours = oracle.e4m3_decode(codes)
+    lib = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(ours), np.isnan(lib))
+    assert np.array_equal(np.nonzero(np.isnan(ours))[0], [0x7F, 0xFF])
+    ok = ~np.isnan(ours)
+    assert np.array_equal(ours[ok], lib[ok])
+    assert np.array_equal(np.signbit(ours[ok]), np.signbit(lib[ok]))   # 0x80 is -0
+
+
+def test_e4m3_encode_matches_torch_inside_the_range():
+    torch = pytest.importorskip("torch")
+    r = np.random.default_rng(7)
+    # float32 values (so torch sees the same number), spread over every binade
+    # and the subnormals; |x| < 448, where torch's conversion does not saturate
+    x = (r.standard_normal(200000) * np.exp2(r.uniform(-12, 9, 200000))).astype(np.float32)
+    x = x[np.abs(x) < 448]
+    grid = oracle.e4m3_decode(np.arange(256, dtype=np.uint8))
+    grid = grid[np.isfinite(grid)]
+    mids = ((np.sort(grid)[1:] + np.sort(grid)[:-1]) / 2).astype(np.float32)   # every tie, exact in f32
+    x = np.concatenate([x, mids[np.abs(mids) < 448]])
+    lib = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e4m3_encode(x.astype(np.float64)), lib)
+
+
+def test_e4m3_round_trip_ties_and_saturation():
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    assert np.array_equal(oracle.e4m3_encode(oracle.e4m3_decode(codes)), codes)
+    cases = {1.0: 0x38, 1.0625: 0x38, 1.1875: 0x3A, 2.0 ** -9: 0x01, 2.0 ** -10: 0x00,
+             3 * 2.0 ** -10: 0x02, 2.0 ** -6: 0x08, 15 * 2.0 ** -10: 0x08, 448.0: 0x7E,
+             460.0: 0x7E, 1e9: 0x7E, -1e9: 0xFE, -math.inf: 0xFE, math.inf: 0x7E, -2.0: 0xC0,
+             3.0: 0x44, -3.0: 0xC4, 0.0: 0x00}
+    got = oracle.e4m3_encode(np.array(list(cases)))
+    assert got.tolist() == list(cases.values())
+    assert oracle.e4m3_encode(np.array([math.nan]))[0] == 0x7F
+
+
+def test_indexer_fp8_equals_indexer_on_small_integers():
+    # the integers -3..3 (the indexer inputs of the workloads) are exact in e4m3
+    q = rng.integers(-3, 4, size=(6, 2, 32)).astype(np.float64)
+    k = rng.integers(-3, 4, size=(40, 32)).astype(np.float64)
+    w = rng.integers(0, 4, size=(6, 2)).astype(np.float64)
+    lim = np.arange(34, 40)
+    a = oracle.indexer(q, w, k, lim)
+    b = oracle.indexer_fp8(oracle.e4m3_encode(q), w, oracle.e4m3_encode(k), lim)
+    assert np.array_equal(a, b)
+    # and a value e4m3 cannot hold moves the score: the codes are really used
+    k2 = k.copy()
+    k2[0, 0] = 1.1
+    b2 = oracle.indexer_fp8(oracle.e4m3_encode(q), w, oracle.e4m3_encode(k2), lim)
+    assert np.all(b2[:, 1:] == a[:, 1:])
+    assert np.allclose(b2[:, 0], oracle.indexer(q, w, np.where(k2 == 1.1, 1.125, k2), lim)[:, 0])
+
+
 # ---------------------------------------------------------------- top-K
 def _dominates(score, i, j):
     """i ranks strictly above j: higher score, or equal score and lower position."""
