@@ -1,6 +1,7 @@
 """Benchmark: fine-grained top-K sparse attention on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--index-fp8]
 
 A step is one pass of the whole path -- indexer -> top-K -> sparse attention
 (for the two-stage workload: pool, coarse scores, coarse top-k, expand, fine
@@ -20,6 +21,9 @@ memory and its output copied back inside the timed region; the copies of
 neighbouring steps run on their own streams under each step's kernels
 (pipeline.HostPipeline, two device buffer sets).  `cpu_baseline` times the CPU
 fp64 oracle on a bounded sample of query rows of the same workload.
+`--index-fp8` runs the indexer on e4m3 operands (quantised before timing);
+the workloads' integer-valued indexer inputs are exact in e4m3, so the
+selected positions are unchanged.
 """
 
 from __future__ import annotations
@@ -138,14 +142,20 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- workloads
-def make_case(name, seed, device):
-    """Device-resident inputs, pinned host copies and a plan for one workload."""
+def make_case(name, seed, device, index_fp8=False):
+    """Device-resident inputs, pinned host copies and a plan for one workload.
+    index_fp8: the indexer operands qI and kI are quantised to e4m3 once, on
+    the device, before any timing (keys enter an FP8 index cache when they
+    are written; the queries come from the producer of qI)."""
     import torch
 
+    from fine_grained_top_b200 import sa_convert_e4m3
     from fine_grained_top_b200.pipeline import DecodePlan, PrefillPlan
     from workloads import CONFIGS, gen_decode, gen_prefill
 
     cfg = dict(CONFIGS[name])
+    if index_fp8 and cfg["kind"] == "two_stage":
+        raise SystemExit("--index-fp8 serves the single-stage prefill and the decode workloads")
     inp = gen_prefill(seed=seed, **cfg) if cfg["kind"] != "decode" else gen_decode(seed=seed, **cfg)
 
     def host(x):
@@ -157,26 +167,34 @@ def make_case(name, seed, device):
 
     hosts = {k: host(v) for k, v in inp.items() if isinstance(v, np.ndarray)}
     devs = {k: v.to(device) for k, v in hosts.items()}
+    if index_fp8:
+        for k in ("qI", "kI"):
+            q8 = torch.empty(devs[k].shape, dtype=torch.uint8, device=device)
+            sa_convert_e4m3(devs[k], q8, devs[k].numel())
+            devs[k] = q8
+            hosts[k] = q8.cpu().pin_memory()
+        torch.cuda.synchronize()
     if cfg["kind"] == "decode":
         B = cfg["B"]
         if cfg.get("paged", False):
             make_plan = lambda: DecodePlan(B, cfg["Hq"], cfg["d"], cfg["H_I"], cfg["D_I"], cfg["K"], cfg["W"],
                                            S_max=0, paged=True, max_pages=inp["page_table"].shape[1],
-                                           pool_pages=inp["k"].shape[0], device=device)
+                                           pool_pages=inp["k"].shape[0], index_fp8=index_fp8, device=device)
         else:
             make_plan = lambda: DecodePlan(B, cfg["Hq"], cfg["d"], cfg["H_I"], cfg["D_I"], cfg["K"], cfg["W"],
-                                           S_max=inp["k"].shape[1], device=device)
+                                           S_max=inp["k"].shape[1], index_fp8=index_fp8, device=device)
         # per step a decode call receives the new tokens; the KV cache is resident state
         step_inputs = ["q", "qI", "w", "lengths"]
         units = B
     else:
         make_plan = lambda: PrefillPlan(cfg["N"], cfg["Hq"], cfg["d"], cfg["H_I"], cfg["D_I"], cfg["K"], cfg["W"],
-                                        block=cfg.get("block"), keep=cfg.get("keep"), device=device)
+                                        block=cfg.get("block"), keep=cfg.get("keep"), index_fp8=index_fp8,
+                                        device=device)
         step_inputs = ["q", "k", "v", "qI", "w", "kI"]
         units = cfg["N"]
     plan = make_plan()
     return dict(cfg=cfg, inp=inp, hosts=hosts, devs=devs, plan=plan, make_plan=make_plan,
-                stages=plan.stages(devs), units=units, step_inputs=step_inputs)
+                stages=plan.stages(devs), units=units, step_inputs=step_inputs, index_fp8=index_fp8)
 
 
 def stage_work(case):
@@ -193,12 +211,14 @@ def stage_work(case):
         pos, rows, pairs = np.arange(N, dtype=np.int64), N, N * (N + 1) // 2
     n_sel = ((topk >= 0) & (topk <= (pos - W)[:, None])).sum(1) + np.minimum(W, pos + 1)
     sum_sel = int(n_sel.sum())
-    qI_b, w_b, idx_b = rows * H * D * 2, rows * H * 2, 4 * rows * K
+    eb = 1 if case.get("index_fp8") else 2   # bytes per qI / kI element
+    qI_b, w_b, idx_b = rows * H * D * eb, rows * H * 2, 4 * rows * K
     q_b = rows * Hq * d * 2
     work = {"sum_selected": sum_sel, "causal_pairs": pairs}
     st = {}
     if cfg["kind"] == "decode":
-        st["indexer"] = dict(bytes=qI_b + w_b + pairs * D * 2 + 4 * pairs, flops=2.0 * pairs * H * D, bound="hbm")
+        st["indexer"] = dict(bytes=qI_b + w_b + pairs * D * eb + 4 * pairs, flops=2.0 * pairs * H * D,
+                             bound="hbm")
         st["topk"] = dict(bytes=4 * pairs + idx_b, flops=0.0, bound="hbm")
         st["attention"] = dict(bytes=2 * q_b + sum_sel * d * 2 * 2 + idx_b, flops=4.0 * Hq * d * sum_sel,
                                bound="hbm")
@@ -207,7 +227,7 @@ def stage_work(case):
         kv_b = 2 * N * d * 2
         st["attention"] = dict(bytes=2 * q_b + kv_b + idx_b, flops=4.0 * Hq * d * sum_sel, bound="tensor")
         if cfg["kind"] == "prefill":
-            st["indexer"] = dict(bytes=qI_b + w_b + N * D * 2 + 4 * pairs, flops=2.0 * pairs * H * D,
+            st["indexer"] = dict(bytes=qI_b + w_b + N * D * eb + 4 * pairs, flops=2.0 * pairs * H * D,
                                  bound="hbm")
             st["topk"] = dict(bytes=4 * pairs + idx_b, flops=0.0, bound="hbm")
         else:
@@ -284,7 +304,7 @@ def run_ours(args, rank, world, local_rank):
     device = "cuda:%d" % local_rank
     torch.cuda.set_device(local_rank)
     peaks = load_peaks()
-    case = make_case(args.workload, seed=rank, device=device)
+    case = make_case(args.workload, seed=rank, device=device, index_fp8=args.index_fp8)
     stream = torch.cuda.current_stream()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
     plan, d = case["plan"], case["devs"]
@@ -401,13 +421,16 @@ def run_ours(args, rank, world, local_rank):
     w = work["stages"][dom]
     roof["kernel"] = dom
     roof["algorithmic"] = w["flops"] if roof["bound"] == "tensor" else w["bytes"]
-    roof["traffic"] = ncu_traffic(args.workload, dom)   # per launch, from a capture of this exact source
+    tag = args.workload + ("+fp8-indexer" if args.index_fp8 else "")
+    roof["traffic"] = ncu_traffic(tag, dom)   # per launch, from a capture of this exact source
     roof["peak_src"] = peaks["src"] + " (burst figure; kernel timed alone per step)"
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16, indexer e4m3" if args.index_fp8 else "bf16",
+        "data": "synthetic",
         "config": {"workload": args.workload, **{k: v for k, v in case["cfg"].items() if k != "kind"},
+                   "indexer_operands": "e4m3 (quantised before timing)" if args.index_fp8 else "bf16",
                    "parallelism": "replicas (an independent sequence per GPU)" if world > 1 else "single GPU",
                    "l2": "flushed between steps (512 MB write outside the timed brackets)",
                    "launch": "step replayed as a captured CUDA graph"},
@@ -463,6 +486,8 @@ def main():
     ap.add_argument("--workload", default="prefill_8k")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--index-fp8", action="store_true",
+                    help="indexer on e4m3 operands (single-stage prefill and decode workloads)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -31,6 +31,9 @@ SIGNATURES = {
     "sa_version": (_i32, []),
     "sa_indexer_scores": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
                                  _vp, _vp, _i64, _vp, _vp]),
+    "sa_indexer_scores_fp8": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
+                                     _vp, _vp, _i64, _vp, _vp]),
+    "sa_convert_e4m3": (_i32, [_vp, _vp, _i64, _vp]),
     "sa_indexer_scores_candidates": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _i64, _vp, _vp,
                                             _i64, _vp, _vp]),
     "sa_block_scores_workspace_bytes": (_sz, [_i32, _i32, _i32]),
@@ -98,6 +101,18 @@ def sa_indexer_scores(qI, w, kI, page_table, max_pages, pool_pages, page_size, B
     _check(_lib.sa_indexer_scores(_ptr(qI), _ptr(w), _ptr(kI), _ptr(page_table), max_pages, pool_pages,
                                   page_size, B, T, S, H_I, D_I, _ptr(n_valid), _ptr(scores), ld_scores,
                                   _ptr(dev_status), _stream(stream)), "sa_indexer_scores")
+
+
+def sa_indexer_scores_fp8(qI, w, kI, page_table, max_pages, pool_pages, page_size, B, T, S, H_I, D_I,
+                          n_valid, scores, ld_scores, dev_status=None, stream=None):
+    """qI, kI: uint8 tensors of e4m3 bits (see sa_convert_e4m3)."""
+    _check(_lib.sa_indexer_scores_fp8(_ptr(qI), _ptr(w), _ptr(kI), _ptr(page_table), max_pages, pool_pages,
+                                      page_size, B, T, S, H_I, D_I, _ptr(n_valid), _ptr(scores), ld_scores,
+                                      _ptr(dev_status), _stream(stream)), "sa_indexer_scores_fp8")
+
+
+def sa_convert_e4m3(src, dst, n, stream=None):
+    _check(_lib.sa_convert_e4m3(_ptr(src), _ptr(dst), n, _stream(stream)), "sa_convert_e4m3")
 
 
 def sa_indexer_scores_candidates(qI, w, kI, T, S, H_I, D_I, cand, ld_cand, n_cand, scores, ld_scores,

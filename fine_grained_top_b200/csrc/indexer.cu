@@ -11,15 +11,20 @@
 //
 // Tile mapping: keys on M, (query, head) pairs on N.  qI is stored
 // [rows, H_I, D_I], so QT consecutive queries x H_I heads are QT*H_I
-// consecutive rows of D_I bf16: one K-major B operand.  One tile:
+// consecutive rows of D_I elements: one K-major B operand.  One tile:
 //     D[s, (t,j)] = kI[s] . qI[t,j]        M = 128 keys, N = 256 (or 16),
 // accumulated in fp32 in TMEM.  The epilogue thread owning TMEM lane s reads
 // the H_I adjacent columns of query t, applies ReLU and the weights w[t,:],
 // and writes scores[t, s]; a warp writes 32 consecutive floats per query.
 //
+// The operands are bf16 (tcgen05.mma kind::f16) or e4m3 bytes (kind::f8f6f4,
+// "Sparse Attention in 2026", "The designs that shipped": the shipped
+// indexer runs in FP8).  Either way the tile machinery only sees rows of RB
+// bytes (RB = 2*D_I or D_I) and K-steps of 32 bytes (16 bf16 or 32 e4m3).
+//
 // Warp roles (persistent CTAs, one per SM):
 //   warp 0     TMA producer (one elected lane) + TMEM allocator
-//   warp 1     MMA issuer (one elected lane): tcgen05.mma kind::f16
+//   warp 1     MMA issuer (one elected lane)
 //   warps 2..  epilogue teams: for the 256-column prefill tile, 2 item groups
 //              (alternate items, one TMEM accumulator each) x 2 column groups;
 //              for the 16-column decode tile, 4 item groups x 8 accumulators
@@ -28,7 +33,7 @@
 // walk the same sequence of non-empty items; the producer resolves the page
 // ids of 32 items in parallel, off the TMA issue path.
 // Shared-memory ring of STAGES {A = 128 keys, B = N query-head rows} tiles,
-// filled by TMA with the 128B (D_I = 64) or 64B (D_I = 32) swizzle that the
+// filled by TMA with the 128B (RB = 128) or 64B (RB = 64) swizzle that the
 // UMMA K-major descriptors expect.
 #include <cudaTypedefs.h>
 
@@ -50,11 +55,11 @@ struct IdxKernelArgs {
     int n_items;
 };
 
-template <int N, int D_I>
+template <int N, int RB>   // RB: bytes per qI / kI row (64 or 128)
 struct IdxCfg {
     static constexpr int kBoxRows = 64;                       // A is loaded as 2 boxes of 64 keys
-    static constexpr int kABytes = 128 * D_I * 2;
-    static constexpr int kBBytes = N * D_I * 2;
+    static constexpr int kABytes = 128 * RB;
+    static constexpr int kBBytes = N * RB;
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kStages = (N == 256) ? 4 : 8;
     // Epilogue teams: CG column groups split one item's queries; IG item
@@ -66,9 +71,9 @@ struct IdxCfg {
     static constexpr int kThreads = (2 + kEpiWarps) * 32;
     static constexpr uint32_t kTmemCols = (kAcc * N <= 32) ? 32 : (kAcc * N <= 64) ? 64 : (kAcc * N <= 128) ? 128
                                         : (kAcc * N <= 256) ? 256 : 512;
-    static constexpr uint32_t kSwizzleBytes = D_I * 2;         // 128 or 64
+    static constexpr uint32_t kSwizzleBytes = RB;              // 128 or 64
     static constexpr uint32_t kSbo = 8 * kSwizzleBytes;        // 8-row core group stride
-    static constexpr uint32_t kLayout = (D_I == 64) ? 2 : 4;   // UMMA layout: 128B / 64B swizzle
+    static constexpr uint32_t kLayout = (RB == 128) ? 2 : 4;   // UMMA layout: 128B / 64B swizzle
     static constexpr int kGroupCols = N / kCG;                 // TMEM columns per epilogue warp
     static constexpr size_t kWStage = (size_t)kEpiWarps * kGroupCols * 8;   // w (fp32) + n_valid per warp
     static constexpr size_t kSmemUsed = 1024 + (size_t)kStages * kStageBytes + 1024 + kWStage;
@@ -107,11 +112,11 @@ __device__ __forceinline__ bool item_at(const IdxKernelArgs &a, int i, ItemInfo 
     return true;
 }
 
-template <int N, int D_I, int H_I>
-__global__ void __launch_bounds__(IdxCfg<N, D_I>::kThreads, 1)
+template <int N, int RB, int H_I, bool F8>
+__global__ void __launch_bounds__(IdxCfg<N, RB>::kThreads, 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                       IdxKernelArgs a) {
-    using C = IdxCfg<N, D_I>;
+    using C = IdxCfg<N, RB>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *stage_base = smem;
@@ -210,7 +215,7 @@ __global__ void __launch_bounds__(IdxCfg<N, D_I>::kThreads, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        constexpr uint32_t idesc = idesc_bf16_f32(128, N);
+        constexpr uint32_t idesc = F8 ? idesc_e4m3_f32(128, N) : idesc_bf16_f32(128, N);
         int stage = 0;
         uint32_t phase = 0;
         int c = 0;   // non-empty items so far
@@ -233,10 +238,11 @@ __global__ void __launch_bounds__(IdxCfg<N, D_I>::kThreads, 1)
                         const uint32_t b_addr = a_addr + C::kABytes;
                         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * N);
 #pragma unroll
-                        for (int kk = 0; kk < D_I / 16; ++kk) {
+                        for (int kk = 0; kk < RB / 32; ++kk) {
                             const uint64_t da = smem_desc(a_addr + kk * 32, C::kSbo, C::kLayout);
                             const uint64_t db = smem_desc(b_addr + kk * 32, C::kSbo, C::kLayout);
-                            tc_mma_f16(d_tmem, da, db, idesc, kk > 0 ? 1u : 0u);
+                            if constexpr (F8) tc_mma_f8(d_tmem, da, db, idesc, kk > 0 ? 1u : 0u);
+                            else tc_mma_f16(d_tmem, da, db, idesc, kk > 0 ? 1u : 0u);
                         }
                         tc_commit(&empty_bar[stage]);
                         tc_commit(&tfull_bar[acc]);
@@ -390,23 +396,26 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
     return fn;
 }
 
-// rows x D_I bf16, row-major; box = box_rows x D_I with the swizzle matching D_I.
-static bool make_map(CUtensorMap *m, const void *base, uint64_t rows, int D_I, int box_rows) {
+// rows x RB bytes (bf16 or e4m3 elements), row-major; box = box_rows whole
+// rows with the swizzle matching RB.
+static bool make_map(CUtensorMap *m, const void *base, uint64_t rows, int RB, bool f8, int box_rows) {
     auto enc = get_encode();
     if (!enc) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)D_I, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)D_I * 2};
-    cuuint32_t box[2] = {(cuuint32_t)D_I, (cuuint32_t)box_rows};
+    const int elems = f8 ? RB : RB / 2;
+    cuuint64_t dims[2] = {(cuuint64_t)elems, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)RB};
+    cuuint32_t box[2] = {(cuuint32_t)elems, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
-    const CUtensorMapSwizzle sw = (D_I == 64) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+    const CUtensorMapSwizzle sw = (RB == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    const CUtensorMapDataType dt = f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    return enc(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int N, int D_I, int H_I>
+template <int N, int RB, int H_I, bool F8>
 static sa_status launch_tc(const IndexerArgs &a, cudaStream_t st) {
-    using C = IdxCfg<N, D_I>;
+    using C = IdxCfg<N, RB>;
     IdxKernelArgs k;
     k.w = a.w; k.page_table = a.page_table; k.n_valid = a.n_valid; k.scores = a.scores; k.ld = a.ld;
     k.dev_status = a.dev_status; k.max_pages = a.max_pages; k.pool_pages = a.pool_pages;
@@ -421,11 +430,11 @@ static sa_status launch_tc(const IndexerArgs &a, cudaStream_t st) {
 
     CUtensorMap mk, mq;
     const uint64_t k_rows = a.page_table ? (uint64_t)a.pool_pages * a.page_size : (uint64_t)a.B * a.S;
-    if (!make_map(&mk, a.kI, k_rows, D_I, C::kBoxRows)) return SA_ERR_CUDA;
-    if (!make_map(&mq, a.qI, (uint64_t)a.B * a.T * H_I, D_I, N)) return SA_ERR_CUDA;
+    if (!make_map(&mk, a.kI, k_rows, RB, F8, C::kBoxRows)) return SA_ERR_CUDA;
+    if (!make_map(&mq, a.qI, (uint64_t)a.B * a.T * H_I, RB, F8, N)) return SA_ERR_CUDA;
 
-    auto kern = indexer_tc_kernel<N, D_I, H_I>;
-    if (prepare_kernel<indexer_tc_kernel<N, D_I, H_I>>(C::kSmem, false) != cudaSuccess) return SA_ERR_CUDA;
+    auto kern = indexer_tc_kernel<N, RB, H_I, F8>;
+    if (prepare_kernel<indexer_tc_kernel<N, RB, H_I, F8>>(C::kSmem, false) != cudaSuccess) return SA_ERR_CUDA;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -434,22 +443,70 @@ static sa_status launch_tc(const IndexerArgs &a, cudaStream_t st) {
     return cuda_ok(cudaGetLastError());
 }
 
-template <int N, int D_I>
+template <int N, int RB, bool F8>
 static sa_status launch_tc_h(const IndexerArgs &a, cudaStream_t st) {
     switch (a.H_I) {
-        case 1: return launch_tc<N, D_I, 1>(a, st);
-        case 2: return launch_tc<N, D_I, 2>(a, st);
-        case 4: return launch_tc<N, D_I, 4>(a, st);
-        case 8: return launch_tc<N, D_I, 8>(a, st);
+        case 1: return launch_tc<N, RB, 1, F8>(a, st);
+        case 2: return launch_tc<N, RB, 2, F8>(a, st);
+        case 4: return launch_tc<N, RB, 4, F8>(a, st);
+        case 8: return launch_tc<N, RB, 8, F8>(a, st);
     }
     return SA_ERR_UNSUPPORTED;
 }
 
-sa_status launch_indexer(const IndexerArgs &a, cudaStream_t st) {
+template <int RB, bool F8>
+static sa_status launch_tc_n(const IndexerArgs &a, cudaStream_t st) {
     const bool small = a.T * a.H_I <= 16;   // decode: a handful of queries per sequence
-    if (a.D_I == 64) return small ? launch_tc_h<16, 64>(a, st) : launch_tc_h<256, 64>(a, st);
-    if (a.D_I == 32) return small ? launch_tc_h<16, 32>(a, st) : launch_tc_h<256, 32>(a, st);
+    return small ? launch_tc_h<16, RB, F8>(a, st) : launch_tc_h<256, RB, F8>(a, st);
+}
+
+sa_status launch_indexer(const IndexerArgs &a, cudaStream_t st) {
+    const int rb = a.fp8 ? a.D_I : 2 * a.D_I;
+    if (rb == 128) return a.fp8 ? launch_tc_n<128, true>(a, st) : launch_tc_n<128, false>(a, st);
+    if (rb == 64) return a.fp8 ? launch_tc_n<64, true>(a, st) : launch_tc_n<64, false>(a, st);
     return SA_ERR_UNSUPPORTED;
+}
+
+// ------------------------------------------------------------------------
+// bf16 -> e4m3 (OCP FP8: 4 exponent bits with bias 7, 3 mantissa bits, no
+// infinities, S.1111.111 is NaN).  The hardware conversion rounds to nearest
+// even and, with .satfinite, clamps finite overflow and infinities to +-448;
+// NaN stays NaN.  Eight elements per thread: one 16-byte load, one 8-byte
+// store; the elements past the last whole group of 8 (or all of them when
+// the buffers are not aligned for that) go one per thread.
+// ------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e4m3_pair(uint32_t bf16x2) {
+    const float lo = __uint_as_float(bf16x2 << 16), hi = __uint_as_float(bf16x2 & 0xFFFF0000u);
+    unsigned short r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));   // hi -> upper byte
+    return r;
+}
+
+__global__ void __launch_bounds__(256) convert_e4m3_kernel(const uint16_t *src, uint8_t *dst, int64_t n,
+                                                           int64_t n_vec) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (int64_t i = i0; i < n_vec; i += stride) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(src) + i);
+        uint2 o;
+        o.x = e4m3_pair(u.x) | (e4m3_pair(u.y) << 16);
+        o.y = e4m3_pair(u.z) | (e4m3_pair(u.w) << 16);
+        reinterpret_cast<uint2 *>(dst)[i] = o;
+    }
+    for (int64_t i = n_vec * 8 + i0; i < n; i += stride) dst[i] = (uint8_t)(e4m3_pair(src[i]) & 0xFFu);
+}
+
+sa_status launch_convert_e4m3(const uint16_t *src, uint8_t *dst, int64_t n, cudaStream_t st) {
+    const bool vec = (reinterpret_cast<uintptr_t>(src) & 15u) == 0 && (reinterpret_cast<uintptr_t>(dst) & 7u) == 0;
+    const int64_t n_vec = vec ? n / 8 : 0;
+    const int64_t work = n_vec + (n - n_vec * 8);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t want = (work + 255) / 256, cap = (int64_t)sms * 8;
+    const int grid = (int)(want < cap ? want : cap);
+    convert_e4m3_kernel<<<grid, 256, 0, st>>>(src, dst, n, n_vec);
+    return cuda_ok(cudaGetLastError());
 }
 
 // ------------------------------------------------------------------------

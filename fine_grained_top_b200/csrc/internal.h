@@ -27,7 +27,9 @@ sa_status launch_topk(TopkArgs a, cudaStream_t st);
 int topk_max_row_len();
 
 struct IndexerArgs {
-    const uint16_t *qI, *w, *kI;
+    const void *qI, *kI;   // bf16 or e4m3 elements (fp8)
+    const uint16_t *w;
+    bool fp8;
     const int32_t *page_table;
     int max_pages, pool_pages, page_size;
     int B, T, S, H_I, D_I;
@@ -37,6 +39,7 @@ struct IndexerArgs {
     int *dev_status;
 };
 sa_status launch_indexer(const IndexerArgs &a, cudaStream_t st);
+sa_status launch_convert_e4m3(const uint16_t *src, uint8_t *dst, int64_t n, cudaStream_t st);
 
 struct CandArgs {
     const uint16_t *qI, *w, *kI;

@@ -13,6 +13,7 @@ namespace {
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool head_dim_ok(int d) { return d == 64 || d == 128; }
 inline bool index_dim_ok(int D) { return D == 32 || D == 64; }
+inline bool index_dim_fp8_ok(int D) { return D == 64 || D == 128; }
 inline bool index_heads_ok(int H) { return H == 1 || H == 2 || H == 4 || H == 8; }
 inline cudaStream_t cs(sa_stream s) { return reinterpret_cast<cudaStream_t>(s); }
 
@@ -48,14 +49,16 @@ sa_status sa_dev_status_decode(int word) {
     return SA_OK;
 }
 
-int sa_version(void) { return 100; }
+int sa_version(void) { return 101; }
 
-sa_status sa_indexer_scores(const sa_bf16 *qI, const sa_bf16 *w, const sa_bf16 *kI, const int32_t *page_table,
-                            int max_pages, int pool_pages, int page_size, int B, int T, int S, int H_I, int D_I,
-                            const int32_t *n_valid, float *scores, int64_t ld_scores, int *dev_status,
-                            sa_stream stream) {
+// Shared by the bf16 and e4m3 entry points: identical argument rules, the
+// element type only changes the row bytes the kernel sees.
+static sa_status indexer_scores(const void *qI, const sa_bf16 *w, const void *kI, bool fp8,
+                                const int32_t *page_table, int max_pages, int pool_pages, int page_size, int B,
+                                int T, int S, int H_I, int D_I, const int32_t *n_valid, float *scores,
+                                int64_t ld_scores, int *dev_status, sa_stream stream) {
     if (B < 0 || T < 0 || S < 0 || ld_scores < S || (ld_scores & 3)) return SA_ERR_INVALID_ARG;
-    if (!index_heads_ok(H_I) || !index_dim_ok(D_I)) return SA_ERR_UNSUPPORTED;
+    if (!index_heads_ok(H_I) || !(fp8 ? index_dim_fp8_ok(D_I) : index_dim_ok(D_I))) return SA_ERR_UNSUPPORTED;
     if (B == 0 || T == 0 || S == 0) return SA_OK;
     if (!qI || !w || !kI || !scores || !aligned16(qI) || !aligned16(kI)) return SA_ERR_INVALID_ARG;
     if (n_valid == nullptr && T > S) return SA_ERR_INVALID_ARG;
@@ -67,12 +70,35 @@ sa_status sa_indexer_scores(const sa_bf16 *qI, const sa_bf16 *w, const sa_bf16 *
     }
     return guarded([&] {
         IndexerArgs a;
-        a.qI = qI; a.w = w; a.kI = kI; a.page_table = page_table;
+        a.qI = qI; a.w = w; a.kI = kI; a.fp8 = fp8; a.page_table = page_table;
         a.max_pages = max_pages; a.pool_pages = pool_pages; a.page_size = page_size;
         a.B = B; a.T = T; a.S = S; a.H_I = H_I; a.D_I = D_I;
         a.n_valid = n_valid; a.scores = scores; a.ld = ld_scores; a.dev_status = dev_status;
         return launch_indexer(a, cs(stream));
     });
+}
+
+sa_status sa_indexer_scores(const sa_bf16 *qI, const sa_bf16 *w, const sa_bf16 *kI, const int32_t *page_table,
+                            int max_pages, int pool_pages, int page_size, int B, int T, int S, int H_I, int D_I,
+                            const int32_t *n_valid, float *scores, int64_t ld_scores, int *dev_status,
+                            sa_stream stream) {
+    return indexer_scores(qI, w, kI, false, page_table, max_pages, pool_pages, page_size, B, T, S, H_I, D_I,
+                          n_valid, scores, ld_scores, dev_status, stream);
+}
+
+sa_status sa_indexer_scores_fp8(const sa_e4m3 *qI, const sa_bf16 *w, const sa_e4m3 *kI,
+                                const int32_t *page_table, int max_pages, int pool_pages, int page_size, int B,
+                                int T, int S, int H_I, int D_I, const int32_t *n_valid, float *scores,
+                                int64_t ld_scores, int *dev_status, sa_stream stream) {
+    return indexer_scores(qI, w, kI, true, page_table, max_pages, pool_pages, page_size, B, T, S, H_I, D_I,
+                          n_valid, scores, ld_scores, dev_status, stream);
+}
+
+sa_status sa_convert_e4m3(const sa_bf16 *src, sa_e4m3 *dst, int64_t n, sa_stream stream) {
+    if (n < 0) return SA_ERR_INVALID_ARG;
+    if (n == 0) return SA_OK;
+    if (!src || !dst) return SA_ERR_INVALID_ARG;
+    return guarded([&] { return launch_convert_e4m3(src, dst, n, cs(stream)); });
 }
 
 sa_status sa_indexer_scores_candidates(const sa_bf16 *qI, const sa_bf16 *w, const sa_bf16 *kI, int T, int S,

@@ -21,7 +21,8 @@ import math
 import torch
 
 from . import (sa_block_scores_workspace_bytes, sa_coarse_block_counts, sa_decode_workspace_bytes,
-               sa_expand_blocks, sa_indexer_scores, sa_indexer_scores_blocks, sa_pool_index_keys,
+               sa_expand_blocks, sa_indexer_scores, sa_indexer_scores_blocks, sa_indexer_scores_fp8,
+               sa_pool_index_keys,
                sa_prefill_workspace_bytes, sa_sparse_attn_decode, sa_sparse_attn_prefill, sa_topk_select)
 
 
@@ -31,10 +32,16 @@ def _ld(n: int) -> int:
 
 class PrefillPlan:
     """Buffers for one sequence of N tokens (queries at positions 0..N-1).
-    Inputs: dict with q [N,Hq,d], k/v [N,d], qI [N,H_I,D_I], w [N,H_I], kI [N,D_I]."""
+    Inputs: dict with q [N,Hq,d], k/v [N,d], qI [N,H_I,D_I], w [N,H_I], kI [N,D_I].
+    index_fp8: qI and kI are e4m3 bytes (uint8) and the indexer runs in FP8
+    (single-stage selection only)."""
 
-    def __init__(self, N, Hq, d, H_I, D_I, K, W, block=None, keep=None, row_blocks=1, device="cuda"):
+    def __init__(self, N, Hq, d, H_I, D_I, K, W, block=None, keep=None, row_blocks=1, index_fp8=False,
+                 device="cuda"):
+        if index_fp8 and block is not None:
+            raise ValueError("the FP8 indexer serves the single-stage selection")
         self.N, self.Hq, self.d, self.H_I, self.D_I, self.K, self.W = N, Hq, d, H_I, D_I, K, W
+        self.index = sa_indexer_scores_fp8 if index_fp8 else sa_indexer_scores
         self.block, self.keep = block, keep
         # single-stage only: score and select the queries in row_blocks blocks,
         # so that a block's scores are still in L2 when top-K reads them
@@ -84,7 +91,7 @@ class PrefillPlan:
                 t0, t1 = bounds[b], bounds[b + 1]
                 if t1 <= t0:
                     continue
-                out.append(("indexer", lambda t0=t0, t1=t1: sa_indexer_scores(
+                out.append(("indexer", lambda t0=t0, t1=t1: self.index(
                     x["qI"][t0:t1], x["w"][t0:t1], x["kI"], None, 0, 0, 64, 1, t1 - t0, t1, H, D, None,
                     self.scores[t0:t1], self.ld, ds, stream)))
                 out.append(("topk", lambda t0=t0, t1=t1: sa_topk_select(
@@ -92,8 +99,8 @@ class PrefillPlan:
             return out + [attn]
         if self.block is None:
             return [
-                ("indexer", lambda: sa_indexer_scores(x["qI"], x["w"], x["kI"], None, 0, 0, 64, 1, N, N, H, D,
-                                                      None, self.scores, self.ld, ds, stream)),
+                ("indexer", lambda: self.index(x["qI"], x["w"], x["kI"], None, 0, 0, 64, 1, N, N, H, D,
+                                               None, self.scores, self.ld, ds, stream)),
                 ("topk", lambda: sa_topk_select(self.scores, self.ld, N, N, None, None, 0, K, self.topk, ds,
                                                 stream)),
                 attn]
@@ -130,11 +137,13 @@ class DecodePlan:
     """Buffers for B sequences, one query each, over a contiguous ([B, S_max, *])
     or paged (pools [P, 64, *] + page_table [B, max_pages]) cache.
     Inputs: dict with q [B,Hq,d], k/v/kI caches, qI [B,H_I,D_I], w [B,H_I],
-    lengths [B] int32 and, when paged, page_table."""
+    lengths [B] int32 and, when paged, page_table.
+    index_fp8: the qI and kI cache hold e4m3 bytes (uint8); FP8 indexer."""
 
     def __init__(self, B, Hq, d, H_I, D_I, K, W, S_max, paged=False, max_pages=0, pool_pages=0,
-                 device="cuda"):
+                 index_fp8=False, device="cuda"):
         self.B, self.Hq, self.d, self.H_I, self.D_I, self.K, self.W = B, Hq, d, H_I, D_I, K, W
+        self.index = sa_indexer_scores_fp8 if index_fp8 else sa_indexer_scores
         self.paged, self.max_pages, self.pool_pages = paged, max_pages, pool_pages
         self.S = max_pages * 64 if paged else S_max
         self.S_max = S_max
@@ -152,9 +161,9 @@ class DecodePlan:
     def stages(self, x, stream=None):
         ds, pt = self.dev_status, x.get("page_table")
         return [
-            ("indexer", lambda: sa_indexer_scores(x["qI"], x["w"], x["kI"], pt, self.max_pages, self.pool_pages,
-                                                  64, self.B, 1, self.S, self.H_I, self.D_I, x["lengths"],
-                                                  self.scores, self.ld, ds, stream)),
+            ("indexer", lambda: self.index(x["qI"], x["w"], x["kI"], pt, self.max_pages, self.pool_pages,
+                                           64, self.B, 1, self.S, self.H_I, self.D_I, x["lengths"],
+                                           self.scores, self.ld, ds, stream)),
             ("topk", lambda: sa_topk_select(self.scores, self.ld, self.B, self.S, x["lengths"], None, 0, self.K,
                                             self.topk, ds, stream)),
             ("attention", lambda: sa_sparse_attn_decode(

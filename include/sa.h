@@ -48,6 +48,7 @@ extern "C" {
 #endif
 
 typedef uint16_t sa_bf16;                 /* raw bfloat16 bits */
+typedef uint8_t sa_e4m3;                  /* raw OCP FP8 e4m3 bits (no inf; 0x7F/0xFF NaN) */
 typedef struct CUstream_st *sa_stream;    /* same type as cudaStream_t */
 
 typedef enum {
@@ -107,6 +108,35 @@ sa_status sa_indexer_scores(const sa_bf16 *qI, const sa_bf16 *w,
                             const int32_t *n_valid, float *scores,
                             int64_t ld_scores, int *dev_status,
                             sa_stream stream);
+
+/* Indexer scores with FP8 operands ("Sparse Attention in 2026", "The designs
+ * that shipped": the shipped lightning indexer is a small FP8 network).
+ *   The same definition, layouts, n_valid rule, errors and unwritten columns
+ *   as sa_indexer_scores, with qI and kI held as e4m3 bytes: the products
+ *   run on the tensor cores as tcgen05.mma kind::f8f6f4 (each e4m3 x e4m3
+ *   product is exact) and sums are fp32.  w stays bf16.
+ *   qI [B, T, H_I, D_I] e4m3, kI contiguous [B, S, D_I] or a paged pool
+ *   [P, 64, D_I] e4m3, both 16-byte aligned; D_I in {64, 128} (rows of 64
+ *   or 128 bytes).
+ *   Scores equal sa_indexer_scores applied to the decoded values whenever
+ *   the fp32 sums are exact (e.g. the integers -3..3 of the tests, which e4m3
+ *   holds exactly). */
+sa_status sa_indexer_scores_fp8(const sa_e4m3 *qI, const sa_bf16 *w,
+                                const sa_e4m3 *kI, const int32_t *page_table,
+                                int max_pages, int pool_pages, int page_size,
+                                int B, int T, int S, int H_I, int D_I,
+                                const int32_t *n_valid, float *scores,
+                                int64_t ld_scores, int *dev_status,
+                                sa_stream stream);
+
+/* Quantise n bf16 values to e4m3 (for indexer keys entering the cache and
+ * indexer queries): round to nearest, ties to even; finite values beyond
+ * +-448 and infinities become +-448; NaN becomes NaN (0x7F with the sign).
+ *   src [n] bf16, dst [n] e4m3, device memory, not overlapping; any n >= 0
+ *   and any alignment (16-byte src and 8-byte dst take the vector path).
+ *   Errors: SA_ERR_INVALID_ARG (n < 0, NULL with n > 0), SA_ERR_CUDA. */
+sa_status sa_convert_e4m3(const sa_bf16 *src, sa_e4m3 *dst, int64_t n,
+                          sa_stream stream);
 
 /* Indexer scores over an explicit candidate list per query (the fine pass of
  * the two-stage selection, "What Fine-Grained Means": the fine pass scores

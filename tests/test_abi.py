@@ -45,7 +45,7 @@ def test_status_strings_and_version(sa):
     lib = sa._lib
     assert lib.sa_status_string(0) == b"SA_OK"
     assert lib.sa_status_string(6) == b"SA_ERR_WORKSPACE"
-    assert sa.sa_version() == 100
+    assert sa.sa_version() == 101
     assert sa.sa_dev_status_decode(0) == sa.SA_OK
     assert sa.sa_dev_status_decode(sa.SA_DEV_INDEX) == sa.SA_ERR_INDEX
     assert sa.sa_dev_status_decode(sa.SA_DEV_ORDER) == sa.SA_ERR_INDEX
@@ -81,6 +81,20 @@ def test_indexer_argument_checks(sa):
     assert f(N0, P, P, N0, 0, 0, 64, 1, 8, 8, 4, 64, N0, P, 8, N0, N0) == sa.SA_ERR_INVALID_ARG
     assert f(P, P, P, N0, 0, 0, 64, 0, 8, 8, 4, 64, N0, P, 8, N0, N0) == sa.SA_OK
     assert ok
+
+
+def test_indexer_fp8_and_convert_argument_checks(sa):
+    f = sa._lib.sa_indexer_scores_fp8
+    assert f(P, P, P, N0, 0, 0, 64, 1, 8, 8, 4, 32, N0, P, 8, N0, N0) == sa.SA_ERR_UNSUPPORTED  # D_I 32
+    assert f(P, P, P, N0, 0, 0, 64, 1, 8, 8, 3, 64, N0, P, 8, N0, N0) == sa.SA_ERR_UNSUPPORTED  # H_I
+    assert f(P, P, P, N0, 0, 0, 64, 1, 8, 8, 4, 128, N0, P, 4, N0, N0) == sa.SA_ERR_INVALID_ARG  # ld < S
+    assert f(P, P, ctypes.c_void_p(24), N0, 0, 0, 64, 1, 8, 8, 4, 64, N0, P, 8, N0, N0) \
+        == sa.SA_ERR_INVALID_ARG   # kI not 16-byte aligned
+    assert f(P, P, P, N0, 0, 0, 64, 1, 8, 0, 4, 128, N0, P, 8, N0, N0) == sa.SA_OK  # S = 0
+    g = sa._lib.sa_convert_e4m3
+    assert g(P, P, -1, N0) == sa.SA_ERR_INVALID_ARG
+    assert g(N0, P, 5, N0) == sa.SA_ERR_INVALID_ARG
+    assert g(N0, N0, 0, N0) == sa.SA_OK
 
 
 def test_attention_argument_checks(sa):

@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import oracle
-from workloads import CONFIGS, config_inputs, gen_decode, gen_prefill
+from workloads import CONFIGS, bf16_bits, bf16_to_f64, config_inputs, gen_decode, gen_prefill
 from tests.gpu_helpers import assert_close_attention, dev, host_f64, status
 
 pytestmark = pytest.mark.gpu
@@ -139,6 +139,103 @@ def test_indexer_decode_contiguous_and_paged(sa):
             assert np.array_equal(got[b, :L], want[0]), (paged, b)
 
 
+# ---------------------------------------------------------------- FP8 indexer
+def _e4m3_dev(sa, x_bf16):
+    out = torch.empty(x_bf16.shape, dtype=torch.uint8, device="cuda")
+    sa.sa_convert_e4m3(x_bf16, out, x_bf16.numel())
+    return out
+
+
+def test_convert_e4m3_matches_oracle(sa):
+    r = np.random.default_rng(11)
+    vals = (r.standard_normal(300007) * np.exp2(r.uniform(-14, 10, 300007))).astype(np.float32)
+    special = np.array([0.0, -0.0, np.inf, -np.inf, 448, 464, 480, 1e30, -1e30, 2.0 ** -9, 2.0 ** -10,
+                        3 * 2.0 ** -10, 2.0 ** -17, 1.0625, 1.1875, -3, 3], dtype=np.float32)
+    vals = np.concatenate([special, vals])
+    bits = bf16_bits(vals.astype(np.float64))
+    x = dev(bits)
+    want = oracle.e4m3_encode(bits)
+    for lo, n in ((0, bits.size), (0, 1), (0, 7), (0, 9), (1, 1000), (3, 4099)):   # ragged, misaligned
+        out = torch.full((n,), 0x55, dtype=torch.uint8, device="cuda")
+        sa.sa_convert_e4m3(x[lo:lo + n], out, n)
+        assert np.array_equal(out.cpu().numpy(), want[lo:lo + n]), (lo, n)
+    nan = dev(bf16_bits(np.array([np.nan, -np.nan])))
+    out = _e4m3_dev(sa, nan).cpu().numpy()
+    assert np.all(out & 0x7F == 0x7F)
+
+
+@pytest.mark.parametrize("N,H_I,D_I,rows", [
+    (512, 2, 64, None), (1000, 4, 64, None), (300, 8, 128, None), (777, 1, 128, None),
+    (129, 4, 64, None), (1, 4, 64, None), (8192, 4, 64, 384), (8192, 8, 128, 200),
+])
+def test_indexer_fp8_prefill_exact(sa, N, H_I, D_I, rows):
+    inp = gen_prefill(N=N, Hq=1, d=64, H_I=H_I, D_I=D_I, seed=N + 7 * H_I)
+    t = _to_dev(inp, ("qI", "w", "kI"))
+    q8, k8 = _e4m3_dev(sa, t["qI"]), _e4m3_dev(sa, t["kI"])
+    ld = (N + 3) // 4 * 4
+    sc = torch.full((N, ld), float("nan"), device="cuda")
+    ds = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sa.sa_indexer_scores_fp8(q8, t["w"], k8, None, 0, 0, 64, 1, N, N, H_I, D_I, None, sc, ld, ds)
+    got = sc.cpu().numpy()
+    assert status(ds) == 0
+    r = np.arange(N) if rows is None else np.unique(np.r_[np.linspace(0, N - 1, rows).astype(int), 0, 127, 128])
+    qc, kc = oracle.e4m3_encode(inp["qI"][r]), oracle.e4m3_encode(inp["kI"])
+    want = oracle.indexer_fp8(qc, inp["w"][r], kc, r)
+    for i, t_ in enumerate(r):
+        assert np.array_equal(got[t_, :t_ + 1], want[i, :t_ + 1]), t_
+
+
+def test_indexer_fp8_general_codes_within_fp32_sum_bound(sa):
+    # non-integer e4m3 operands: every product is exact, only the fp32 sums
+    # round; bound each score by the textbook bound for n fp32 additions,
+    # n * 2^-24 of the sum of the terms' magnitudes (n = D_I + H_I)
+    N, H_I, D_I = 640, 4, 128
+    r = np.random.default_rng(3)
+    codes = r.integers(0, 256, size=(N * H_I * D_I + N * D_I,), dtype=np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x38   # no NaN
+    qc = codes[:N * H_I * D_I].reshape(N, H_I, D_I)
+    kc = codes[N * H_I * D_I:].reshape(N, D_I)
+    inp = gen_prefill(N=N, Hq=1, d=64, H_I=H_I, D_I=D_I, seed=4)
+    sc = torch.full((N, N), float("nan"), device="cuda")
+    ds = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sa.sa_indexer_scores_fp8(dev(qc), dev(inp["w"]), dev(kc), None, 0, 0, 64, 1, N, N, H_I, D_I, None,
+                             sc, N, ds)
+    got = sc.cpu().numpy()
+    assert status(ds) == 0
+    rows = np.arange(0, N, 7)
+    want = oracle.indexer_fp8(qc[rows], inp["w"][rows], kc, rows)
+    qv, kv, wv = oracle.e4m3_decode(qc[rows]), oracle.e4m3_decode(kc), bf16_to_f64(inp["w"][rows])
+    mag = np.einsum("rj,rjc,sc->rs", wv, np.abs(qv), np.abs(kv))
+    for i, t_ in enumerate(rows):
+        err = np.abs(got[t_, :t_ + 1] - want[i, :t_ + 1])
+        assert np.all(err <= (D_I + H_I) * 2.0 ** -24 * mag[i, :t_ + 1]), (t_, err.max())
+
+
+def test_indexer_fp8_decode_contiguous_and_paged(sa):
+    lengths = [131072, 5000, 1, 64, 65, 130000]
+    B = len(lengths)
+    for paged in (False, True):
+        inp = gen_decode(B=B, lengths=lengths, Hq=16, d=64, H_I=8, D_I=64, paged=paged, seed=6)
+        t = _to_dev(inp, ("qI", "w", "kI"))
+        q8, k8 = _e4m3_dev(sa, t["qI"]), _e4m3_dev(sa, t["kI"])
+        sl = dev(inp["lengths"])
+        if paged:
+            S = inp["page_table"].shape[1] * 64
+            pt, mp, pp = dev(inp["page_table"]), inp["page_table"].shape[1], inp["kI"].shape[0]
+        else:
+            S, pt, mp, pp = inp["kI"].shape[1], None, 0, 0
+        sc = torch.full((B, S), float("nan"), device="cuda")
+        ds = torch.zeros(1, dtype=torch.int32, device="cuda")
+        sa.sa_indexer_scores_fp8(q8, t["w"], k8, pt, mp, pp, 64, B, 1, S, 8, 64, sl, sc, S, ds)
+        got = sc.cpu().numpy()
+        assert status(ds) == 0
+        for b, L in enumerate(lengths):
+            _, _, kI = oracle.decode_sequence(inp, b)
+            want = oracle.indexer_fp8(oracle.e4m3_encode(inp["qI"][b:b + 1]), inp["w"][b:b + 1],
+                                      oracle.e4m3_encode(kI), [L - 1])
+            assert np.array_equal(got[b, :L], want[0]), (paged, b)
+
+
 @pytest.mark.parametrize("N,keep,H_I,D_I,rows", [(1000, 4, 4, 64, None), (4096, 16, 8, 64, 200),
                                                    (700, 3, 2, 32, None), (333, 8, 1, 32, None),
                                                    (65, 2, 4, 64, None), (4160, 64, 4, 64, 150)])
@@ -224,12 +321,14 @@ def test_prefill_chunk_of_long_sequence(sa, use_ws):
 
 
 # ====================================================================== end to end
-def _prefill_e2e(sa, inp, K, W, rows=None, block=None, keep=None):
+def _prefill_e2e(sa, inp, K, W, rows=None, block=None, keep=None, index_fp8=False):
     PrefillPlan, _ = _pl()
     N, Hq, d = inp["q"].shape
     H_I, D_I = inp["qI"].shape[1:]
-    plan = PrefillPlan(N, Hq, d, H_I, D_I, K, W, block=block, keep=keep)
+    plan = PrefillPlan(N, Hq, d, H_I, D_I, K, W, block=block, keep=keep, index_fp8=index_fp8)
     t = _to_dev(inp)
+    if index_fp8:   # the integer indexer inputs are exact in e4m3: same oracle
+        t["qI"], t["kI"] = _e4m3_dev(sa, t["qI"]), _e4m3_dev(sa, t["kI"])
     plan.run(t["q"], t["k"], t["v"], t["qI"], t["w"], t["kI"])
     assert status(plan.dev_status) == 0
     ref = oracle.prefill(inp, K, W, rows=rows, block=block, keep=keep)
@@ -284,12 +383,13 @@ def test_e2e_prefill_512(sa):
     _prefill_e2e(sa, config_inputs("prefill_512"), c["K"], c["W"])
 
 
-def test_e2e_prefill_8k(sa):
+@pytest.mark.parametrize("index_fp8", [False, True])
+def test_e2e_prefill_8k(sa, index_fp8):
     c = CONFIGS["prefill_8k"]
     inp = config_inputs("prefill_8k")
     N = c["N"]
     rows = np.unique(np.r_[np.linspace(0, N - 1, 160).astype(int), 1023, 1024, 1151, 1152, N - 1])
-    plan, _ = _prefill_e2e(sa, inp, c["K"], c["W"], rows=rows)
+    plan, _ = _prefill_e2e(sa, inp, c["K"], c["W"], rows=rows, index_fp8=index_fp8)
     # every row's index set, bit for bit (the oracle's selection of all 8192 rows)
     sc = oracle.indexer(inp["qI"], inp["w"], inp["kI"], np.arange(N))
     want = oracle.topk(sc, np.arange(N) + 1, c["K"])
@@ -312,20 +412,23 @@ def test_e2e_two_stage_64k_sampled(sa):
     assert np.array_equal(plan.blocks.cpu().numpy()[rows], ref["blocks"])
 
 
-def _decode_e2e(sa, inp, K, W):
+def _decode_e2e(sa, inp, K, W, index_fp8=False):
     _, DecodePlan = _pl()
     B, Hq, d = inp["q"].shape
     H_I, D_I = inp["qI"].shape[1:]
     paged = "page_table" in inp
     t = _to_dev(inp)
+    if index_fp8:   # the integer indexer inputs are exact in e4m3: same oracle
+        t["qI"], t["kI"] = _e4m3_dev(sa, t["qI"]), _e4m3_dev(sa, t["kI"])
     sl = dev(inp["lengths"])
     if paged:
         pt = dev(inp["page_table"])
         plan = DecodePlan(B, Hq, d, H_I, D_I, K, W, S_max=0, paged=True,
-                          max_pages=inp["page_table"].shape[1], pool_pages=inp["k"].shape[0])
+                          max_pages=inp["page_table"].shape[1], pool_pages=inp["k"].shape[0],
+                          index_fp8=index_fp8)
     else:
         pt = None
-        plan = DecodePlan(B, Hq, d, H_I, D_I, K, W, S_max=inp["k"].shape[1])
+        plan = DecodePlan(B, Hq, d, H_I, D_I, K, W, S_max=inp["k"].shape[1], index_fp8=index_fp8)
     plan.run(t["q"], t["k"], t["v"], t["qI"], t["w"], t["kI"], sl, pt)
     assert status(plan.dev_status) == 0
     ref = oracle.decode(inp, K, W)
@@ -334,14 +437,16 @@ def _decode_e2e(sa, inp, K, W):
     assert np.max(np.abs(host_f64(plan.lse) - ref["lse"])) < 1e-3
 
 
-def test_e2e_decode_8x128k(sa):
+@pytest.mark.parametrize("index_fp8", [False, True])
+def test_e2e_decode_8x128k(sa, index_fp8):
     c = CONFIGS["decode_8x128k"]
-    _decode_e2e(sa, config_inputs("decode_8x128k"), c["K"], c["W"])
+    _decode_e2e(sa, config_inputs("decode_8x128k"), c["K"], c["W"], index_fp8=index_fp8)
 
 
-def test_e2e_decode_paged_16(sa):
+@pytest.mark.parametrize("index_fp8", [False, True])
+def test_e2e_decode_paged_16(sa, index_fp8):
     c = CONFIGS["decode_paged_16x256k"]
-    _decode_e2e(sa, config_inputs("decode_paged_16x256k"), c["K"], c["W"])
+    _decode_e2e(sa, config_inputs("decode_paged_16x256k"), c["K"], c["W"], index_fp8=index_fp8)
 
 
 @pytest.mark.parametrize("lengths,K,W", [([1, 2, 63, 64, 65, 3000], 100, 16), ([5000, 700], 4096, 0),
