@@ -55,10 +55,19 @@ struct IdxKernelArgs {
     int n_items;
 };
 
-template <int N, int RB>   // RB: bytes per qI / kI row (64 or 128)
+// RB: bytes per qI / kI row (64 or 128).  PAIR: 64-byte e4m3 keys are loaded
+// two to a 128-byte row (the TMA engine's cost is per row, not per byte), so
+// an item covers 256 keys: A row r holds keys 2r and 2r+1 in its two halves.
+template <int N, int RB, bool PAIR = false>
 struct IdxCfg {
-    static constexpr int kBoxRows = 64;                       // A is loaded as 2 boxes of 64 keys
-    static constexpr int kABytes = 128 * RB;
+    static_assert(!PAIR || (RB == 64 && N == 16), "paired rows serve the 64-byte decode tile");
+    static constexpr int kKeys = PAIR ? 256 : 128;            // keys per item
+    static constexpr int kKeysPerRow = PAIR ? 2 : 1;
+    static constexpr int kARowBytes = RB * kKeysPerRow;       // 128 rows of A per item
+    static constexpr int kBoxRows = 64 / kKeysPerRow;         // one TMA box = 64 keys (one cache page)
+    static constexpr int kBoxes = kKeys / 64;
+    static constexpr int kABytes = 128 * kARowBytes;
+    static constexpr int kBoxBytes = kABytes / kBoxes;
     static constexpr int kBBytes = N * RB;
     static constexpr int kStageBytes = kABytes + kBBytes;
     static constexpr int kStages = (N == 256) ? 4 : 8;
@@ -67,13 +76,16 @@ struct IdxCfg {
     static constexpr int kCG = (N == 256) ? 2 : 1;
     static constexpr int kIG = (N == 256) ? 2 : 4;
     static constexpr int kAcc = (N == 256) ? 2 : 8;           // TMEM accumulators (multiple of kIG)
+    static constexpr int kAccCols = N * kKeysPerRow;           // PAIR: even keys, then odd keys
     static constexpr int kEpiWarps = 4 * kCG * kIG;
     static constexpr int kThreads = (2 + kEpiWarps) * 32;
-    static constexpr uint32_t kTmemCols = (kAcc * N <= 32) ? 32 : (kAcc * N <= 64) ? 64 : (kAcc * N <= 128) ? 128
-                                        : (kAcc * N <= 256) ? 256 : 512;
-    static constexpr uint32_t kSwizzleBytes = RB;              // 128 or 64
-    static constexpr uint32_t kSbo = 8 * kSwizzleBytes;        // 8-row core group stride
-    static constexpr uint32_t kLayout = (RB == 128) ? 2 : 4;   // UMMA layout: 128B / 64B swizzle
+    static constexpr int kCols = kAcc * kAccCols;
+    static constexpr uint32_t kTmemCols = (kCols <= 32) ? 32 : (kCols <= 64) ? 64 : (kCols <= 128) ? 128
+                                        : (kCols <= 256) ? 256 : 512;
+    // UMMA K-major operands: 8-row core group stride and layout (2 = 128B,
+    // 4 = 64B swizzle), for A (keys) and B (query-head rows)
+    static constexpr uint32_t kSboA = 8 * kARowBytes, kLayoutA = (kARowBytes == 128) ? 2 : 4;
+    static constexpr uint32_t kSboB = 8 * RB, kLayoutB = (RB == 128) ? 2 : 4;
     static constexpr int kGroupCols = N / kCG;                 // TMEM columns per epilogue warp
     static constexpr size_t kWStage = (size_t)kEpiWarps * kGroupCols * 8;   // w (fp32) + n_valid per warp
     static constexpr size_t kSmemUsed = 1024 + (size_t)kStages * kStageBytes + 1024 + kWStage;
@@ -83,7 +95,7 @@ struct IdxCfg {
     static_assert(kAcc % kIG == 0, "item groups must own whole accumulators");
 };
 
-// One work item: query tile qt of batch b against key tile kt (128 keys).
+// One work item: query tile qt of batch b against key tile kt (kKeys keys).
 struct ItemInfo {
     int b, qt, kt, ext;   // ext: the tile's key extent (largest n_valid of its queries)
 };
@@ -112,11 +124,11 @@ __device__ __forceinline__ bool item_at(const IdxKernelArgs &a, int i, ItemInfo 
     return true;
 }
 
-template <int N, int RB, int H_I, bool F8>
-__global__ void __launch_bounds__(IdxCfg<N, RB>::kThreads, 1)
+template <int N, int RB, int H_I, bool F8, bool PAIR>
+__global__ void __launch_bounds__(IdxCfg<N, RB, PAIR>::kThreads, 1)
     indexer_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_q,
                       IdxKernelArgs a) {
-    using C = IdxCfg<N, RB>;
+    using C = IdxCfg<N, RB, PAIR>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *stage_base = smem;
@@ -159,25 +171,23 @@ __global__ void __launch_bounds__(IdxCfg<N, RB>::kThreads, 1)
         for (int base = 0; ok; base += 32) {
             ItemInfo it;
             const bool in = item_at(a, base + lane, it);
-            const bool valid = in && it.kt * 128 < it.ext;
-            // the two 64-key boxes of this lane's item: cache rows, or -1 (skip)
-            int row0 = -1, row1 = -1;
-            if (valid) {
+            const bool valid = in && it.kt * C::kKeys < it.ext;
+            // the 64-key boxes of this lane's item: rows of the key map, or -1 (skip)
+            int rows[C::kBoxes];
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const int s0 = it.kt * 128 + i * C::kBoxRows;
-                    int row = -1;
-                    if (s0 < it.ext) {
-                        if (a.page_table) {
-                            const int pid = __ldg(a.page_table + (int64_t)it.b * a.max_pages + (s0 >> 6));
-                            if (pid < 0 || pid >= a.pool_pages) report(a.dev_status, SA_DEV_INDEX);
-                            else row = pid * 64;
-                        } else {
-                            row = it.b * a.S + s0;
-                        }
+            for (int i = 0; i < C::kBoxes; ++i) {
+                const int s0 = it.kt * C::kKeys + i * 64;
+                int row = -1;
+                if (valid && s0 < it.ext) {
+                    if (a.page_table) {
+                        const int pid = __ldg(a.page_table + (int64_t)it.b * a.max_pages + (s0 >> 6));
+                        if (pid < 0 || pid >= a.pool_pages) report(a.dev_status, SA_DEV_INDEX);
+                        else row = pid * C::kBoxRows;
+                    } else {
+                        row = (it.b * a.S + s0) / C::kKeysPerRow;   // even for PAIR (S even)
                     }
-                    (i == 0 ? row0 : row1) = row;
                 }
+                rows[i] = row;
             }
             if (__ballot_sync(0xffffffffu, in) == 0) break;
             uint32_t vmask = __ballot_sync(0xffffffffu, valid);
@@ -185,16 +195,22 @@ __global__ void __launch_bounds__(IdxCfg<N, RB>::kThreads, 1)
                 const int j = __ffs(vmask) - 1;
                 vmask &= vmask - 1;
                 const int qrow = __shfl_sync(0xffffffffu, (it.b * a.T + it.qt * a.QT) * H_I, j);
-                const int r0 = __shfl_sync(0xffffffffu, row0, j), r1 = __shfl_sync(0xffffffffu, row1, j);
+                int r[C::kBoxes];
+                uint32_t nbox = 0;
+#pragma unroll
+                for (int i = 0; i < C::kBoxes; ++i) {
+                    r[i] = __shfl_sync(0xffffffffu, rows[i], j);
+                    nbox += r[i] >= 0;
+                }
                 if (lane == 0) {
                     ok = mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag);
                     if (ok) {
                         uint8_t *sa_ = stage_base + stage * C::kStageBytes;
-                        const uint32_t bytes = C::kBBytes + (uint32_t)((r0 >= 0) + (r1 >= 0)) * (C::kABytes / 2);
-                        mbar_arrive_expect_tx(&full_bar[stage], bytes);
+                        mbar_arrive_expect_tx(&full_bar[stage], C::kBBytes + nbox * C::kBoxBytes);
                         tma_load_2d(sa_ + C::kABytes, &map_q, 0, qrow, &full_bar[stage]);
-                        if (r0 >= 0) tma_load_2d(sa_, &map_k, 0, r0, &full_bar[stage]);
-                        if (r1 >= 0) tma_load_2d(sa_ + C::kABytes / 2, &map_k, 0, r1, &full_bar[stage]);
+#pragma unroll
+                        for (int i = 0; i < C::kBoxes; ++i)
+                            if (r[i] >= 0) tma_load_2d(sa_ + i * C::kBoxBytes, &map_k, 0, r[i], &full_bar[stage]);
                         ++issued;
                     }
                 }
@@ -223,7 +239,7 @@ __global__ void __launch_bounds__(IdxCfg<N, RB>::kThreads, 1)
         for (int base = 0; ok; base += 32) {
             ItemInfo it;
             const bool in = item_at(a, base + lane, it);
-            const bool valid = in && it.kt * 128 < it.ext;
+            const bool valid = in && it.kt * C::kKeys < it.ext;
             if (__ballot_sync(0xffffffffu, in) == 0) break;
             const int nvalid = __popc(__ballot_sync(0xffffffffu, valid));
             for (int k = 0; k < nvalid; ++k, ++c) {
@@ -236,13 +252,19 @@ __global__ void __launch_bounds__(IdxCfg<N, RB>::kThreads, 1)
                         tc_fence_after();
                         const uint32_t a_addr = smem_u32(stage_base + stage * C::kStageBytes);
                         const uint32_t b_addr = a_addr + C::kABytes;
-                        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * N);
+                        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * C::kAccCols);
+                        // PAIR: the even keys sit in bytes 0..63 of each A row,
+                        // the odd keys in bytes 64..127; one accumulator each
 #pragma unroll
-                        for (int kk = 0; kk < RB / 32; ++kk) {
-                            const uint64_t da = smem_desc(a_addr + kk * 32, C::kSbo, C::kLayout);
-                            const uint64_t db = smem_desc(b_addr + kk * 32, C::kSbo, C::kLayout);
-                            if constexpr (F8) tc_mma_f8(d_tmem, da, db, idesc, kk > 0 ? 1u : 0u);
-                            else tc_mma_f16(d_tmem, da, db, idesc, kk > 0 ? 1u : 0u);
+                        for (int h = 0; h < C::kKeysPerRow; ++h) {
+#pragma unroll
+                            for (int kk = 0; kk < RB / 32; ++kk) {
+                                const uint64_t da = smem_desc(a_addr + h * RB + kk * 32, C::kSboA, C::kLayoutA);
+                                const uint64_t db = smem_desc(b_addr + kk * 32, C::kSboB, C::kLayoutB);
+                                const uint32_t d = d_tmem + (uint32_t)(h * N);
+                                if constexpr (F8) tc_mma_f8(d, da, db, idesc, kk > 0 ? 1u : 0u);
+                                else tc_mma_f16(d, da, db, idesc, kk > 0 ? 1u : 0u);
+                            }
                         }
                         tc_commit(&empty_bar[stage]);
                         tc_commit(&tfull_bar[acc]);
@@ -281,7 +303,7 @@ __global__ void __launch_bounds__(IdxCfg<N, RB>::kThreads, 1)
         for (int base = 0; ok; base += 32) {
             ItemInfo mine;
             const bool in = item_at(a, base + lane, mine);
-            const bool valid = in && mine.kt * 128 < mine.ext;
+            const bool valid = in && mine.kt * C::kKeys < mine.ext;
             if (__ballot_sync(0xffffffffu, in) == 0) break;
             uint32_t vmask = __ballot_sync(0xffffffffu, valid);
             for (; vmask; ++c) {
@@ -327,17 +349,21 @@ __global__ void __launch_bounds__(IdxCfg<N, RB>::kThreads, 1)
                 for (int k = 0; k < NVREGS; ++k)
                     if (lane + 32 * k < QPG) nvs[lane + 32 * k] = nvr[k];
                 __syncwarp();
-                const int s = kt * 128 + quad * 32 + lane;
+                constexpr int KPR = C::kKeysPerRow;
+                const int s = kt * C::kKeys + (quad * 32 + lane) * KPR;   // PAIR: keys s and s + 1
                 const uint32_t t_cols = tmem_base + ((uint32_t)(quad * 32) << 16) +
-                                        (uint32_t)(acc * N + cg * C::kGroupCols);
+                                        (uint32_t)(acc * C::kAccCols + cg * C::kGroupCols);
                 float *op = a.scores + row0 * a.ld + s;
                 const bool causal = a.n_valid == nullptr;
                 const int causal_end = a.S - a.T + t_base + 1;   // row length of query q: causal_end + q
 #pragma unroll
                 for (int l0 = 0; l0 < NLD; l0 += BATCH) {
-                    uint32_t v[BATCH][16];
+                    uint32_t v[BATCH][KPR][16];
 #pragma unroll
-                    for (int bb = 0; bb < BATCH; ++bb) tmem_ld_x16(t_cols + (uint32_t)((l0 + bb) * 16), v[bb]);
+                    for (int bb = 0; bb < BATCH; ++bb)
+#pragma unroll
+                        for (int h = 0; h < KPR; ++h)
+                            tmem_ld_x16(t_cols + (uint32_t)(h * N + (l0 + bb) * 16), v[bb][h]);
                     tmem_ld_wait();
 #pragma unroll
                     for (int bb = 0; bb < BATCH; ++bb) {
@@ -356,12 +382,26 @@ __global__ void __launch_bounds__(IdxCfg<N, RB>::kThreads, 1)
 #pragma unroll
                                     for (int j1 = 0; j1 < H_I; ++j1) wv[j1] = ws[q * H_I + j1];
                                 }
-                                float sc = 0.f;
+                                float sc[KPR];
 #pragma unroll
-                                for (int j1 = 0; j1 < H_I; ++j1)
-                                    sc = fmaf(wv[j1], fmaxf(__uint_as_float(v[bb][qq * H_I + j1]), 0.f), sc);
+                                for (int h = 0; h < KPR; ++h) {
+                                    sc[h] = 0.f;
+#pragma unroll
+                                    for (int j1 = 0; j1 < H_I; ++j1)
+                                        sc[h] = fmaf(wv[j1], fmaxf(__uint_as_float(v[bb][h][qq * H_I + j1]), 0.f), sc[h]);
+                                }
                                 // causal rows (no n_valid) end at their own position
-                                if (causal ? s < causal_end + q : s < nvs[q]) *op = sc;
+                                const int lim = causal ? causal_end + q : nvs[q];
+                                if constexpr (KPR == 2) {
+                                    if (s + 1 < lim && (reinterpret_cast<uintptr_t>(op) & 7u) == 0) {
+                                        *reinterpret_cast<float2 *>(op) = make_float2(sc[0], sc[1]);
+                                    } else {
+                                        if (s < lim) op[0] = sc[0];
+                                        if (s + 1 < lim) op[1] = sc[1];
+                                    }
+                                } else {
+                                    if (s < lim) *op = sc[0];
+                                }
                             }
                             op += a.ld;
                         }
@@ -413,16 +453,16 @@ static bool make_map(CUtensorMap *m, const void *base, uint64_t rows, int RB, bo
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int N, int RB, int H_I, bool F8>
+template <int N, int RB, int H_I, bool F8, bool PAIR>
 static sa_status launch_tc(const IndexerArgs &a, cudaStream_t st) {
-    using C = IdxCfg<N, RB>;
+    using C = IdxCfg<N, RB, PAIR>;
     IdxKernelArgs k;
     k.w = a.w; k.page_table = a.page_table; k.n_valid = a.n_valid; k.scores = a.scores; k.ld = a.ld;
     k.dev_status = a.dev_status; k.max_pages = a.max_pages; k.pool_pages = a.pool_pages;
     k.B = a.B; k.T = a.T; k.S = a.S;
     k.QT = N / H_I;
     k.QTN = (a.T + k.QT - 1) / k.QT;
-    k.KT = (a.S + 127) / 128;
+    k.KT = (a.S + C::kKeys - 1) / C::kKeys;
     const long long items = (long long)a.B * k.QTN * k.KT;
     if (items > 0x7fffffffLL) return SA_ERR_UNSUPPORTED;
     k.n_items = (int)items;
@@ -430,11 +470,12 @@ static sa_status launch_tc(const IndexerArgs &a, cudaStream_t st) {
 
     CUtensorMap mk, mq;
     const uint64_t k_rows = a.page_table ? (uint64_t)a.pool_pages * a.page_size : (uint64_t)a.B * a.S;
-    if (!make_map(&mk, a.kI, k_rows, RB, F8, C::kBoxRows)) return SA_ERR_CUDA;
+    // PAIR: the key cache viewed as rows of two keys (k_rows is even: S even, or 64-key pages)
+    if (!make_map(&mk, a.kI, k_rows / C::kKeysPerRow, C::kARowBytes, F8, C::kBoxRows)) return SA_ERR_CUDA;
     if (!make_map(&mq, a.qI, (uint64_t)a.B * a.T * H_I, RB, F8, N)) return SA_ERR_CUDA;
 
-    auto kern = indexer_tc_kernel<N, RB, H_I, F8>;
-    if (prepare_kernel<indexer_tc_kernel<N, RB, H_I, F8>>(C::kSmem, false) != cudaSuccess) return SA_ERR_CUDA;
+    auto kern = indexer_tc_kernel<N, RB, H_I, F8, PAIR>;
+    if (prepare_kernel<indexer_tc_kernel<N, RB, H_I, F8, PAIR>>(C::kSmem, false) != cudaSuccess) return SA_ERR_CUDA;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -443,13 +484,13 @@ static sa_status launch_tc(const IndexerArgs &a, cudaStream_t st) {
     return cuda_ok(cudaGetLastError());
 }
 
-template <int N, int RB, bool F8>
+template <int N, int RB, bool F8, bool PAIR = false>
 static sa_status launch_tc_h(const IndexerArgs &a, cudaStream_t st) {
     switch (a.H_I) {
-        case 1: return launch_tc<N, RB, 1, F8>(a, st);
-        case 2: return launch_tc<N, RB, 2, F8>(a, st);
-        case 4: return launch_tc<N, RB, 4, F8>(a, st);
-        case 8: return launch_tc<N, RB, 8, F8>(a, st);
+        case 1: return launch_tc<N, RB, 1, F8, PAIR>(a, st);
+        case 2: return launch_tc<N, RB, 2, F8, PAIR>(a, st);
+        case 4: return launch_tc<N, RB, 4, F8, PAIR>(a, st);
+        case 8: return launch_tc<N, RB, 8, F8, PAIR>(a, st);
     }
     return SA_ERR_UNSUPPORTED;
 }
@@ -457,7 +498,11 @@ static sa_status launch_tc_h(const IndexerArgs &a, cudaStream_t st) {
 template <int RB, bool F8>
 static sa_status launch_tc_n(const IndexerArgs &a, cudaStream_t st) {
     const bool small = a.T * a.H_I <= 16;   // decode: a handful of queries per sequence
-    return small ? launch_tc_h<16, RB, F8>(a, st) : launch_tc_h<256, RB, F8>(a, st);
+    if (!small) return launch_tc_h<256, RB, F8>(a, st);
+    // 64-byte e4m3 keys, two to a TMA row, when rows pair up: 64-key pages, or an even S
+    if constexpr (F8 && RB == 64)
+        if (a.page_table || a.S % 2 == 0) return launch_tc_h<16, 64, true, true>(a, st);
+    return launch_tc_h<16, RB, F8>(a, st);
 }
 
 sa_status launch_indexer(const IndexerArgs &a, cudaStream_t st) {

@@ -167,6 +167,7 @@ def test_convert_e4m3_matches_oracle(sa):
 @pytest.mark.parametrize("N,H_I,D_I,rows", [
     (512, 2, 64, None), (1000, 4, 64, None), (300, 8, 128, None), (777, 1, 128, None),
     (129, 4, 64, None), (1, 4, 64, None), (8192, 4, 64, 384), (8192, 8, 128, 200),
+    (2, 8, 64, None), (4, 4, 64, None), (3, 4, 64, None),   # 16-column tile: paired rows iff S even
 ])
 def test_indexer_fp8_prefill_exact(sa, N, H_I, D_I, rows):
     inp = gen_prefill(N=N, Hq=1, d=64, H_I=H_I, D_I=D_I, seed=N + 7 * H_I)
@@ -209,6 +210,33 @@ def test_indexer_fp8_general_codes_within_fp32_sum_bound(sa):
     for i, t_ in enumerate(rows):
         err = np.abs(got[t_, :t_ + 1] - want[i, :t_ + 1])
         assert np.all(err <= (D_I + H_I) * 2.0 ** -24 * mag[i, :t_ + 1]), (t_, err.max())
+
+
+@pytest.mark.parametrize("lengths", [[1, 2, 3, 255, 256, 257, 511, 1000],   # even S: two keys per TMA row
+                                     [1, 999, 513, 64]])                     # odd S: one key per row
+def test_indexer_fp8_decode_edge_lengths(sa, lengths):
+    B = len(lengths)
+    for paged in (False, True):
+        inp = gen_decode(B=B, lengths=lengths, Hq=16, d=64, H_I=8, D_I=64, paged=paged, seed=8)
+        t = _to_dev(inp, ("qI", "w", "kI"))
+        q8, k8 = _e4m3_dev(sa, t["qI"]), _e4m3_dev(sa, t["kI"])
+        if paged:
+            S = inp["page_table"].shape[1] * 64
+            pt, mp, pp = dev(inp["page_table"]), inp["page_table"].shape[1], inp["kI"].shape[0]
+        else:
+            S, pt, mp, pp = inp["kI"].shape[1], None, 0, 0
+        ld = (S + 3) // 4 * 4
+        sc = torch.full((B, ld), float("nan"), device="cuda")
+        ds = torch.zeros(1, dtype=torch.int32, device="cuda")
+        sa.sa_indexer_scores_fp8(q8, t["w"], k8, pt, mp, pp, 64, B, 1, S, 8, 64, dev(inp["lengths"]), sc, ld, ds)
+        got = sc.cpu().numpy()
+        assert status(ds) == 0
+        for b, L in enumerate(lengths):
+            _, _, kI = oracle.decode_sequence(inp, b)
+            want = oracle.indexer_fp8(oracle.e4m3_encode(inp["qI"][b:b + 1]), inp["w"][b:b + 1],
+                                      oracle.e4m3_encode(kI), [L - 1])
+            assert np.array_equal(got[b, :L], want[0]), (paged, b)
+            assert np.all(np.isnan(got[b, L:S])), (paged, b)   # columns past the row are not written
 
 
 def test_indexer_fp8_decode_contiguous_and_paged(sa):
