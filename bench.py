@@ -88,6 +88,34 @@ def ncu_traffic(workload: str, stage: str):
     return None
 
 
+# --------------------------------------------------------------------------- ranks
+def barrier(world, local_rank=None):
+    """All ranks meet (NCCL: on this rank's GPU); a no-op for one rank."""
+    if world > 1:
+        import torch.distributed as dist
+        if local_rank is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[local_rank])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(x: float, world: int, device="cpu") -> float:
+    """The largest of the ranks' values (a timed region ends when the slowest
+    rank's does); every rank gets the result."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: int, world: int, steps: int, total_ms: float) -> float:
+    """Units processed by all ranks per second of the (max-over-ranks) timed region."""
+    return units_per_rank * world * steps / (total_ms / 1e3)
+
+
 # --------------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
@@ -299,7 +327,6 @@ def oracle_rate(case, budget_s=8.0):
 # --------------------------------------------------------------------------- arms
 def run_ours(args, rank, world, local_rank):
     import torch
-    import torch.distributed as dist
 
     device = "cuda:%d" % local_rank
     torch.cuda.set_device(local_rank)
@@ -320,9 +347,8 @@ def run_ours(args, rank, world, local_rank):
     if int(plan.dev_status.item()) != 0:
         raise RuntimeError("device status %d during warm-up" % int(plan.dev_status.item()))
 
-    def barrier():
-        if world > 1:
-            dist.barrier(device_ids=[local_rank])
+    def sync_all():
+        barrier(world, local_rank)
         torch.cuda.synchronize()
 
     # ---- device-resident timed steps.  The step -- every C-ABI call of the
@@ -345,22 +371,18 @@ def run_ours(args, rank, world, local_rank):
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
     gpu_idx = vis.split(",")[local_rank] if vis else str(local_rank)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    barrier()
+    sync_all()
     with ClockSampler(gpu_idx) as clk:
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
             ev[i][0].record(stream)
             graph.replay()
             ev[i][1].record(stream)
-        barrier()
+        sync_all()
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = float(sum(step_ms))
-    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(float(sum(step_ms)), world, device)
     ms_per_step = total_ms / args.steps
-    value = case["units"] * world * args.steps / (total_ms / 1e3)
+    value = whole_job_rate(case["units"], world, args.steps, total_ms)
 
     # per-kernel times: the stage graphs replayed back to back in step order,
     # an event between consecutive kernels (not part of the reported value)
@@ -388,7 +410,7 @@ def run_ours(args, rank, world, local_rank):
     d2h = out_host.numel() * out_host.element_size()
     pipe.run([hin] * 2, [out_host] * 2)   # warm-up
     torch.cuda.synchronize()
-    barrier()
+    sync_all()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(pipe.up)
     # no L2 flush here: each step uploads fresh inputs and moves far more than
@@ -397,11 +419,9 @@ def run_ours(args, rank, world, local_rank):
     pipe.run([hin] * args.steps, [out_host] * args.steps)
     e1.record(pipe.down)
     torch.cuda.synchronize()
-    barrier()
-    t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    e2e_value = case["units"] * world * args.steps / (float(t.item()) / 1e3)
+    sync_all()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device)
+    e2e_value = whole_job_rate(case["units"], world, args.steps, e2e_ms)
     if int(plan.dev_status.item()) != 0 or pipe.dev_status() != 0:
         raise RuntimeError("device status %d" % (int(plan.dev_status.item()) | pipe.dev_status()))
     del pipe
