@@ -144,7 +144,7 @@ def test_e4m3_round_trip_ties_and_saturation():
     assert np.array_equal(oracle.e4m3_encode(oracle.e4m3_decode(codes)), codes)
     cases = {1.0: 0x38, 1.0625: 0x38, 1.1875: 0x3A, 2.0 ** -9: 0x01, 2.0 ** -10: 0x00,
              3 * 2.0 ** -10: 0x02, 2.0 ** -6: 0x08, 15 * 2.0 ** -10: 0x08, 448.0: 0x7E,
-             460.0: 0x7E, 1e9: 0x7E, -1e9: 0xFE, -math.inf: 0xFE, math.inf: 0x7E, -2.0: 0xC0,
+             460.0: 0x7E, 470.0: 0x7E, 480.0: 0x7E, 1e9: 0x7E, -1e9: 0xFE, -math.inf: 0xFE, math.inf: 0x7E, -2.0: 0xC0,
              3.0: 0x44, -3.0: 0xC4, 0.0: 0x00}
     got = oracle.e4m3_encode(np.array(list(cases)))
     assert got.tolist() == list(cases.values())
