@@ -13,6 +13,7 @@ Functions (each cites the passage it follows in ``sa_oracle.c``):
 ``topk``              K best scores per row, ties -> lower position, ascending
 ``pool_mean``         mean of each complete block of index keys
 ``two_stage``         coarse block top-k, then fine top-K inside the blocks
+``page_selection``    whole kept blocks (+ own block), no fine pass
 ``selection``         S(t) = TopK(t) U {max(0,t-W+1) .. t}
 ``sparse_attention``  softmax(q.k * scale) v over S(t)
 ``prefill`` / ``decode``  the three stages end to end
@@ -163,6 +164,18 @@ def two_stage(t_pos, qI, w, kI, blk, keep, K):
     _load().oracle_two_stage(R, t_pos, H, D, qI.reshape(-1), w.reshape(-1), kI.shape[0],
                              kI.reshape(-1), blk, keep, K, topk_out, blocks, threads())
     return topk_out, blocks
+
+
+def page_selection(t_pos, qI, w, kI, blk, keep):
+    """Page-granular selection: whole blocks instead of single tokens (the
+    64-token page selection of "Sparse Attention" (completesystemdesign.dev),
+    DSA list, and the block routing of "Sparse Attention in 2026", "The
+    designs that shipped").  The coarse pass keeps `keep` blocks, and the
+    selection is every token of those blocks plus the query's own block up to
+    t, with no fine pass.  That is the two-stage selection whose fine top-K
+    may keep all keep*blk + blk candidates, so it is computed as such.
+    Returns (positions [R, keep*blk + blk] ascending, -1 padded; blocks)."""
+    return two_stage(t_pos, qI, w, kI, blk, keep, keep * blk + blk)
 
 
 def selection(topk_rows, W, t_pos):

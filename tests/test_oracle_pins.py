@@ -272,6 +272,43 @@ def test_two_stage_planted_block_and_own_block():
     assert list(top2[0]) == list(range(24, 32))      # score 1 beats the own block's 0
 
 
+def _page_selection_brute(t, qI, w, kI, blk, keep):
+    """Plain-Python page selection: pooled block keys, coarse scores, the best
+    `keep` eligible blocks (ties to the lower block), their tokens and the
+    query's own block up to t, ascending."""
+    own = t // blk
+    scored = []
+    for b in range(own):
+        kb = kI[b * blk:(b + 1) * blk].mean(axis=0)
+        sc = sum(w[j] * max(0.0, float(np.dot(qI[j], kb))) for j in range(qI.shape[0]))
+        scored.append((-sc, b))
+    kept = sorted(b for _, b in sorted(scored)[:keep])
+    return [s for b in kept for s in range(b * blk, (b + 1) * blk)] + list(range(own * blk, t + 1))
+
+
+@pytest.mark.parametrize("keep", [0, 1, 3, 50])
+def test_page_selection_brute_force(keep):
+    blk, N = 8, 160
+    inp = gen_prefill(N=N, Hq=1, d=64, H_I=2, D_I=32, seed=21 + keep)   # small integers: many ties
+    qI, w, kI = (oracle._f64(inp[x]) for x in ("qI", "w", "kI"))
+    rows = np.arange(N)
+    pos, blocks = oracle.page_selection(rows, qI, w, kI, blk, keep)
+    assert pos.shape == (N, keep * blk + blk)
+    for t in rows:
+        want = _page_selection_brute(int(t), qI[t], w[t], kI, blk, keep)
+        assert list(pos[t, :len(want)]) == want, t
+        assert np.all(pos[t, len(want):] == -1), t
+
+
+def test_page_selection_keeping_every_block_is_dense_causal():
+    blk, N = 16, 96
+    inp = gen_prefill(N=N, Hq=2, d=64, H_I=2, D_I=32, seed=9)
+    keep = N // blk
+    res = oracle.prefill(inp, K=keep * blk + blk, W=4, block=blk, keep=keep)
+    q, k, v = (oracle._f64(inp[x]) for x in "qkv")
+    assert np.max(np.abs(res["out"] - _dense_causal_textbook(q, k, v, 1.0 / 8.0))) < 1e-12
+
+
 # ---------------------------------------------------------------- selection
 def test_selection_window_and_union():
     ptr, idx = oracle.selection(np.array([[-1, -1]]), 3, [0])
