@@ -128,9 +128,12 @@ class PrefillPlan:
         return self.out
 
     def launches(self) -> int:
-        """Kernels one run() enqueues."""
+        """Kernels one run() enqueues: indexer + top-K (per row block), or for
+        the two-stage selection pool, block counts, coarse indexer, coarse
+        top-k, expand, the fine scores' invert count / scan / scatter and
+        block kernel, and the fine top-K (10); then the attention."""
         attn = 2 if self.attn_ws is not None else 1   # (selection bitmap +) attention
-        return (2 * self.row_blocks if self.block is None else 11) + attn
+        return (2 * self.row_blocks if self.block is None else 10) + attn
 
 
 class DecodePlan:
@@ -179,7 +182,14 @@ class DecodePlan:
         return self.out
 
     def launches(self) -> int:
-        return 4   # indexer, top-K, split attention, merge
+        """Kernels one run() enqueues: indexer, top-K, then the attention of
+        sa_sparse_attn_decode.  That is one kernel when a thread-block cluster
+        of G = min(16, max(1, ceil((K+W)/128), ceil(Hq/8))) CTAs per sequence
+        leaves each CTA at most 1024 keys (partials merged in distributed
+        shared memory), else a split-K kernel and a merge kernel."""
+        kw = self.K + self.W
+        G = min(16, max(1, -(-kw // 128), -(-self.Hq // 8)))
+        return 2 + (1 if -(-kw // G) <= 1024 else 2)
 
 
 class HostPipeline:
