@@ -6,8 +6,9 @@
 A step is one pass of the whole path -- indexer -> top-K -> sparse attention
 (for the two-stage workload: pool, coarse scores, coarse top-k, expand, fine
 scores, top-K, attention) -- over one synthetic batch.  The default workload is
-the 8K-token causal prefill (16 query heads, d=128, indexer 4 x 64, top-K 1024,
-window 128).  Each rank runs its own independent sequence (weak scaling, no
+the largest one that fits one GPU: the two-stage 65536-token causal prefill (16
+query heads, d=128, one KV head, indexer 4 x 64, 64-token blocks, 64 kept
+blocks, top-K 2048, window 512).  Each rank runs its own independent sequence (weak scaling, no
 collective on the data path).  One JSON line is printed by rank 0.
 
 Timing: the step (every C-ABI call of the path) is captured once as a CUDA
@@ -75,16 +76,17 @@ def source_hash(cu: str) -> str:
 
 
 def ncu_traffic(workload: str, stage: str):
-    """DRAM read+write bytes per launch from profiles/dram_traffic.md, if that
-    capture was taken from the kernel source that is built now; else None."""
-    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    """DRAM read+write bytes per launch for a stage, from the ncu capture data
+    in profiles/dram_traffic.json, if that capture was taken from the kernel
+    source that is built now (scaled to the full workload when the capture ran
+    a smaller case); else None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if stage not in STAGE_SOURCE or not os.path.exists(path):
         return None
     want = source_hash(STAGE_SOURCE[stage])
-    for line in open(path):
-        f = [x.strip() for x in line.strip().strip("|").split("|")]
-        if len(f) == 5 and f[0] == workload and f[1] == stage and f[3] == want and f[4].isdigit():
-            return int(f[4])
+    for e in json.load(open(path)).get("entries", []):
+        if e.get("workload") == workload and e.get("stage") == stage and e.get("source_hash") == want:
+            return int(round(float(e["bytes_per_launch"]) * float(e.get("scale", 1.0))))
     return None
 
 
@@ -503,7 +505,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="prefill_8k")
+    ap.add_argument("--workload", default="prefill_64k_two_stage")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--index-fp8", action="store_true",

@@ -165,8 +165,9 @@ __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
 
 // 2^y for a pair, on the FMA pipe instead of the ex2 unit.  Range reduction:
 // adding 1.5 * 2^23 rounds y to the nearest integer r in the low mantissa bits
-// of t (exact for |y| < 2^22), f = y - r lies in [-1/2, 1/2], and 2^f is a
-// cubic fitted to it in relative error (max 7.5e-5, well below bf16's 2^-8
+// of t (exact for |y| < 2^22), f = y - r lies in [-1/2, 1/2], and 2^f is the
+// cubic of least maximum relative error on [-1/2, 1/2] (the minimax fit, found
+// by the Remez exchange algorithm: max 7.48e-5, well below bf16's 2^-8
 // spacing).  r is added to the exponent field of 2^f: the shifter's own bits
 // shifted left by 23 vanish mod 2^32, so t_bits << 23 == r << 23.  y is first
 // raised to -126, where 2^y is below 2^-125 (masked keys, y = -inf, end there

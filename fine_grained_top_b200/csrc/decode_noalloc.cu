@@ -22,7 +22,11 @@
 //     same call has written first.
 // The first call on a device looks up the array's device address (once per
 // device, with that device current); make that first call before any stream
-// capture.  Nothing here calls cudaMalloc, cudaFree or an allocating routine.
+// capture.  The address is cached per device index for the life of the
+// process.  cudaDeviceReset unloads the device's copy of the library's module,
+// which leaves the cached address stale: a process that resets a device must
+// not call this entry point on that device afterwards.  Nothing here calls
+// cudaMalloc, cudaFree or an allocating routine.
 #include <mutex>
 
 #include "../../include/sa.h"
@@ -47,7 +51,12 @@ sa_status scratch_address(void **out) {
     std::lock_guard<std::mutex> lock(g_scratch_mu);
     if (g_scratch_addr[dev] == nullptr) {
         void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return SA_ERR_CUDA;
+        if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) {
+            // clear the runtime's last-error slot, so that the failure is not
+            // reported again by an unrelated later call
+            (void)cudaGetLastError();
+            return SA_ERR_CUDA;
+        }
         g_scratch_addr[dev] = p;
     }
     *out = g_scratch_addr[dev];
@@ -59,26 +68,16 @@ sa_status scratch_address(void **out) {
 
 using namespace sa;
 
+
 extern "C" sa_status sa_sparse_attn_decode_noalloc(const sa_bf16 *q, const sa_bf16 *k_cache,
                                                    const sa_bf16 *v_cache, const int32_t *page_table,
                                                    int max_pages, int pool_pages, int page_size, int S_max,
                                                    const int32_t *seq_lens, const int32_t *topk, int K, int W,
                                                    int B, int Hq, int d, float scale, sa_bf16 *out, float *lse,
                                                    int *dev_status, sa_stream stream) {
-    if (K < 0 || W < 0 || B < 0 || S_max < 0) return SA_ERR_INVALID_ARG;
-    if (!(d == 64 || d == 128) || Hq < 1 || Hq > 64) return SA_ERR_UNSUPPORTED;
-    if (B == 0) return SA_OK;
-    if (!q || !k_cache || !v_cache || !seq_lens || !out || (K > 0 && !topk)) return SA_ERR_INVALID_ARG;
-    const uintptr_t mis = (reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k_cache) |
-                           reinterpret_cast<uintptr_t>(v_cache)) & 15u;
-    if (mis) return SA_ERR_INVALID_ARG;
-    if (page_table) {
-        if (page_size != 64) return SA_ERR_UNSUPPORTED;
-        if (max_pages <= 0 || pool_pages <= 0) return SA_ERR_INVALID_ARG;
-        if ((int64_t)pool_pages * 64 > INT32_MAX) return SA_ERR_UNSUPPORTED;
-    } else if ((int64_t)B * S_max > INT32_MAX) {
-        return SA_ERR_UNSUPPORTED;
-    }
+    const sa_status chk = check_decode_args(q, k_cache, v_cache, page_table, max_pages, pool_pages, page_size,
+                                            S_max, seq_lens, topk, K, W, B, Hq, d, out);
+    if (chk != SA_OK || B == 0) return chk;
     if (decode_workspace_bytes(B, Hq, d, K, W) > (size_t)SA_DECODE_NOALLOC_SCRATCH_BYTES)
         return SA_ERR_WORKSPACE;   // the partial results would not fit in the fixed array
     try {

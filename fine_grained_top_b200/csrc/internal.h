@@ -98,6 +98,30 @@ struct DecodeArgs {
 size_t decode_workspace_bytes(int B, int Hq, int d, int K, int W);
 sa_status launch_decode(const DecodeArgs &a, cudaStream_t st);
 
+// Argument rules shared by every decode entry point (with or without a caller
+// workspace): SA_OK when the call may proceed to its workspace checks.  A call
+// with B == 0 passes and enqueues nothing.
+inline sa_status check_decode_args(const void *q, const void *k_cache, const void *v_cache,
+                                   const int32_t *page_table, int max_pages, int pool_pages, int page_size,
+                                   int S_max, const int32_t *seq_lens, const int32_t *topk, int K, int W, int B,
+                                   int Hq, int d, const void *out) {
+    if (K < 0 || W < 0 || B < 0 || S_max < 0) return SA_ERR_INVALID_ARG;
+    if (!(d == 64 || d == 128) || Hq < 1 || Hq > 64) return SA_ERR_UNSUPPORTED;
+    if (B == 0) return SA_OK;
+    if (!q || !k_cache || !v_cache || !seq_lens || !out || (K > 0 && !topk)) return SA_ERR_INVALID_ARG;
+    const uintptr_t mis = (reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(k_cache) |
+                           reinterpret_cast<uintptr_t>(v_cache)) & 15u;
+    if (mis) return SA_ERR_INVALID_ARG;
+    if (page_table) {
+        if (page_size != 64) return SA_ERR_UNSUPPORTED;
+        if (max_pages <= 0 || pool_pages <= 0) return SA_ERR_INVALID_ARG;
+        if ((int64_t)pool_pages * 64 > INT32_MAX) return SA_ERR_UNSUPPORTED;
+    } else if ((int64_t)B * S_max > INT32_MAX) {
+        return SA_ERR_UNSUPPORTED;
+    }
+    return SA_OK;
+}
+
 sa_status launch_pool(const uint16_t *kI, int S, int D_I, int block, uint16_t *kB, cudaStream_t st);
 sa_status launch_block_counts(int T, int S, int block, int32_t *n_blocks, cudaStream_t st);
 sa_status launch_expand(const int32_t *blocks, int T, int S, int keep, int block, int32_t *cand,

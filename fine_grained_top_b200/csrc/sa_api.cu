@@ -197,18 +197,9 @@ sa_status sa_sparse_attn_decode(const sa_bf16 *q, const sa_bf16 *k_cache, const 
                                 const int32_t *seq_lens, const int32_t *topk, int K, int W, int B, int Hq, int d,
                                 float scale, sa_bf16 *out, float *lse, void *workspace, size_t workspace_bytes,
                                 int *dev_status, sa_stream stream) {
-    if (K < 0 || W < 0 || B < 0 || S_max < 0) return SA_ERR_INVALID_ARG;
-    if (!head_dim_ok(d) || Hq < 1 || Hq > 64) return SA_ERR_UNSUPPORTED;
-    if (B == 0) return SA_OK;
-    if (!q || !k_cache || !v_cache || !seq_lens || !out || (K > 0 && !topk)) return SA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return SA_ERR_INVALID_ARG;
-    if (page_table) {
-        if (page_size != 64) return SA_ERR_UNSUPPORTED;
-        if (max_pages <= 0 || pool_pages <= 0) return SA_ERR_INVALID_ARG;
-        if ((int64_t)pool_pages * 64 > INT32_MAX) return SA_ERR_UNSUPPORTED;
-    } else if ((int64_t)B * S_max > INT32_MAX) {
-        return SA_ERR_UNSUPPORTED;
-    }
+    const sa_status chk = check_decode_args(q, k_cache, v_cache, page_table, max_pages, pool_pages, page_size,
+                                            S_max, seq_lens, topk, K, W, B, Hq, d, out);
+    if (chk != SA_OK || B == 0) return chk;
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return SA_ERR_INVALID_ARG;
     if (workspace_bytes < decode_workspace_bytes(B, Hq, d, K, W)) return SA_ERR_WORKSPACE;
     return guarded([&] {

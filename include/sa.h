@@ -255,9 +255,14 @@ sa_status sa_sparse_attn_prefill(const sa_bf16 *q, const sa_bf16 *k,
  *   (its own k/v/kI already appended).  Key set and output as in prefill.
  *   k_cache/v_cache: contiguous (page_table == NULL) [B, S_max, d]; paged:
  *   pools [P, page_size, d] addressed through page_table [B, max_pages].
- *   The selection is split into chunks processed by separate CTAs; their
- *   partial softmax states go to `workspace` and a second kernel merges them
- *   (log-sum-exp).  workspace: device memory of at least
+ *   Each sequence's selection is split into chunks processed by separate
+ *   CTAs, whose partial softmax states are merged by log-sum-exp.  When
+ *   every chunk fits one CTA of a thread-block cluster (G = min(16,
+ *   max(ceil((K+W)/128), ceil(Hq/8))) CTAs per sequence, at most 1024 keys
+ *   each), the merge runs inside the same kernel through distributed shared
+ *   memory and `workspace` is not touched.  Otherwise the partial states go to
+ *   `workspace` and a second kernel merges them.  workspace: device memory of
+ *   at least
  *   sa_decode_workspace_bytes(B, Hq, d, K, W) bytes, 256-byte aligned, owned
  *   by the caller; contents on entry do not matter.
  *   Errors: SA_ERR_WORKSPACE if too small; SA_ERR_UNSUPPORTED if B * S_max
@@ -296,7 +301,8 @@ sa_status sa_sparse_attn_decode(const sa_bf16 *q, const sa_bf16 *k_cache,
  *   The array keeps the previous call's contents; nothing in it needs to start
  *   at zero.  The first call on a device looks up the array's address on that
  *   device (set-up, once per device); make that first call before any stream
- *   capture.  This entry point never calls cudaMalloc, cudaFree or any
+ *   capture.  The address stays cached for the life of the process; after
+ *   cudaDeviceReset on a device, do not call this entry point on it again.  This entry point never calls cudaMalloc, cudaFree or any
  *   allocating routine.
  * ---------------------------------------------------------------------- */
 #define SA_DECODE_NOALLOC_SCRATCH_BYTES (16u << 20)

@@ -59,3 +59,34 @@ def test_relative_error_over_kernel_range():
 def test_masked_keys_end_below_2_pow_minus_125():
     got = _exp2_fma(np.array([-np.inf, -1e30, -200.0, -126.0], np.float32)).astype(np.float64)
     assert np.all(got >= 0.0) and np.all(got < 2.0 ** -125)
+
+
+def _remez_relative(deg, a, b, f, iters=40):
+    """Minimax polynomial of degree `deg` in relative error on [a, b], by the
+    Remez exchange: solve for equioscillation on deg + 2 reference points,
+    move the references to the extrema of the error, repeat."""
+    n = deg + 2
+    x = (a + b) / 2 + (b - a) / 2 * np.cos(np.pi * np.arange(n)[::-1] / (n - 1))
+    grid = np.linspace(a, b, 200001)
+    for _ in range(iters):
+        A = np.zeros((n, n))
+        A[:, :deg + 1] = x[:, None] ** np.arange(deg + 1)
+        A[:, deg + 1] = (-1.0) ** np.arange(n) * f(x)
+        coef = np.linalg.solve(A, f(x))[:deg + 1]
+        err = np.polyval(coef[::-1], grid) / f(grid) - 1.0
+        segs = np.split(np.arange(len(grid)), np.where(np.diff(np.sign(err)) != 0)[0] + 1)
+        ext = [s[np.argmax(np.abs(err[s]))] for s in segs]
+        if len(ext) != n:
+            break
+        x = grid[ext]
+    return coef, np.abs(err).max()
+
+
+def test_cubic_is_the_remez_minimax_fit():
+    # the kernel's coefficients are the minimax cubic for 2^f on [-1/2, 1/2]
+    # in relative error, to float32 precision
+    coef, emax = _remez_relative(3, -0.5, 0.5, np.exp2)
+    c = _constants()
+    got = np.array([c["kExp2C0"], c["kExp2C1"], c["kExp2C2"], c["kExp2C3"]], np.float64)
+    assert np.allclose(got, coef, rtol=2e-7, atol=0), (got, coef)
+    assert 7.4e-5 < emax < 7.6e-5

@@ -431,13 +431,25 @@ def test_e2e_two_stage_small(sa, N, block, keep, K, W):
     _prefill_e2e(sa, inp, K, W, block=block, keep=keep)
 
 
-def test_e2e_two_stage_64k_sampled(sa):
+def test_e2e_two_stage_64k(sa):
+    # every row's kept blocks and fine top-K index set, bit for bit; attention
+    # outputs on 2100+ rows: evenly spaced ones plus block, window and
+    # selection-size edges
     c = CONFIGS["prefill_64k_two_stage"]
     inp = config_inputs("prefill_64k_two_stage")
-    N = c["N"]
-    rows = np.unique(np.r_[np.linspace(0, N - 1, 40).astype(int), 63, 64, 4159, 4160, 4223, N - 1])
-    plan, ref = _prefill_e2e(sa, inp, c["K"], c["W"], rows=rows, block=c["block"], keep=c["keep"])
+    N, blk, keep, K, W = c["N"], c["block"], c["keep"], c["K"], c["W"]
+    edges = []
+    for e in (63, 64, 65, 511, 512, 513, 2047, 2048, 2559, 2560, 2561, 4095, 4096, 4159, 4160, 4161, 4223,
+              4224, 32767, 32768, N - 65, N - 64, N - 2, N - 1):
+        edges += [e - 1, e, e + 1]
+    rows = np.unique(np.clip(np.r_[np.linspace(0, N - 1, 2048).astype(int), edges], 0, N - 1))
+    plan, ref = _prefill_e2e(sa, inp, K, W, rows=rows, block=blk, keep=keep)
+    assert len(rows) >= 2048
     assert np.array_equal(plan.blocks.cpu().numpy()[rows], ref["blocks"])
+    all_rows = np.arange(N, dtype=np.int64)
+    want_top, want_blocks = oracle.two_stage(all_rows, inp["qI"], inp["w"], inp["kI"], blk, keep, K)
+    assert np.array_equal(plan.blocks.cpu().numpy(), want_blocks)
+    assert np.array_equal(plan.topk.cpu().numpy(), want_top)
 
 
 def _decode_e2e(sa, inp, K, W, index_fp8=False):
@@ -483,6 +495,25 @@ def test_decode_edge_lengths(sa, lengths, K, W):
     for paged in (False, True):
         inp = gen_decode(B=len(lengths), lengths=lengths, Hq=64, d=128, H_I=8, D_I=64, paged=paged, seed=11)
         _decode_e2e(sa, inp, K, W)
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_decode_split_k_merge_matches_oracle(sa, paged):
+    # K + W > 16 * 1024 leaves more than 1024 keys per CTA of a 16-CTA cluster,
+    # so sa_sparse_attn_decode takes its split-K path: partial states in the
+    # caller's workspace, merged by decode_merge_kernel
+    K, W = 16000, 1000
+    lengths = [40000, 17001, 16999, 5000, 90000, 1]
+    inp = gen_decode(B=len(lengths), lengths=lengths, Hq=64, d=128, H_I=8, D_I=64, paged=paged, seed=31)
+    _, DecodePlan = _pl()
+    B = len(lengths)
+    if paged:
+        plan = DecodePlan(B, 64, 128, 8, 64, K, W, S_max=0, paged=True, max_pages=inp["page_table"].shape[1],
+                          pool_pages=inp["k"].shape[0])
+    else:
+        plan = DecodePlan(B, 64, 128, 8, 64, K, W, S_max=inp["k"].shape[1])
+    assert plan.launches() == 4   # indexer, top-K, split-K attention, merge
+    _decode_e2e(sa, inp, K, W)
 
 
 # ====================================================================== device errors

@@ -1,21 +1,23 @@
-"""sa_sparse_attn_decode_noalloc against sa_sparse_attn_decode.
+"""sa_sparse_attn_decode_noalloc against the CPU fp64 oracle and the regular decode.
 
 The allocation-free decode exists for callers that cannot allocate device
 memory (a plugin in an engine that owns all of the GPU's memory and passes
 only inputs and outputs; a loop where cudaMalloc / cudaFree must not run).
 It keeps its split partials in a fixed array inside the library instead of a
-caller workspace.  This test calls it twice in a row through the C ABI -- on
-two different problems, so the second call starts from the first call's
-leftovers in the shared array -- and checks each result against the regular
-entry point's output on the same inputs, within the attention tolerance used
-by every other GPU test.  It passes alone in a fresh process and after the
-rest of the suite.
+caller workspace, and always runs the split-K kernels and their merge kernel.
+This test calls it twice in a row through the C ABI -- on two different
+problems, so the second call starts from the first call's leftovers in the
+shared array.  Each result is checked against the oracle's decode on the same
+inputs, within the attention tolerance used by every other GPU test, and
+against the regular entry point's output.  It passes alone in a fresh process
+and after the rest of the suite.
 """
 
 import numpy as np
 import pytest
 import torch
 
+import oracle
 from workloads import gen_decode
 from tests.gpu_helpers import MAX_ABS, MEAN_ABS, dev, host_f64, status
 
@@ -49,11 +51,16 @@ def _one_call(sa, lengths, paged, K, W, seed):
     sa.sa_sparse_attn_decode_noalloc(x["q"], x["k"], x["v"], pt, mp, pp, 64, s_max, sl, plan.topk, K, W, B,
                                      Hq, d, plan.scale, out, lse, ds)
     assert status(ds) == 0
-    want, got = host_f64(plan.out), host_f64(out)
-    err = np.abs(got - want)
+    ref = oracle.decode(inp, K, W)
+    assert np.array_equal(plan.topk.cpu().numpy(), ref["topk"])
+    got = host_f64(out)
     assert np.all(np.isfinite(got))
+    err = np.abs(got - ref["out"])
     assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (err.max(), err.mean())
-    assert np.max(np.abs(host_f64(lse) - host_f64(plan.lse))) < 1e-3
+    assert np.max(np.abs(host_f64(lse) - ref["lse"])) < 1e-3
+    # and the regular entry point on the same selection
+    err2 = np.abs(got - host_f64(plan.out))
+    assert err2.max() <= MAX_ABS and err2.mean() <= MEAN_ABS, (err2.max(), err2.mean())
 
 
 def test_noalloc_decode_matches_workspace_decode_twice(sa):
