@@ -519,6 +519,8 @@ sa_status launch_prefill(const PrefillArgs &a, cudaStream_t st) {
         const sa_status s = launch_prefill_tc(a, st);
         if (s != SA_ERR_UNSUPPORTED) return s;   // else the gathered path below
     }
+    // Sparse selections: gather each query's rows onto tcgen05 tiles
+    if (prefill_gather_supported(a)) return launch_prefill_gather(a, st);
     AttnParams p = base_params(a.q, a.k, a.v, a.topk, a.K, a.W, a.Hq, a.d, a.scale, a.out, a.lse, a.dev_status);
     p.T = a.T;
     p.S = a.S;

@@ -81,6 +81,8 @@ sa_status launch_prefill(const PrefillArgs &a, cudaStream_t st);
 bool prefill_tc_supported(const PrefillArgs &a);
 size_t prefill_tc_workspace_bytes(int T, int S);
 sa_status launch_prefill_tc(const PrefillArgs &a, cudaStream_t st);
+bool prefill_gather_supported(const PrefillArgs &a);
+sa_status launch_prefill_gather(const PrefillArgs &a, cudaStream_t st);
 
 struct DecodeArgs {
     const uint16_t *q, *k, *v;

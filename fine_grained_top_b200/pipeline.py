@@ -31,21 +31,27 @@ def _ld(n: int) -> int:
 
 
 class PrefillPlan:
-    """Buffers for one sequence of N tokens (queries at positions 0..N-1).
-    Inputs: dict with q [N,Hq,d], k/v [N,d], qI [N,H_I,D_I], w [N,H_I], kI [N,D_I].
+    """Buffers for N queries of one causal sequence of S keys (default S = N):
+    the queries sit at the last N positions, S - N .. S - 1 (S > N is one
+    rank's chunk of a longer sequence, see ``shard``).
+    Inputs: dict with q [N,Hq,d], qI [N,H_I,D_I], w [N,H_I] and k/v [S,d],
+    kI [S,D_I].
     index_fp8: qI and kI are e4m3 bytes (uint8) and the indexer runs in FP8
     (single-stage selection only)."""
 
     def __init__(self, N, Hq, d, H_I, D_I, K, W, block=None, keep=None, row_blocks=1, index_fp8=False,
-                 device="cuda"):
+                 device="cuda", S=None):
         if index_fp8 and block is not None:
             raise ValueError("the FP8 indexer serves the single-stage selection")
-        self.N, self.Hq, self.d, self.H_I, self.D_I, self.K, self.W = N, Hq, d, H_I, D_I, K, W
+        S = N if S is None else int(S)
+        if S < N:
+            raise ValueError("a plan's N queries are the last N of its S keys (S >= N)")
+        self.N, self.S, self.Hq, self.d, self.H_I, self.D_I, self.K, self.W = N, S, Hq, d, H_I, D_I, K, W
         self.index = sa_indexer_scores_fp8 if index_fp8 else sa_indexer_scores
         self.block, self.keep = block, keep
         # single-stage only: score and select the queries in row_blocks blocks,
         # so that a block's scores are still in L2 when top-K reads them
-        self.row_blocks = max(1, int(row_blocks)) if block is None else 1
+        self.row_blocks = max(1, int(row_blocks)) if (block is None and S == N) else 1
         self.scale = 1.0 / math.sqrt(d)
         dev = torch.device(device)
         i32, f32 = torch.int32, torch.float32
@@ -55,17 +61,17 @@ class PrefillPlan:
         self.dev_status = torch.zeros(1, dtype=i32, device=dev)
         # The masked tensor-core attention (selected by passing its bitmap
         # workspace) runs one CTA per 256 query-head rows; below one CTA per SM
-        # the gathered kernel, one CTA per query, is faster.
+        # the gathered kernel is faster.
         groups = N * Hq // 256
         sms = torch.cuda.get_device_properties(dev).multi_processor_count if dev.type == "cuda" else 148
-        self.attn_ws_bytes = sa_prefill_workspace_bytes(N, N, K, W, Hq, d) if groups >= sms else 0
+        self.attn_ws_bytes = sa_prefill_workspace_bytes(N, S, K, W, Hq, d) if groups >= sms else 0
         self.attn_ws = (torch.empty(self.attn_ws_bytes, dtype=torch.uint8, device=dev)
                         if self.attn_ws_bytes else None)
         if block is None:
-            self.ld = _ld(N)
+            self.ld = _ld(S)
             self.scores = torch.empty((N, self.ld), dtype=f32, device=dev)
         else:
-            self.nb = N // block
+            self.nb = S // block
             self.ld_coarse = _ld(self.nb)
             self.kB = torch.empty((max(self.nb, 1), D_I), dtype=torch.bfloat16, device=dev)
             self.n_blocks = torch.empty(N, dtype=i32, device=dev)
@@ -75,13 +81,13 @@ class PrefillPlan:
             self.cand = torch.empty((N, self.ld_cand), dtype=i32, device=dev)
             self.n_cand = torch.empty(N, dtype=i32, device=dev)
             self.fine = torch.empty((N, self.ld_cand), dtype=f32, device=dev)
-            self.ws_bytes = sa_block_scores_workspace_bytes(N, N, keep)
+            self.ws_bytes = sa_block_scores_workspace_bytes(N, S, keep)
             self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=dev)
 
     def stages(self, x, stream=None):
-        N, K, ds, H, D = self.N, self.K, self.dev_status, self.H_I, self.D_I
+        N, S, K, ds, H, D = self.N, self.S, self.K, self.dev_status, self.H_I, self.D_I
         attn = ("attention", lambda: sa_sparse_attn_prefill(
-            x["q"], x["k"], x["v"], self.topk, K, self.W, N, N, self.Hq, self.d, self.scale, self.out,
+            x["q"], x["k"], x["v"], self.topk, K, self.W, N, S, self.Hq, self.d, self.scale, self.out,
             self.lse, self.attn_ws, self.attn_ws_bytes, ds, stream))
         if self.block is None and self.row_blocks > 1:
             # queries t0..t1-1 are the last t1 - t0 of a t1-key causal sequence
@@ -99,23 +105,23 @@ class PrefillPlan:
             return out + [attn]
         if self.block is None:
             return [
-                ("indexer", lambda: self.index(x["qI"], x["w"], x["kI"], None, 0, 0, 64, 1, N, N, H, D,
+                ("indexer", lambda: self.index(x["qI"], x["w"], x["kI"], None, 0, 0, 64, 1, N, S, H, D,
                                                None, self.scores, self.ld, ds, stream)),
-                ("topk", lambda: sa_topk_select(self.scores, self.ld, N, N, None, None, 0, K, self.topk, ds,
+                ("topk", lambda: sa_topk_select(self.scores, self.ld, N, S, None, None, 0, K, self.topk, ds,
                                                 stream)),
                 attn]
         blk, keep = self.block, self.keep
         return [
-            ("pool", lambda: sa_pool_index_keys(x["kI"], N, D, blk, self.kB, stream)),
-            ("block_counts", lambda: sa_coarse_block_counts(N, N, blk, self.n_blocks, stream)),
+            ("pool", lambda: sa_pool_index_keys(x["kI"], S, D, blk, self.kB, stream)),
+            ("block_counts", lambda: sa_coarse_block_counts(N, S, blk, self.n_blocks, stream)),
             ("coarse_indexer", lambda: sa_indexer_scores(x["qI"], x["w"], self.kB, None, 0, 0, 64, 1, N, self.nb,
                                                          H, D, self.n_blocks, self.coarse, self.ld_coarse, ds,
                                                          stream)),
             ("coarse_topk", lambda: sa_topk_select(self.coarse, self.ld_coarse, N, self.nb, self.n_blocks, None,
                                                    0, keep, self.blocks, ds, stream)),
-            ("expand", lambda: sa_expand_blocks(self.blocks, N, N, keep, blk, self.cand, self.ld_cand,
+            ("expand", lambda: sa_expand_blocks(self.blocks, N, S, keep, blk, self.cand, self.ld_cand,
                                                 self.n_cand, ds, stream)),
-            ("fine_indexer", lambda: sa_indexer_scores_blocks(x["qI"], x["w"], x["kI"], N, N, H, D, self.blocks,
+            ("fine_indexer", lambda: sa_indexer_scores_blocks(x["qI"], x["w"], x["kI"], N, S, H, D, self.blocks,
                                                               keep, blk, self.fine, self.ld_cand, self.workspace,
                                                               self.ws_bytes, ds, stream)),
             ("fine_topk", lambda: sa_topk_select(self.fine, self.ld_cand, N, self.ld_cand, self.n_cand,

@@ -295,6 +295,8 @@ def test_block_scores_match_oracle(sa, N, keep, H_I, D_I, rows):
     (512, 4, 64, 64, 32), (700, 16, 128, 100, 17), (300, 20, 64, 50, 0), (257, 64, 128, 64, 64),
     (90, 16, 128, 200, 8), (1, 16, 128, 4, 4), (200, 32, 64, 0, 5), (1000, 8, 128, 300, 40),
     (130, 32, 64, 64, 0), (2048, 16, 128, 256, 64), (1500, 4, 128, 64, 1),
+    (3000, 32, 128, 2048, 512), (600, 16, 128, 0, 33), (5000, 16, 128, 2048, 512), (777, 12, 128, 129, 127),
+    (400, 16, 128, 2500, 16),
 ])
 def test_prefill_attention_given_oracle_topk(sa, N, Hq, d, K, W, use_ws):
     # use_ws=False: the gathered kernel; True: the masked tensor-core kernel
@@ -316,6 +318,29 @@ def test_prefill_attention_given_oracle_topk(sa, N, Hq, d, K, W, use_ws):
                               ws, nb, ds)
     ptr, idx = oracle.selection(top, W, np.arange(N))
     o, l = oracle.sparse_attention(inp["q"], inp["k"], inp["v"], ptr, idx, 1 / math.sqrt(d))
+    assert status(ds) == 0
+    assert_close_attention(host_f64(out), o, "out")
+    assert np.max(np.abs(host_f64(lse) - l)) < 1e-3
+
+
+def test_prefill_gathered_chunk_two_stage_shape(sa):
+    # the last 600 queries of a 70000-token sequence at the two-stage
+    # workload's attention shape (16 heads, d=128, K=2048, W=512): more queries
+    # than SMs, so the persistent CTAs take several queries each
+    S, T, Hq, d, K, W = 70000, 600, 16, 128, 2048, 512
+    inp = gen_prefill(N=S, Hq=Hq, d=d, H_I=2, D_I=32, seed=8)
+    pos = np.arange(S - T, S)
+    sc = oracle.indexer(inp["qI"][S - T:], inp["w"][S - T:], inp["kI"], pos)
+    top = oracle.topk(sc, pos + 1, K)
+    q = dev(np.ascontiguousarray(inp["q"][S - T:]))
+    t = _to_dev(inp, ("k", "v"))
+    out = torch.empty((T, Hq, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((T, Hq), dtype=torch.float32, device="cuda")
+    ds = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sa.sa_sparse_attn_prefill(q, t["k"], t["v"], dev(top.astype(np.int32)), K, W, T, S, Hq, d, 1 / math.sqrt(d),
+                              out, lse, None, 0, ds)
+    ptr, idx = oracle.selection(top, W, pos)
+    o, l = oracle.sparse_attention(inp["q"][S - T:], inp["k"], inp["v"], ptr, idx, 1 / math.sqrt(d))
     assert status(ds) == 0
     assert_close_attention(host_f64(out), o, "out")
     assert np.max(np.abs(host_f64(lse) - l)) < 1e-3
@@ -365,6 +390,23 @@ def _prefill_e2e(sa, inp, K, W, rows=None, block=None, keep=None, index_fp8=Fals
     assert_close_attention(host_f64(plan.out)[r], ref["out"], "out")
     assert np.max(np.abs(host_f64(plan.lse)[r] - ref["lse"])) < 1e-3
     return plan, ref
+
+
+@pytest.mark.parametrize("T,S,block,keep,K,W", [(300, 5000, None, None, 512, 64), (700, 4096, 64, 16, 512, 64)])
+def test_plan_for_the_last_rows_of_a_longer_sequence(sa, T, S, block, keep, K, W):
+    # one rank's share of a query-row partition: T queries at positions
+    # S - T .. S - 1 over S keys, against the oracle on those rows
+    PrefillPlan, _ = _pl()
+    inp = gen_prefill(N=S, Hq=16, d=128, H_I=4, D_I=64, seed=T + S)
+    plan = PrefillPlan(T, 16, 128, 4, 64, K, W, block=block, keep=keep, S=S)
+    q, qI, w = (dev(np.ascontiguousarray(inp[n][S - T:])) for n in ("q", "qI", "w"))
+    t = _to_dev(inp, ("k", "v", "kI"))
+    plan.run(q, t["k"], t["v"], qI, w, t["kI"])
+    assert status(plan.dev_status) == 0
+    ref = oracle.prefill(inp, K, W, rows=np.arange(S - T, S), block=block, keep=keep)
+    assert np.array_equal(plan.topk.cpu().numpy(), ref["topk"])
+    assert_close_attention(host_f64(plan.out), ref["out"], "out")
+    assert np.max(np.abs(host_f64(plan.lse) - ref["lse"])) < 1e-3
 
 
 def test_host_pipeline_matches_direct_runs(sa):
