@@ -4,8 +4,8 @@
                     [--index-fp8]
 
 A step is one pass of the whole path -- indexer -> top-K -> sparse attention
-(for the two-stage workload: pool, coarse scores, coarse top-k, expand, fine
-scores, top-K, attention) -- over one synthetic batch.  The default workload is
+(for the two-stage workload: pool, block counts, coarse scores, coarse top-k,
+fine scores, top-K over the kept blocks, attention) -- over one synthetic batch.  The default workload is
 the largest one that fits one GPU: the two-stage 65536-token causal prefill (16
 query heads, d=128, one KV head, indexer 4 x 64, 64-token blocks, 64 kept
 blocks, top-K 2048, window 512).  Each rank runs its own independent sequence (weak scaling, no
@@ -60,7 +60,7 @@ def load_peaks():
 # --------------------------------------------------------------------------- ncu traffic
 STAGE_SOURCE = {"indexer": "indexer.cu", "coarse_indexer": "indexer.cu", "topk": "topk.cu",
                 "coarse_topk": "topk.cu", "fine_topk": "topk.cu", "attention": "attention.cu+attention_tc.cu",
-                "fine_indexer": "block_scores.cu", "expand": "two_stage.cu", "pool": "two_stage.cu",
+                "fine_indexer": "block_scores.cu", "pool": "two_stage.cu",
                 "block_counts": "two_stage.cu"}
 
 
@@ -264,17 +264,17 @@ def stage_work(case):
             blk, keep = cfg["block"], cfg["keep"]
             nb = N // blk
             cpairs = int(sum(t // blk for t in range(N)))
-            fpairs = int(plan.n_cand.cpu().numpy().astype(np.int64).sum())
+            t = np.arange(N, dtype=np.int64)   # candidates: min(keep, t // blk) kept blocks + own block up to t
+            fpairs = int((np.minimum(keep, t // blk) * blk + t % blk + 1).sum())
             work.update(coarse_pairs=cpairs, fine_pairs=fpairs)
             st["pool"] = dict(bytes=N * D * 2 + nb * D * 2, flops=float(N * D), bound="hbm")
             st["block_counts"] = dict(bytes=4 * N, flops=0.0, bound="hbm")
             st["coarse_indexer"] = dict(bytes=qI_b + w_b + nb * D * 2 + 4 * N + 4 * cpairs,
                                         flops=2.0 * cpairs * H * D, bound="hbm")
             st["coarse_topk"] = dict(bytes=4 * cpairs + 4 * N + 4 * N * keep, flops=0.0, bound="hbm")
-            st["expand"] = dict(bytes=4 * N * keep + 4 * fpairs + 4 * N, flops=0.0, bound="hbm")
             st["fine_indexer"] = dict(bytes=qI_b + w_b + N * D * 2 + 4 * N + 8 * fpairs,
                                       flops=2.0 * fpairs * H * D, bound="hbm")
-            st["fine_topk"] = dict(bytes=8 * fpairs + 4 * N + idx_b, flops=0.0, bound="hbm")
+            st["fine_topk"] = dict(bytes=4 * fpairs + 4 * N * keep + idx_b, flops=0.0, bound="hbm")
     work["stages"] = st
     return work
 

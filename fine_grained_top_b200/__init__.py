@@ -40,6 +40,7 @@ SIGNATURES = {
     "sa_indexer_scores_blocks": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp, _i32, _i32, _vp, _i64,
                                         _vp, _sz, _vp, _vp]),
     "sa_topk_select": (_i32, [_vp, _i64, _i32, _i32, _vp, _vp, _i64, _i32, _vp, _vp, _vp]),
+    "sa_topk_select_blocks": (_i32, [_vp, _i64, _i32, _i32, _vp, _i32, _i32, _i32, _vp, _vp, _vp]),
     "sa_prefill_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
     "sa_sparse_attn_prefill": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp,
                                       _vp, _vp, _sz, _vp, _vp]),
@@ -138,6 +139,11 @@ def sa_topk_select(scores, ld_scores, rows, row_len, n_valid, cand_map, ld_cand,
                    dev_status=None, stream=None):
     _check(_lib.sa_topk_select(_ptr(scores), ld_scores, rows, row_len, _ptr(n_valid), _ptr(cand_map),
                                ld_cand, K, _ptr(topk), _ptr(dev_status), _stream(stream)), "sa_topk_select")
+
+
+def sa_topk_select_blocks(scores, ld_scores, T, S, blocks, keep, block, K, topk, dev_status=None, stream=None):
+    _check(_lib.sa_topk_select_blocks(_ptr(scores), ld_scores, T, S, _ptr(blocks), keep, block, K, _ptr(topk),
+                                      _ptr(dev_status), _stream(stream)), "sa_topk_select_blocks")
 
 
 def sa_prefill_workspace_bytes(T, S, K, W, Hq, d) -> int:

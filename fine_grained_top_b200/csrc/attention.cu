@@ -108,14 +108,38 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(AttnParams P)
     {
         int cnt = 0;
         bool bad_idx = false, bad_ord = false;
-        for (int i = tid; i < P.K; i += kAttnThreads) {
-            const int e = trow[i];
+        auto check = [&](int i, int e, int prev) {
             if (e >= 0 && e <= p - P.W) ++cnt;
             if (e > p) bad_idx = true;
-            if (e >= 0 && i > 0) {
-                const int prev = trow[i - 1];
-                if (!(prev >= 0 && prev < e)) bad_ord = true;
+            if (e >= 0 && i > 0 && !(prev >= 0 && prev < e)) bad_ord = true;
+        };
+        if ((P.K & 3) == 0 && (reinterpret_cast<uintptr_t>(P.topk) & 15u) == 0) {
+            // 16-byte loads, four per thread in flight at once (one L2 round trip
+            // for a 2048-entry row instead of one per entry)
+            const int nv = P.K >> 2;
+            for (int base = 0; base < nv; base += 4 * kAttnThreads) {
+                int4 v[4];
+                int pv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int idx = base + u * kAttnThreads + tid;
+                    v[u] = idx < nv ? __ldg(reinterpret_cast<const int4 *>(trow) + idx) : make_int4(-1, -1, -1, -1);
+                    pv[u] = (idx < nv && idx > 0) ? __ldg(trow + 4 * idx - 1) : -1;
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int idx = base + u * kAttnThreads + tid;
+                    if (idx < nv) {
+                        const int i = 4 * idx;
+                        check(i, v[u].x, pv[u]);
+                        check(i + 1, v[u].y, v[u].x);
+                        check(i + 2, v[u].z, v[u].y);
+                        check(i + 3, v[u].w, v[u].z);
+                    }
+                }
             }
+        } else {
+            for (int i = tid; i < P.K; i += kAttnThreads) check(i, trow[i], i > 0 ? trow[i - 1] : -1);
         }
         if (bad_idx) report(P.dev_status, SA_DEV_INDEX);
         if (bad_ord) report(P.dev_status, SA_DEV_ORDER);
@@ -142,22 +166,40 @@ __global__ void __launch_bounds__(kAttnThreads) sparse_attn_kernel(AttnParams P)
     // ---- this CTA's key list as cache rows, built once in shared memory
     // (entry i < n_top is a top-K position, the rest is the window)
     const int n_list = hi > lo ? hi - lo : 0;
-    for (int j = tid; j < nchunks * kChunk; j += kAttnThreads) {
-        const int i = lo + j;
-        int32_t row = -1;
-        if (i < hi) {
-            const int s = (i < n_top) ? trow[i] : w0 + (i - n_top);
-            if (s < 0 || s > p) {
-                report(P.dev_status, SA_DEV_INDEX);
-            } else if (DECODE && P.page_table) {
-                const int pid = P.page_table[(int64_t)b * P.max_pages + (s >> 6)];
-                if (pid < 0 || pid >= P.pool_pages) report(P.dev_status, SA_DEV_INDEX);
-                else row = pid * 64 + (s & 63);
-            } else {
-                row = DECODE ? b * P.S_max + s : s;
-            }
+    // (two entries per thread at a time, their loads -- and then their page
+    // lookups -- in flight together)
+    for (int j0 = 0; j0 < nchunks * kChunk; j0 += 2 * kAttnThreads) {
+        int sv[2];
+        bool in[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int j = j0 + u * kAttnThreads + tid, i = lo + j;
+            in[u] = j < nchunks * kChunk && i < hi;
+            sv[u] = in[u] ? ((i < n_top) ? __ldg(trow + i) : w0 + (i - n_top)) : -1;
         }
-        s_rows[j] = row;
+        int pid[2] = {0, 0};
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+            if (DECODE && P.page_table && in[u] && sv[u] >= 0 && sv[u] <= p)
+                pid[u] = __ldg(P.page_table + (int64_t)b * P.max_pages + (sv[u] >> 6));
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int j = j0 + u * kAttnThreads + tid;
+            if (j >= nchunks * kChunk) continue;
+            int32_t row = -1;
+            if (in[u]) {
+                const int s = sv[u];
+                if (s < 0 || s > p) {
+                    report(P.dev_status, SA_DEV_INDEX);
+                } else if (DECODE && P.page_table) {
+                    if (pid[u] < 0 || pid[u] >= P.pool_pages) report(P.dev_status, SA_DEV_INDEX);
+                    else row = pid[u] * 64 + (s & 63);
+                } else {
+                    row = DECODE ? b * P.S_max + s : s;
+                }
+            }
+            s_rows[j] = row;
+        }
     }
     (void)n_list;
     __syncthreads();

@@ -24,17 +24,21 @@
 //
 // Persistent CTAs (one per SM) take queries T-1-c, T-1-c-G, ... (heavy first)
 // and stream their tiles through a pipeline of warp roles:
-//   warp 9      index builder: copies the query's top-K row to shared memory,
+//   warp 13     index builder: copies the query's top-K row to shared memory,
 //               validates it (SA_DEV_INDEX / SA_DEV_ORDER), finds the prefix
-//               of entries <= p - W and writes the cache rows of each
-//               128-key tile (top-K prefix, then the window) into a ring
-//   warps 0..3  gather: 16-byte cp.async of every selected K and V row into a
-//               128B-swizzled tile (rows past the selection are zero-filled),
-//               the query's Q rows with its first tile; completion is tracked
-//               by the stage's mbarrier (cp.async.mbarrier.arrive.noinc)
-//   warp 8      MMA issuer (one thread) and TMEM owner
-//   warps 4..7  softmax of tile g (TMEM lane quadrant = warp % 4), then the
-//               epilogue of each query: O^T / l -> out (bf16), lse
+//               of entries <= p - W and writes the byte offsets of each
+//               128-key tile's cache rows (top-K prefix, then the window;
+//               0xffffffff past the selection) into a ring
+//   warps 0..3  gather: 16-byte cp.async of every selected K row (warps 0-1,
+//               with the query's Q rows at its first tile) and V row (warps
+//               2-3) into 128B-swizzled tiles of separate K and V rings (rows
+//               past the selection are zero-filled); completion is tracked by
+//               the slot's mbarrier (cp.async.mbarrier.arrive.noinc)
+//   warp 12     S issuer (one thread) and TMEM owner
+//   warp 14     P V issuer (one thread)
+//   warps 4..11 softmax of tile g in two groups of four warps, each group
+//               owning half of the heads (TMEM lane quadrant = warp % 4), then
+//               the epilogue of each query: O^T / l -> out (bf16), lse
 // Every wait is bounded (SA_DEV_TIMEOUT), and the softmax warps take each
 // wait's outcome together (bar.red) before any barrier among them.
 #include <math_constants.h>
@@ -47,9 +51,15 @@ namespace sa {
 namespace {
 
 constexpr int kGTile = 128;                  // keys per tile (MMA M)
-constexpr int kGThreads = 10 * 32;
-constexpr int kGRing = 8;                    // row-index tiles the builder runs ahead
+constexpr int kGThreads = 15 * 32;
+// warp roles: 0..3 gather, 4..11 softmax (two groups of four, each owning half
+// of the heads), then the S issuer (TMEM owner), the index builder, the P V issuer
+constexpr int kWarpS = 12, kWarpBuild = 13, kWarpPV = 14;
+constexpr int kGRing = 6;                    // row-index tiles the builder runs ahead
 constexpr int kGMaxK = 2048;                 // top-K entries held in shared memory per query
+constexpr int kGInfo = 8;                    // tile records in flight (K issue .. P V done)
+constexpr int kGSB = 4;                      // S^T buffers in TMEM
+constexpr int kGPB = 3;                      // P^T buffers in shared memory
 constexpr size_t kGSmemLimit = 232448;
 
 struct GParams {
@@ -78,31 +88,38 @@ struct TileHdr {
 template <int HQP>
 struct GCfg {
     static constexpr int kD = 128;
-    static constexpr int kHalf = kGTile * 128;                 // one 64-column SW128 half of a K/V tile
+    static constexpr int kHalf = kGTile * 128;                 // one 64-column SW128 half of a K or V tile
     static constexpr int kKV = 2 * kHalf;                      // 128 keys x 256 bytes
-    static constexpr int kStage = 2 * kKV;                     // K + V
     static constexpr int kQHalf = HQP * 128;
     static constexpr int kQ = 2 * kQHalf;                      // HQP rows x 256 bytes
     static constexpr int kP = 2 * kQHalf;                      // HQP heads x 128 keys bf16
+    // everything but the K and V rings (barriers counted for 3 + 3 ring slots)
     static constexpr size_t fixed() {
-        return 1024 + 2 * (size_t)kQ + 2 * (size_t)kP + kGRing * (kGTile * 4 + sizeof(TileHdr)) + kGMaxK * 4 +
-               2 * 4 * HQP * 4 + 1024;
+        return 1024 + 2 * (size_t)kQ + kGPB * (size_t)kP + kGRing * (kGTile * 4 + sizeof(TileHdr)) +
+               kGInfo * sizeof(TileHdr) + kGMaxK * 4 + 4 * 4 * HQP * 4 + 8 +
+               (4 * 3 + 2 * kGRing + 2 * kGInfo + 2 * kGSB + kGPB + 2 * 4) * 8 + 16;
     }
-    static constexpr int kNS = fixed() + 3 * (size_t)kStage <= kGSmemLimit ? 3 : 2;
-    static constexpr int kOffKV = 0;                                   // [kNS] stages
-    static constexpr int kOffQ = kOffKV + kNS * kStage;                // [2]
-    static constexpr int kOffP = kOffQ + 2 * kQ;                       // [2]
-    static constexpr int kOffRows = kOffP + 2 * kP;                    // [kGRing][128] int32
+    // K and V tiles live in separate rings: K(g) is released when S(g) is
+    // done, V(g) when P V(g) is done
+    static constexpr int kNK = fixed() + 6 * (size_t)kKV <= kGSmemLimit ? 3 : 2;
+    static constexpr int kNV = kNK;
+    static constexpr int kOffK = 0;                                    // [kNK] K tiles
+    static constexpr int kOffV = kOffK + kNK * kKV;                    // [kNV] V tiles
+    static constexpr int kOffQ = kOffV + kNV * kKV;                    // [2]
+    static constexpr int kOffP = kOffQ + 2 * kQ;                       // [kGPB]
+    static constexpr int kOffRows = kOffP + kGPB * kP;                 // [kGRing][128] row byte offsets
     static constexpr int kOffRowHdr = kOffRows + kGRing * kGTile * 4;  // [kGRing] TileHdr
-    static constexpr int kOffTi = kOffRowHdr + kGRing * (int)sizeof(TileHdr);   // [kNS] TileHdr
-    static constexpr int kOffList = kOffTi + kNS * (int)sizeof(TileHdr);       // [kGMaxK] int32
-    static constexpr int kOffRed = kOffList + kGMaxK * 4;              // [2][4][HQP] f32
-    static constexpr int kOffBar = (kOffRed + 2 * 4 * HQP * 4 + 7) & ~7;
-    // kv_full/kv_empty [kNS], row_full/row_empty [kGRing], six pairs (s_full,
-    // p_full, p_empty, o_full, o_empty, q_empty) and drain
-    static constexpr int kNumBar = 2 * kNS + 2 * kGRing + 2 * 6 + 1;
+    static constexpr int kOffTi = kOffRowHdr + kGRing * (int)sizeof(TileHdr);   // [kGInfo] TileHdr
+    static constexpr int kOffList = kOffTi + kGInfo * (int)sizeof(TileHdr);    // [kGMaxK] int32
+    static constexpr int kOffRed = kOffList + kGMaxK * 4;              // [4][HQP] max, [4][HQP] sums, [2][2][HQP] m, l
+    static constexpr int kOffBar = (kOffRed + 4 * 4 * HQP * 4 + 7) & ~7;
+    // k_full/k_empty [kNK], v_full/v_empty [kNV], row_full/row_empty [kGRing],
+    // ti_full / ti_empty [kGInfo], s_full / p_full [kGSB], p_empty [kGPB], four
+    // pairs (o_full, o_empty, q_empty, drain)
+    static constexpr int kNumBar = 2 * kNK + 2 * kNV + 2 * kGRing + 2 * kGInfo + 2 * kGSB + kGPB + 2 * 4;
     static constexpr size_t kSmem = 1024 + (size_t)kOffBar + kNumBar * 8 + 16;
-    static constexpr uint32_t kTmemCols = 4 * HQP <= 32 ? 32 : (4 * HQP <= 64 ? 64 : (4 * HQP <= 128 ? 128 : 256));
+    static constexpr int kCols = (kGSB + 2) * HQP;              // S^T buffers, then O^T [2]
+    static constexpr uint32_t kTmemCols = kCols <= 32 ? 32 : (kCols <= 64 ? 64 : (kCols <= 128 ? 128 : 256));
 };
 
 // ------------------------------------------------------------------ PTX helpers
@@ -116,13 +133,33 @@ __device__ __forceinline__ void cp_async16_zfill(void *smem_dst, const void *gsr
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
+// Bounded wait for a phase that parks the thread in mbarrier.try_wait (with a
+// suspend-time hint of 20 us) instead of polling: eleven warps wait on
+// barriers most of the time here, and polling waits flood the issue slots
+// and the pipe that executes the barrier tests.  Gives up like mbar_wait.
+__device__ __forceinline__ bool try_wait_parked(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool gwait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    if (try_wait_parked(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    while (true) {
+        if (try_wait_parked(bar, parity)) return true;
+        if (*abort) return false;
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            *abort = 1;
+            return false;
+        }
+    }
+}
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ float warp_max(float v) {
-    float r;
-    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
-    return r;
-}
 // Barrier `id` over `n` threads that also returns the OR / AND of a predicate.
 __device__ __forceinline__ bool bar_or(int id, int n, bool p) {
     uint32_t r;
@@ -148,13 +185,10 @@ __device__ __forceinline__ float ex2f(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-            taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+                 "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
 }
 __device__ __forceinline__ void tmem_st_wait_all() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void mma_acc(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
@@ -182,7 +216,7 @@ __device__ __forceinline__ uint32_t sw_off(int r, int ch, int half) {
 template <int HQP>
 __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P) {
     using C = GCfg<HQP>;
-    constexpr int NS = C::kNS;
+    constexpr int NK = C::kNK, NV = C::kNV;
     constexpr int D = C::kD;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -190,13 +224,15 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
     TileHdr *rhdr = reinterpret_cast<TileHdr *>(sm + C::kOffRowHdr);
     TileHdr *ti = reinterpret_cast<TileHdr *>(sm + C::kOffTi);
     int32_t *list = reinterpret_cast<int32_t *>(sm + C::kOffList);
-    float *redmax = reinterpret_cast<float *>(sm + C::kOffRed);     // [4][HQP]
-    float *redsum = redmax + 4 * HQP;                                // [4][HQP]
+    float *redmax = reinterpret_cast<float *>(sm + C::kOffRed);     // [2 groups][4 warps][HQP / 2]
+    float *redsum = redmax + 4 * HQP;                                // [2 groups][4 warps][HQP / 2]
+    float *epi_m = redsum + 4 * HQP, *epi_l = epi_m + 2 * HQP;       // [2 queries][HQP]
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + C::kOffBar);
-    uint64_t *kv_full = bar, *kv_empty = bar + NS;
-    uint64_t *row_full = bar + 2 * NS, *row_empty = row_full + kGRing;
-    uint64_t *s_full = row_empty + kGRing, *p_full = s_full + 2, *p_empty = p_full + 2;
-    uint64_t *o_full = p_empty + 2, *o_empty = o_full + 2;
+    uint64_t *k_full = bar, *k_empty = k_full + NK, *v_full = k_empty + NK, *v_empty = v_full + NV;
+    uint64_t *row_full = v_empty + NV, *row_empty = row_full + kGRing, *ti_full = row_empty + kGRing;
+    uint64_t *ti_empty = ti_full + kGInfo;
+    uint64_t *s_full = ti_empty + kGInfo, *p_full = s_full + kGSB, *p_empty = p_full + kGSB;
+    uint64_t *o_full = p_empty + kGPB, *o_empty = o_full + 2;
     uint64_t *q_empty = o_empty + 2, *drain = q_empty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + C::kNumBar);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -206,23 +242,34 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
     const int n_mine = P.T > (int)blockIdx.x ? (P.T - 1 - (int)blockIdx.x) / G + 1 : 0;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NS; ++i) {
-            mbar_init(&kv_full[i], 128 + 1);   // 128 cp.async arrivals + the header writer
-            mbar_init(&kv_empty[i], 1);
+        for (int i = 0; i < NK; ++i) {
+            mbar_init(&k_full[i], 64 + 1);     // 64 cp.async arrivals + the record writer
+            mbar_init(&k_empty[i], 1);
+        }
+        for (int i = 0; i < NV; ++i) {
+            mbar_init(&v_full[i], 64);         // 64 cp.async arrivals
+            mbar_init(&v_empty[i], 1);
+        }
+        for (int i = 0; i < kGInfo; ++i) {
+            mbar_init(&ti_full[i], 1);
+            mbar_init(&ti_empty[i], 1);   // the P V issuer has read the record
         }
         for (int i = 0; i < kGRing; ++i) {
             mbar_init(&row_full[i], 1);
             mbar_init(&row_empty[i], 4);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kGSB; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&p_full[i], 4);
-            mbar_init(&p_empty[i], 1);
+            mbar_init(&p_full[i], 8);
+        }
+        for (int i = 0; i < kGPB; ++i) mbar_init(&p_empty[i], 1);
+        for (int i = 0; i < 2; ++i) {
             mbar_init(&o_full[i], 1);
-            mbar_init(&o_empty[i], 4);
+            mbar_init(&o_empty[i], 8);
             mbar_init(&q_empty[i], 1);
         }
-        mbar_init(drain, 1);
+        mbar_init(&drain[0], 1);
+        mbar_init(&drain[1], 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -230,7 +277,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
     for (int i = threadIdx.x; i < 2 * C::kQ / 16; i += kGThreads)
         reinterpret_cast<uint4 *>(sm + C::kOffQ)[i] = make_uint4(0, 0, 0, 0);
     fence_async_smem();
-    if (warp == 8) {
+    if (warp == kWarpS) {
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
@@ -239,7 +286,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;   // S[0], S[1] at columns 0, HQP; O[0], O[1] at 2 HQP, 3 HQP
 
-    if (warp == 9) {
+    if (warp == kWarpBuild) {
         // ------------------------------------------------------------ index builder
         int g = 0;
         bool ok = true;
@@ -305,14 +352,15 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
             const int n_tiles = (n_keys + kGTile - 1) / kGTile;
             for (int i = 0; i < n_tiles && ok; ++i, ++g) {
                 const int slot = g % kGRing;
-                ok = __all_sync(0xffffffffu, mbar_wait(&row_empty[slot], ((uint32_t)(g / kGRing) & 1u) ^ 1u,
+                ok = __all_sync(0xffffffffu, gwait(&row_empty[slot], ((uint32_t)(g / kGRing) & 1u) ^ 1u,
                                                        abort_flag));
                 if (!ok) break;
                 int32_t *rr = rows + slot * kGTile;
 #pragma unroll
                 for (int u = 0; u < kGTile / 32; ++u) {
                     const int kk = i * kGTile + u * 32 + lane;
-                    rr[u * 32 + lane] = kk < n_top ? list[kk] : (kk < n_keys ? w0 + (kk - n_top) : -1);
+                    const int row = kk < n_top ? list[kk] : (kk < n_keys ? w0 + (kk - n_top) : -1);
+                    rr[u * 32 + lane] = row >= 0 ? (int32_t)((uint32_t)row * (uint32_t)(D * 2)) : -1;
                 }
                 if (lane == 0) {
                     TileHdr h;
@@ -328,7 +376,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
         }
         if (ok) {   // end marker
             const int slot = g % kGRing;
-            ok = __all_sync(0xffffffffu, mbar_wait(&row_empty[slot], ((uint32_t)(g / kGRing) & 1u) ^ 1u, abort_flag));
+            ok = __all_sync(0xffffffffu, gwait(&row_empty[slot], ((uint32_t)(g / kGRing) & 1u) ^ 1u, abort_flag));
             if (ok && lane == 0) {
                 TileHdr h = {};
                 h.end = 1;
@@ -339,188 +387,249 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
         __syncwarp();
     } else if (warp < 4) {
         // ------------------------------------------------------------ gather
-        const int tid = threadIdx.x;   // 0..127
+        // Warps 0-1 copy K rows (and a query's Q rows with its first tile),
+        // warps 2-3 copy V rows, each pair on its own ring: K(g) waits only for
+        // S(g - kNK) to finish with its slot, V(g) only for P V(g - kNV).
+        const bool kside = warp < 2;
+        const int pw = warp & 1, t64 = pw * 32 + lane;   // thread within the side
         const int sub = lane >> 4, ch = lane & 15;
+        const uint8_t *base = reinterpret_cast<const uint8_t *>(kside ? P.k : P.v) + ch * 16;
         bool ok = true;
         for (int g = 0; ok; ++g) {
-            const int slot = g % kGRing, s = g % NS;
-            ok = mbar_wait(&row_full[slot], (uint32_t)(g / kGRing) & 1u, abort_flag) &&
-                 mbar_wait(&kv_empty[s], ((uint32_t)(g / NS) & 1u) ^ 1u, abort_flag);
+            const int slot = g % kGRing;
+            ok = gwait(&row_full[slot], (uint32_t)(g / kGRing) & 1u, abort_flag);
             if (!ok) break;
             const TileHdr h = rhdr[slot];
-            if (h.end) {
-                if (tid == 0) ti[s] = h;
-                cp_async_arrive_noinc(&kv_full[s]);
-                if (tid == 0) mbar_arrive(&kv_full[s]);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&row_empty[slot]);
-                break;
-            }
-            uint8_t *sk = sm + C::kOffKV + s * C::kStage, *sv = sk + C::kKV;
-            if (h.i == 0) {
-                // the query's Q rows into buffer j % 2, once the S products of
-                // query j - 2 are done with it
-                if (h.j >= 2) {
-                    ok = mbar_wait(&q_empty[h.j & 1], ((uint32_t)(h.j >> 1) & 1u) ^ 1u, abort_flag);
+            if (!h.end) {
+                uint8_t *dst;
+                if (kside) {
+                    ok = gwait(&k_empty[g % NK], ((uint32_t)(g / NK) & 1u) ^ 1u, abort_flag);
+                    if (ok && h.i == 0 && h.j >= 2)   // Q buffer j % 2, once the S products of query j - 2 are done
+                        ok = gwait(&q_empty[h.j & 1], ((uint32_t)(h.j >> 1) & 1u) ^ 1u, abort_flag);
                     if (!ok) break;
+                    if (h.i == 0) {
+                        uint8_t *sq = sm + C::kOffQ + (h.j & 1) * C::kQ;
+                        const uint16_t *qrow = P.q + (int64_t)h.t * P.Hq * D;
+                        for (int idx = t64; idx < P.Hq * 16; idx += 64) {
+                            const int r = idx >> 4, c = idx & 15;
+                            cp_async16(sq + sw_off(r, c, C::kQHalf), qrow + (int64_t)r * D + c * 8);
+                        }
+                    }
+                    dst = sm + C::kOffK + (g % NK) * C::kKV;
+                } else {
+                    ok = gwait(&v_empty[g % NV], ((uint32_t)(g / NV) & 1u) ^ 1u, abort_flag);
+                    if (!ok) break;
+                    dst = sm + C::kOffV + (g % NV) * C::kKV;
                 }
-                uint8_t *sq = sm + C::kOffQ + (h.j & 1) * C::kQ;
-                const uint16_t *qrow = P.q + (int64_t)h.t * P.Hq * D;
-                for (int idx = tid; idx < P.Hq * 16; idx += 128) {
-                    const int r = idx >> 4, c = idx & 15;
-                    cp_async16(sq + sw_off(r, c, C::kQHalf), qrow + (int64_t)r * D + c * 8);
+                // this warp's 64 keys: byte offsets first, then the copies (a key
+                // past the selection is zero-filled: source size 0)
+                const uint32_t *rr = reinterpret_cast<const uint32_t *>(rows + slot * kGTile) + pw * 64;
+                uint32_t ro[32];
+#pragma unroll
+                for (int it = 0; it < 32; ++it) ro[it] = rr[2 * it + sub];
+#pragma unroll
+                for (int it = 0; it < 32; ++it) {
+                    const int key = pw * 64 + 2 * it + sub;
+                    const bool valid = ro[it] != 0xffffffffu;
+                    cp_async16_zfill(dst + sw_off(key, ch, C::kHalf), base + (valid ? ro[it] : 0u), valid ? 16u : 0u);
                 }
             }
-            const int32_t *rr = rows + slot * kGTile;
-#pragma unroll 4
-            for (int it = 0; it < 16; ++it) {
-                const int key = warp * 32 + 2 * it + sub;
-                const int row = rr[key];
-                const uint32_t off = sw_off(key, ch, C::kHalf);
-                if (key < h.nvalid && row >= 0) {
-                    cp_async16(sk + off, P.k + (int64_t)row * D + ch * 8);
-                    cp_async16(sv + off, P.v + (int64_t)row * D + ch * 8);
-                } else {
-                    cp_async16_zfill(sk + off, P.k, 0u);
-                    cp_async16_zfill(sv + off, P.v, 0u);
+            if (kside) {
+                // the tile's record, once the P V issuer has read the record of
+                // tile g - kGInfo from the slot; then K(g) complete
+                if (t64 == 0) {
+                    if (g >= kGInfo)
+                        ok = gwait(&ti_empty[g % kGInfo], ((uint32_t)(g / kGInfo) & 1u) ^ 1u, abort_flag);
+                    if (ok) {
+                        ti[g % kGInfo] = h;
+                        mbar_arrive(&ti_full[g % kGInfo]);
+                    }
                 }
+                ok = __shfl_sync(0xffffffffu, ok, 0);   // lane 0 of warp 0 waited: its warp follows its result
+                if (!ok) break;
+                if (!h.end) {
+                    cp_async_arrive_noinc(&k_full[g % NK]);
+                    if (t64 == 0) mbar_arrive(&k_full[g % NK]);
+                }
+            } else if (!h.end) {
+                cp_async_arrive_noinc(&v_full[g % NV]);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&row_empty[slot]);
-            if (tid == 0) ti[s] = h;
-            cp_async_arrive_noinc(&kv_full[s]);
-            if (tid == 0) mbar_arrive(&kv_full[s]);
+            if (h.end) break;
         }
         cp_async_wait_all();
-    } else if (warp == 8) {
-        // ------------------------------------------------------------ MMA issuer
+    } else if (warp == kWarpS) {
+        // ------------------------------------------------------------ S issuer
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, HQP);
-            constexpr uint32_t idesc_o = idesc_bf16_f32(128, HQP) | (1u << 15);   // A (V^T) MN-major
-            const uint64_t kv_d = smem_desc(smem_u32(sm + C::kOffKV), 1024, 2);
-            const uint64_t v_d = desc_mn128(smem_u32(sm + C::kOffKV + C::kKV), C::kHalf);
+            const uint64_t k_d = smem_desc(smem_u32(sm + C::kOffK), 1024, 2);
             const uint64_t q_d = smem_desc(smem_u32(sm + C::kOffQ), 1024, 2);
-            const uint64_t p_d = smem_desc(smem_u32(sm + C::kOffP), 1024, 2);
-            int gs = 0, gp = 0, g_end = 0x7fffffff;
-            int info_j[2] = {0, 0}, info_first[2] = {0, 0}, info_last[2] = {0, 0};
-            bool ok = true;
-            unsigned long long t0 = globaltimer();
-            while (gp < g_end && ok) {
-                bool progressed = false;
-                // S(gs) = K(gs) Q^T once the tile landed and S buffer gs % 2 is free
-                if (gs < g_end && gs < gp + 2 && mbar_try_wait(&kv_full[gs % NS], (uint32_t)(gs / NS) & 1u)) {
-                    const TileHdr h = ti[gs % NS];
-                    if (h.end) {
-                        g_end = gs;
-                    } else {
-                        tc_fence_after();
-                        const uint32_t dt = tmem + (uint32_t)((gs & 1) * HQP);
-                        const uint64_t kd = kv_d + (uint64_t)(((gs % NS) * C::kStage) >> 4);
-                        const uint64_t qd = q_d + (uint64_t)(((h.j & 1) * C::kQ) >> 4);
+            for (int g = 0;; ++g) {
+                // the tile's record and K(g) (the record is written before K's
+                // completion), and S buffer g % 2 read by the softmax of tile g - 2
+                bool ok = gwait(&ti_full[g % kGInfo], (uint32_t)(g / kGInfo) & 1u, abort_flag);
+                if (!ok) break;
+                const TileHdr h = ti[g % kGInfo];
+                if (h.end) break;
+                ok = gwait(&k_full[g % NK], (uint32_t)(g / NK) & 1u, abort_flag);
+                if (ok && g >= kGSB)   // S buffer g % kGSB, read by the softmax of tile g - kGSB
+                    ok = gwait(&p_full[g % kGSB], ((uint32_t)(g / kGSB) & 1u) ^ 1u, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t dt = tmem + (uint32_t)((g % kGSB) * HQP);
+                const uint64_t kd = k_d + (uint64_t)(((g % NK) * C::kKV) >> 4);
+                const uint64_t qd = q_d + (uint64_t)(((h.j & 1) * C::kQ) >> 4);
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint64_t ka = (uint64_t)(((kk >> 2) * C::kHalf + (kk & 3) * 32) >> 4);
-                            const uint64_t qa = (uint64_t)(((kk >> 2) * C::kQHalf + (kk & 3) * 32) >> 4);
-                            mma_acc(dt, kd + ka, qd + qa, idesc_s, kk > 0 ? 1u : 0u);
-                        }
-                        tc_commit(&s_full[gs & 1]);
-                        if (h.last) tc_commit(&q_empty[h.j & 1]);
-                        info_j[gs & 1] = h.j;
-                        info_first[gs & 1] = h.i == 0;
-                        info_last[gs & 1] = h.last;
-                        ++gs;
-                    }
-                    progressed = true;
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t ka = (uint64_t)(((kk >> 2) * C::kHalf + (kk & 3) * 32) >> 4);
+                    const uint64_t qa = (uint64_t)(((kk >> 2) * C::kQHalf + (kk & 3) * 32) >> 4);
+                    mma_acc(dt, kd + ka, qd + qa, idesc_s, kk > 0 ? 1u : 0u);
                 }
-                // O^T += V^T P^T once the softmax wrote P(gp) (and, for a
-                // query's first tile, the epilogue of query j - 2 read its O)
-                if (gp < gs && mbar_try_wait(&p_full[gp & 1], (uint32_t)(gp >> 1) & 1u)) {
-                    const int j = info_j[gp & 1];
-                    const bool first = info_first[gp & 1] != 0;
-                    if (!first || j < 2 || mbar_try_wait(&o_empty[j & 1], ((uint32_t)(j >> 1) & 1u) ^ 1u)) {
-                        tc_fence_after();
-                        const uint32_t dt = tmem + (uint32_t)((2 + (j & 1)) * HQP);
-                        const uint64_t vd = v_d + (uint64_t)(((gp % NS) * C::kStage) >> 4);
-                        const uint64_t pd = p_d + (uint64_t)(((gp & 1) * C::kP) >> 4);
-#pragma unroll
-                        for (int kk = 0; kk < kGTile / 16; ++kk) {
-                            const uint64_t pa = (uint64_t)(((kk >> 2) * C::kQHalf + (kk & 3) * 32) >> 4);
-                            mma_acc(dt, vd + (uint64_t)((kk * 2048) >> 4), pd + pa, idesc_o,
-                                    (first && kk == 0) ? 0u : 1u);
-                        }
-                        tc_commit(&p_empty[gp & 1]);
-                        tc_commit(&kv_empty[gp % NS]);
-                        if (info_last[gp & 1]) tc_commit(&o_full[j & 1]);
-                        ++gp;
-                        progressed = true;
-                    }
-                }
-                if (progressed) {
-                    t0 = globaltimer();
-                } else if (*abort_flag || globaltimer() - t0 > kWaitLimitNs) {
-                    *abort_flag = 1;
-                    ok = false;
-                }
+                tc_commit(&s_full[g % kGSB]);
+                tc_commit(&k_empty[g % NK]);
+                if (h.last) tc_commit(&q_empty[h.j & 1]);
             }
-            tc_commit(drain);
+            tc_commit(&drain[0]);
             volatile int no_abort = 0;
-            mbar_wait(drain, 0, &no_abort);
+            gwait(&drain[0], 0, &no_abort);
+        }
+        __syncwarp();
+    } else if (warp == kWarpPV) {
+        // ------------------------------------------------------------ P V issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_o = idesc_bf16_f32(128, HQP) | (1u << 15);   // A (V^T) MN-major
+            const uint64_t v_d = desc_mn128(smem_u32(sm + C::kOffV), C::kHalf);
+            const uint64_t p_d = smem_desc(smem_u32(sm + C::kOffP), 1024, 2);
+            for (int g = 0;; ++g) {
+                bool ok = gwait(&ti_full[g % kGInfo], (uint32_t)(g / kGInfo) & 1u, abort_flag);
+                if (!ok) break;
+                const TileHdr h = ti[g % kGInfo];
+                if (h.end) break;
+                mbar_arrive(&ti_empty[g % kGInfo]);   // every reader of the record is done with it
+                // P(g) written, V(g) landed and, for a query's first tile, its O
+                // buffer read by the epilogue of query j - 2
+                ok = gwait(&p_full[g % kGSB], (uint32_t)(g / kGSB) & 1u, abort_flag) &&
+                     gwait(&v_full[g % NV], (uint32_t)(g / NV) & 1u, abort_flag);
+                if (ok && h.i == 0 && h.j >= 2)
+                    ok = gwait(&o_empty[h.j & 1], ((uint32_t)(h.j >> 1) & 1u) ^ 1u, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t dt = tmem + (uint32_t)((kGSB + (h.j & 1)) * HQP);
+                const uint64_t vd = v_d + (uint64_t)(((g % NV) * C::kKV) >> 4);
+                const uint64_t pd = p_d + (uint64_t)(((g % kGPB) * C::kP) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < kGTile / 16; ++kk) {
+                    const uint64_t pa = (uint64_t)(((kk >> 2) * C::kQHalf + (kk & 3) * 32) >> 4);
+                    mma_acc(dt, vd + (uint64_t)((kk * 2048) >> 4), pd + pa, idesc_o, (h.i == 0 && kk == 0) ? 0u : 1u);
+                }
+                tc_commit(&p_empty[g % kGPB]);
+                tc_commit(&v_empty[g % NV]);
+                if (h.last) tc_commit(&o_full[h.j & 1]);
+            }
+            tc_commit(&drain[1]);
+            volatile int no_abort = 0;
+            gwait(&drain[1], 0, &no_abort);
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ softmax + epilogue (warps 4..7)
-        const int quad = warp & 3;
+        // ------------------------------------------------------------ softmax + epilogue (warps 4..11)
+        constexpr int HG = HQP / 2;                       // heads of this group
+        const int quad = warp & 3, hg = (warp - 4) >> 2, h0 = hg * HG;
+        const int bar_red = 2 + 2 * hg, bar_x = 3 + 2 * hg;   // this group's named barriers
         const int key = quad * 32 + lane;                 // TMEM lane: key (S^T) or head dim (O^T)
-        const uint32_t lane_t = tmem + ((uint32_t)(quad * 32) << 16);
+        const uint32_t lane_t = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)h0;
+        float *gmax = redmax + hg * 4 * HG, *gsum = redsum + hg * 4 * HG;
         const float sl2 = P.scale_log2;
-        float m[HQP], l[HQP];
+        float m[HG], l[HG];
 #pragma unroll
-        for (int h = 0; h < HQP; ++h) { m[h] = -CUDART_INF_F; l[h] = 0.f; }
-        bool ok = true;
-        for (int g = 0; ok; ++g) {
-            const int s = g % NS, b = g & 1;
-            // the tile's record, then its S^T (both waits decided together)
-            bool w = mbar_wait(&kv_full[s], (uint32_t)(g / NS) & 1u, abort_flag);
-            TileHdr h = {};
-            if (w) {
-                h = ti[s];
-                if (!h.end) w = mbar_wait(&s_full[b], (uint32_t)(g >> 1) & 1u, abort_flag);
-            }
-            ok = bar_and(2, 128, w);
-            if (!ok || h.end) break;
-            tc_fence_after();
-            float x[HQP];
+        for (int h = 0; h < HG; ++h) { m[h] = -CUDART_INF_F; l[h] = 0.f; }
+        auto tload = [&](uint32_t col, float (&v)[HG]) {
 #pragma unroll
-            for (int c = 0; c < HQP; c += 16) {
-                uint32_t v[16];
-                tmem_ld_x16(lane_t + (uint32_t)(b * HQP + c), v);
+            for (int c = 0; c < HG; c += 8) {
+                uint32_t u[8];
+                tmem_ld_x8(lane_t + col + (uint32_t)c, u);
                 tmem_ld_wait();
 #pragma unroll
-                for (int u = 0; u < 16; ++u) x[c + u] = __uint_as_float(v[u]);
+                for (int e = 0; e < 8; ++e) v[c + e] = __uint_as_float(u[e]);
             }
+        };
+        // The epilogue of a query (O^T / l -> out, lse) runs one tile later, so
+        // that the softmax does not wait for the query's last P V.
+        int pend_j = -1, pend_t = 0;
+        auto epilogue = [&]() -> bool {
+            if (pend_j < 0) return true;
+            const int jb = pend_j & 1;
+            if (!bar_and(bar_red, 128, gwait(&o_full[jb], (uint32_t)(pend_j >> 1) & 1u, abort_flag))) return false;
+            tc_fence_after();
+            float o[HG];
+            tload((uint32_t)((kGSB + jb) * HQP), o);
+            uint16_t *orow = P.out + (int64_t)pend_t * P.Hq * D;
+#pragma unroll
+            for (int hh = 0; hh < HG; ++hh) {
+                if (h0 + hh < P.Hq) {
+                    const float L = epi_l[jb * HQP + h0 + hh];
+                    const __nv_bfloat16 ob = __float2bfloat16_rn(o[hh] * (L > 0.f ? 1.f / L : 0.f));
+                    orow[(int64_t)(h0 + hh) * D + key] = *reinterpret_cast<const uint16_t *>(&ob);
+                }
+            }
+            if (P.lse && quad == 0 && lane < HG && h0 + lane < P.Hq) {
+                const float L = epi_l[jb * HQP + h0 + lane];
+                P.lse[(int64_t)pend_t * P.Hq + h0 + lane] =
+                    (L > 0.f ? epi_m[jb * HQP + h0 + lane] + __log2f(L) : -CUDART_INF_F) * 0.69314718055994531f;
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&o_empty[jb]);
+            pend_j = -1;
+            return true;
+        };
+        bool ok = true;
+        for (int g = 0; ok; ++g) {
+            const int sb = g % kGSB, pb_i = g % kGPB;
+            // the tile's record, its S^T, and P buffer g % kGPB (free once P V of
+            // tile g - kGPB is done); the waits are decided together
+            bool w = gwait(&ti_full[g % kGInfo], (uint32_t)(g / kGInfo) & 1u, abort_flag);
+            TileHdr h = {};
+            if (w) {
+                h = ti[g % kGInfo];
+                if (!h.end) w = gwait(&s_full[sb], (uint32_t)(g / kGSB) & 1u, abort_flag);
+                if (!h.end && w && g >= kGPB)
+                    w = gwait(&p_empty[pb_i], ((uint32_t)(g / kGPB) & 1u) ^ 1u, abort_flag);
+            }
+            ok = bar_and(bar_red, 128, w);
+            if (!ok) break;
+            if (h.end) {
+                ok = epilogue();
+                break;
+            }
+            tc_fence_after();
+            float x[HG];
+            tload((uint32_t)(sb * HQP), x);
             const bool valid = key < h.nvalid;
 #pragma unroll
-            for (int hh = 0; hh < HQP; ++hh) x[hh] = valid ? x[hh] * sl2 : -CUDART_INF_F;
-            float wmax[HQP];
+            for (int hh = 0; hh < HG; ++hh) x[hh] = valid ? x[hh] * sl2 : -CUDART_INF_F;
+            // Is any score of this tile more than 2^8 above its head's running
+            // maximum?  (Always at a query's first tile, where the maximum is set.)
             bool need = h.i == 0;
 #pragma unroll
-            for (int hh = 0; hh < HQP; ++hh) {
-                wmax[hh] = warp_max(x[hh]);
-                need |= wmax[hh] > m[hh] + 8.f;
-            }
-            if (bar_or(2, 128, need)) {
-                // exact tile maximum of every head over the 128 key lanes
-                if (lane == 0) {
+            for (int hh = 0; hh < HG; ++hh) need |= x[hh] > m[hh] + 8.f;
+            if (bar_or(bar_red, 128, need)) {
+                // exact tile maximum of every head over the 128 key lanes:
+                // butterfly within each warp, then across the group's four warps
 #pragma unroll
-                    for (int hh = 0; hh < HQP; ++hh) redmax[quad * HQP + hh] = wmax[hh];
+                for (int hh = 0; hh < HG; ++hh) {
+                    float v = x[hh];
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+                    if (lane == 0) gmax[quad * HG + hh] = v;
                 }
-                bar_sync_n(3, 128);
-                float f[HQP];
+                bar_sync_n(bar_x, 128);
+                float f[HG];
                 bool resc = false;
 #pragma unroll
-                for (int hh = 0; hh < HQP; ++hh) {
-                    const float tm = fmaxf(fmaxf(redmax[hh], redmax[HQP + hh]),
-                                           fmaxf(redmax[2 * HQP + hh], redmax[3 * HQP + hh]));
+                for (int hh = 0; hh < HG; ++hh) {
+                    const float tm = fmaxf(fmaxf(gmax[hh], gmax[HG + hh]), fmaxf(gmax[2 * HG + hh], gmax[3 * HG + hh]));
                     f[hh] = 1.f;
                     if (h.i == 0) {
                         m[hh] = tm;
@@ -534,97 +643,68 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
                 }
                 if (resc) {
                     // O^T holds the query's earlier tiles: wait for P V of tile g - 1
-                    ok = bar_and(2, 128, mbar_wait(&p_empty[(g - 1) & 1], (uint32_t)((g - 1) >> 1) & 1u, abort_flag));
+                    ok = bar_and(bar_red, 128, gwait(&p_empty[(g - 1) % kGPB], (uint32_t)((g - 1) / kGPB) & 1u,
+                                                       abort_flag));
                     if (!ok) break;
                     tc_fence_after();
-                    const uint32_t ot = lane_t + (uint32_t)((2 + (h.j & 1)) * HQP);
+                    const uint32_t ot = lane_t + (uint32_t)((kGSB + (h.j & 1)) * HQP);
 #pragma unroll
-                    for (int c = 0; c < HQP; c += 16) {
-                        uint32_t o[16];
-                        tmem_ld_x16(ot + (uint32_t)c, o);
+                    for (int c = 0; c < HG; c += 8) {
+                        uint32_t o[8];
+                        tmem_ld_x8(ot + (uint32_t)c, o);
                         tmem_ld_wait();
 #pragma unroll
-                        for (int u = 0; u < 16; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * f[c + u]);
-                        tmem_st16(ot + (uint32_t)c, o);
+                        for (int e = 0; e < 8; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f[c + e]);
+                        tmem_st8(ot + (uint32_t)c, o);
                     }
                     tmem_st_wait_all();
                 }
             }
-            // P buffer g % 2 is free once P V of tile g - 2 is done
-            if (g >= 2) {
-                ok = bar_and(2, 128, mbar_wait(&p_empty[b], ((uint32_t)(g >> 1) & 1u) ^ 1u, abort_flag));
-                if (!ok) break;
-            }
-            // P^T (heads x keys, K-major SW128): key = this lane
-            uint8_t *pb = sm + C::kOffP + b * C::kP;
-            const int khalf = key >> 6, kc = key & 63;
+            // P^T (heads x keys, K-major SW128): key = this lane, heads h0 ..
+            uint8_t *pbuf = sm + C::kOffP + pb_i * C::kP + (key >> 6) * C::kQHalf;
+            const int kc = key & 63;
 #pragma unroll
-            for (int hh = 0; hh < HQP; ++hh) {
+            for (int hh = 0; hh < HG; ++hh) {
+                const int row = h0 + hh;
                 const float pv = ex2f(x[hh] - m[hh]);
                 l[hh] += pv;
                 const __nv_bfloat16 bv = __float2bfloat16_rn(pv);
-                *reinterpret_cast<__nv_bfloat16 *>(pb + khalf * C::kQHalf + hh * 128 +
-                                                   ((((kc >> 3) ^ (hh & 7)) << 4) | ((kc & 7) << 1))) = bv;
+                *reinterpret_cast<__nv_bfloat16 *>(pbuf + row * 128 + ((((kc >> 3) ^ (row & 7)) << 4) | ((kc & 7) << 1))) = bv;
             }
             fence_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&p_full[b]);
+            if (lane == 0) mbar_arrive(&p_full[sb]);
+            // the previous query's epilogue, now that this tile is handed over
+            if (!(ok = epilogue())) break;
             if (h.last) {
-                // ---- epilogue of query h.t: O^T / l
-                ok = bar_and(2, 128, mbar_wait(&o_full[h.j & 1], (uint32_t)(h.j >> 1) & 1u, abort_flag));
-                if (!ok) break;
-                tc_fence_after();
-                float L[HQP];
+                // the query's row sums over all 128 key lanes and its maxima,
+                // kept for its epilogue
 #pragma unroll
-                for (int hh = 0; hh < HQP; ++hh) {
+                for (int hh = 0; hh < HG; ++hh) {
                     float v = l[hh];
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                    L[hh] = v;
+                    if (lane == 0) gsum[quad * HG + hh] = v;
                 }
-                if (lane == 0) {
+                bar_sync_n(bar_x, 128);
+                if (quad == 0 && lane < HG) {
+                    const int jb = h.j & 1;
+                    epi_l[jb * HQP + h0 + lane] = (gsum[lane] + gsum[HG + lane]) + (gsum[2 * HG + lane] + gsum[3 * HG + lane]);
 #pragma unroll
-                    for (int hh = 0; hh < HQP; ++hh) redsum[quad * HQP + hh] = L[hh];
+                    for (int hh = 0; hh < HG; ++hh)
+                        if (hh == lane) epi_m[jb * HQP + h0 + lane] = m[hh];
                 }
-                bar_sync_n(3, 128);
-#pragma unroll
-                for (int hh = 0; hh < HQP; ++hh)
-                    L[hh] = (redsum[hh] + redsum[HQP + hh]) + (redsum[2 * HQP + hh] + redsum[3 * HQP + hh]);
-                const uint32_t ot = lane_t + (uint32_t)((2 + (h.j & 1)) * HQP);
-                uint16_t *orow = P.out + (int64_t)h.t * P.Hq * D;
-#pragma unroll
-                for (int c = 0; c < HQP; c += 16) {
-                    uint32_t o[16];
-                    tmem_ld_x16(ot + (uint32_t)c, o);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        const int hh = c + u;
-                        if (hh < P.Hq) {
-                            const float inv = L[hh] > 0.f ? 1.f / L[hh] : 0.f;
-                            const __nv_bfloat16 ob = __float2bfloat16_rn(__uint_as_float(o[u]) * inv);
-                            orow[(int64_t)hh * D + key] = *reinterpret_cast<const uint16_t *>(&ob);
-                        }
-                    }
-                }
-                if (P.lse && quad == 0) {
-#pragma unroll
-                    for (int hh = 0; hh < HQP; ++hh)
-                        if (lane == hh && hh < P.Hq)
-                            P.lse[(int64_t)h.t * P.Hq + hh] =
-                                (L[hh] > 0.f ? m[hh] + __log2f(L[hh]) : -CUDART_INF_F) * 0.69314718055994531f;
-                }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&o_empty[h.j & 1]);
+                bar_sync_n(bar_x, 128);   // epi_* written before any warp's epilogue reads them
+                pend_j = h.j;
+                pend_t = h.t;
             }
         }
     }
     // Once every role is past its last TMEM access, warp 8 frees TMEM.
     tc_fence_before();
     bar_sync_n(1, kGThreads);
-    if (warp == 8) {
+    if (warp == kWarpS) {
         if (lane == 0 && *abort_flag) report(P.dev_status, SA_DEV_TIMEOUT);
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);

@@ -22,6 +22,12 @@ struct TopkArgs {
     int32_t *out;
     int *dev_status;
     int chunk;   // columns per CTA (set by the launcher)
+    // two-stage candidates given by block ids instead of a position map:
+    // columns are the tokens of the valid (ascending) ids of blocks[r, :keep],
+    // then the query's own block up to its position p = S - rows + r
+    bool by_blocks = false;
+    const int32_t *blocks = nullptr;   // [rows, keep]; may be NULL when keep == 0
+    int keep = 0, block = 0, S = 0;
 };
 sa_status launch_topk(TopkArgs a, cudaStream_t st);
 int topk_max_row_len();

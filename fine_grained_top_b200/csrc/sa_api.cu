@@ -160,6 +160,23 @@ sa_status sa_topk_select(const float *scores, int64_t ld_scores, int rows, int r
     });
 }
 
+sa_status sa_topk_select_blocks(const float *scores, int64_t ld_scores, int T, int S, const int32_t *blocks, int keep,
+                                int block, int K, int32_t *topk, int *dev_status, sa_stream stream) {
+    if (T < 0 || S < T || keep < 0 || block <= 0 || K < 0) return SA_ERR_INVALID_ARG;
+    const int64_t row_len = (int64_t)keep * block + block;
+    if (ld_scores < row_len || (ld_scores & 3)) return SA_ERR_INVALID_ARG;
+    if (row_len > topk_max_row_len()) return SA_ERR_UNSUPPORTED;
+    if (T == 0 || K == 0) return SA_OK;
+    if (!scores || !topk || (keep > 0 && !blocks) || !aligned16(scores)) return SA_ERR_INVALID_ARG;
+    return guarded([&] {
+        TopkArgs a;
+        a.scores = scores; a.ld = ld_scores; a.rows = T; a.row_len = (int)row_len; a.n_valid = nullptr;
+        a.cand = nullptr; a.ld_cand = 0; a.K = K; a.out = topk; a.dev_status = dev_status; a.chunk = 0;
+        a.by_blocks = true; a.blocks = keep > 0 ? blocks : nullptr; a.keep = keep; a.block = block; a.S = S;
+        return launch_topk(a, cs(stream));
+    });
+}
+
 size_t sa_prefill_workspace_bytes(int T, int S, int K, int W, int Hq, int d) {
     if (T < 0 || S < 0 || K < 0 || W < 0) return 0;
     PrefillArgs a = {};

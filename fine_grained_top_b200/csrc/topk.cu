@@ -6,7 +6,9 @@
 // scores ranked by lower position, emitted in ascending position order.
 //
 // Design (sm_100a):
-//   * one row per thread-block cluster of G = 1..16 CTAs; CTA c of the
+//   * rows of at most 1024 columns: one warp per row, the keys in registers,
+//     a bitwise search for the K-th key (topk_rows_kernel);
+//   * longer rows: one row per thread-block cluster of G = 1..16 CTAs; CTA c of the
 //     cluster owns a contiguous chunk of the row, loaded once from HBM with
 //     16-byte vector loads into shared memory as order-preserving uint32 keys;
 //   * exact radix select over the keys in three passes of 12, 10 and 10 bits.
@@ -130,7 +132,35 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     int n;
-    if (a.n_valid) {
+    int n_kept = 0, own0 = 0;   // block-id candidates: valid kept blocks, first token of the own block
+    const bool byb = a.by_blocks;
+    const int32_t *brow = (byb && a.keep > 0) ? a.blocks + (int64_t)r * a.keep : nullptr;
+    if (byb) {
+        const int p = a.S - a.rows + r, own = p / a.block;
+        own0 = own * a.block;
+        // the valid ids form a prefix, strictly ascending, each below the own block
+        if (tid == 0) cta_counts[0] = 0u;
+        __syncthreads();
+        uint32_t valid = 0;
+        for (int i = tid; i < a.keep; i += kTopkThreads) {
+            const int b = brow[i];
+            if (b >= 0) {
+                ++valid;
+                if (rank == 0 && b >= own) report(a.dev_status, SA_DEV_INDEX);
+                if (rank == 0 && i > 0 && !(brow[i - 1] >= 0 && brow[i - 1] < b)) report(a.dev_status, SA_DEV_ORDER);
+            }
+        }
+        valid = __reduce_add_sync(0xffffffffu, valid);
+        if (lane == 0 && valid) atomicAdd(&cta_counts[0], valid);
+        __syncthreads();
+        n_kept = (int)cta_counts[0];
+        __syncthreads();
+        n = n_kept * a.block + (p - own0 + 1);
+        if (n > a.row_len) {
+            if (rank == 0 && tid == 0) report(a.dev_status, SA_DEV_INDEX);
+            n = a.row_len;
+        }
+    } else if (a.n_valid) {
         n = a.n_valid[r];
         if (n < 0 || n > a.row_len) {
             if (rank == 0 && tid == 0) report(a.dev_status, SA_DEV_INDEX);
@@ -146,6 +176,14 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     int32_t *out = a.out + (int64_t)r * a.K;
     const float *row = a.scores + (int64_t)r * a.ld;
     const int32_t *cand = a.cand ? a.cand + (int64_t)r * a.ld_cand : nullptr;
+    // position of column col: through the block ids, the position map, or itself
+    auto pos = [&](int col) -> int32_t {
+        if (byb) {
+            const int kb = n_kept * a.block;
+            return col < kb ? brow[col / a.block] * a.block + col % a.block : own0 + (col - kb);
+        }
+        return cand ? cand[col] : col;
+    };
 
     if (cand) {   // the position map must be strictly ascending and non-negative
         for (int i = tid; i < len; i += kTopkThreads) {
@@ -157,7 +195,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     }
 
     if (n <= a.K) {   // every candidate is kept: no select needed
-        for (int i = tid; i < len; i += kTopkThreads) out[c0 + i] = cand ? cand[c0 + i] : c0 + i;
+        for (int i = tid; i < len; i += kTopkThreads) out[c0 + i] = pos(c0 + i);
         if (rank == 0)
             for (int i = n + tid; i < a.K; i += kTopkThreads) out[i] = -1;
         return;   // uniform over the cluster: no distributed smem was touched
@@ -323,8 +361,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
             for (int e = 0; e < 4; ++e) {
                 const bool is_gt = (f >> e) & 1u, is_eq = (f >> (4 + e)) & 1u;
                 if (is_gt || (is_eq && eq_before < need)) {
-                    const int col = c0 + p + e;
-                    out[gt_before + min(eq_before, need)] = cand ? cand[col] : col;
+                    out[gt_before + min(eq_before, need)] = pos(c0 + p + e);
                 }
                 gt_before += is_gt ? 1u : 0u;
                 eq_before += is_eq ? 1u : 0u;
@@ -333,6 +370,171 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
         run += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (G > 1) cluster_sync();   // peers may still read this CTA's counters
+}
+
+// Short rows (the coarse block selection, small prefills): a group of W warps
+// per row (W = 1 for the rows of at most 1024 columns it is used for), the row's keys
+// in registers, thread t of the group holding the PER consecutive columns
+// from t * PER.  The K-th largest key tau is found bit by bit from the top:
+// a candidate bit is kept when at least K keys are >= the candidate (counts
+// summed over the group).  The kept keys are then written in column order
+// after one scan of the "> tau" and "== tau" counts over the group, the
+// lowest-positioned ties first.
+constexpr int kRowsThreads = 256;
+
+template <int PER, int W>
+__global__ void __launch_bounds__(kRowsThreads) topk_rows_kernel(TopkArgs a) {
+    constexpr int GT = 32 * W;                        // threads per row
+    constexpr int RPC = kRowsThreads / GT;            // rows per CTA
+    __shared__ uint32_t red[RPC][2][W];               // per-warp partial counts (double-buffered by round)
+    __shared__ uint32_t scan[RPC][W];
+    const int grp = threadIdx.x / GT, t = threadIdx.x % GT, lane = t & 31, wg = t >> 5;
+    const int r = blockIdx.x * RPC + grp;
+    if (r >= a.rows) return;   // whole groups leave together (rows are group-uniform)
+    auto group_sync = [&]() {
+        if (W > 1) asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(GT) : "memory");
+    };
+    // sum of v over the group; `round` alternates the exchange buffer, so one
+    // barrier per sum suffices
+    auto group_sum = [&](uint32_t v, int round) -> uint32_t {
+        v = __reduce_add_sync(0xffffffffu, v);
+        if (W == 1) return v;
+        if (lane == 0) red[grp][round & 1][wg] = v;
+        group_sync();
+        uint32_t s2 = 0;
+#pragma unroll
+        for (int w = 0; w < W; ++w) s2 += red[grp][round & 1][w];
+        return s2;
+    };
+    int n;
+    int n_kept = 0, own0 = 0;   // block-id candidates: valid kept blocks, first token of the own block
+    const bool byb = a.by_blocks;
+    const int32_t *brow = (byb && a.keep > 0) ? a.blocks + (int64_t)r * a.keep : nullptr;
+    if (byb) {
+        const int p = a.S - a.rows + r, own = p / a.block;
+        own0 = own * a.block;
+        // the valid ids form a prefix, strictly ascending, each below the own block
+        uint32_t valid = 0;
+        for (int i = t; i < a.keep; i += GT) {
+            const int b = brow[i];
+            if (b >= 0) {
+                ++valid;
+                if (b >= own) report(a.dev_status, SA_DEV_INDEX);
+                if (i > 0 && !(brow[i - 1] >= 0 && brow[i - 1] < b)) report(a.dev_status, SA_DEV_ORDER);
+            }
+        }
+        n_kept = (int)group_sum(valid, 0);
+        group_sync();   // the count's exchange buffer is reused by the search
+        n = n_kept * a.block + (p - own0 + 1);
+        if (n > a.row_len) {
+            if (t == 0) report(a.dev_status, SA_DEV_INDEX);
+            n = a.row_len;
+        }
+    } else if (a.n_valid) {
+        n = a.n_valid[r];
+        if (n < 0 || n > a.row_len) {
+            if (t == 0) report(a.dev_status, SA_DEV_INDEX);
+            n = n < 0 ? 0 : a.row_len;
+        }
+    } else {
+        n = a.row_len - a.rows + r + 1;
+        n = n < 0 ? 0 : (n > a.row_len ? a.row_len : n);
+    }
+    int32_t *out = a.out + (int64_t)r * a.K;
+    const float *row = a.scores + (int64_t)r * a.ld;
+    const int32_t *cand = a.cand ? a.cand + (int64_t)r * a.ld_cand : nullptr;
+    // position of column col: through the block ids, the position map, or itself
+    auto pos = [&](int col) -> int32_t {
+        if (byb) {
+            const int kb = n_kept * a.block;
+            return col < kb ? brow[col / a.block] * a.block + col % a.block : own0 + (col - kb);
+        }
+        return cand ? cand[col] : col;
+    };
+    const int c_lo = t * PER;
+    if (cand) {   // the position map must be strictly ascending and non-negative
+        for (int col = t; col < n; col += GT) {
+            const int32_t c = cand[col];
+            if (c < 0) report(a.dev_status, SA_DEV_INDEX);
+            if (col > 0 && cand[col - 1] >= c) report(a.dev_status, SA_DEV_ORDER);
+        }
+    }
+    if (n <= a.K) {   // every column is kept
+        for (int col = t; col < a.K; col += GT) out[col] = col < n ? pos(col) : -1;
+        return;
+    }
+    uint32_t key[PER];
+    if (PER % 4 == 0 && c_lo + PER <= n) {   // 16-byte loads (rows start 16-byte aligned, PER % 4 == 0)
+#pragma unroll
+        for (int e = 0; e < PER; e += 4) {
+            const float4 f = __ldg(reinterpret_cast<const float4 *>(row + c_lo + e));
+            key[e] = order_key(f.x); key[e + 1] = order_key(f.y);
+            key[e + 2] = order_key(f.z); key[e + 3] = order_key(f.w);
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+            const int col = c_lo + e;
+            key[e] = col < n ? order_key(__ldg(row + col)) : 0u;   // 0 ranks below every score
+        }
+    }
+    // tau = the largest value with at least K keys >= tau
+    uint32_t tau = 0u;
+#pragma unroll 1
+    for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t c = tau | (1u << bit);
+        uint32_t cnt = 0;
+#pragma unroll
+        for (int e = 0; e < PER; ++e) cnt += key[e] >= c ? 1u : 0u;
+        if (group_sum(cnt, bit) >= (uint32_t)a.K) tau = c;
+    }
+    uint32_t gt = 0, eq = 0;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+        gt += key[e] > tau ? 1u : 0u;
+        eq += key[e] == tau ? 1u : 0u;
+    }
+    // packed (eq << 16 | gt) counts: exclusive scan over the group's threads
+    const uint32_t packed = gt | (eq << 16);
+    uint32_t incl = packed;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+    }
+    uint32_t before_w = 0, total = incl;
+    if (W > 1) {
+        if (lane == 31) scan[grp][wg] = incl;
+        group_sync();
+        total = 0;
+#pragma unroll
+        for (int w = 0; w < W; ++w) {
+            const uint32_t v = scan[grp][w];
+            before_w += w < wg ? v : 0u;
+            total += v;
+        }
+    } else {
+        total = __shfl_sync(0xffffffffu, incl, 31);
+    }
+    const uint32_t need = (uint32_t)a.K - (total & 0xFFFFu);   // ties to take
+    const uint32_t excl = before_w + incl - packed;
+    uint32_t gt_before = excl & 0xFFFFu, eq_before = excl >> 16;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+        const bool is_gt = key[e] > tau, is_eq = key[e] == tau;
+        if (is_gt || (is_eq && eq_before < need)) {
+            out[gt_before + min(eq_before, need)] = pos(c_lo + e);
+        }
+        gt_before += is_gt ? 1u : 0u;
+        eq_before += is_eq ? 1u : 0u;
+    }
+}
+
+template <int PER, int W>
+static sa_status launch_topk_rows(const TopkArgs &a, cudaStream_t st) {
+    constexpr int RPC = kRowsThreads / (32 * W);
+    topk_rows_kernel<PER, W><<<(a.rows + RPC - 1) / RPC, kRowsThreads, 0, st>>>(a);
+    return cuda_ok(cudaGetLastError());
 }
 
 template <int G>
@@ -355,6 +557,12 @@ static sa_status launch_topk_g(const TopkArgs &a, size_t smem, cudaStream_t st) 
 }
 
 sa_status launch_topk(TopkArgs a, cudaStream_t st) {
+    // Rows of at most 1024 columns: the register search (32 rounds over at most
+    // 32 keys per lane).  Longer rows: the histogram select, whose passes cost
+    // a few operations per key rather than 32.
+    if (a.row_len <= 256) return launch_topk_rows<8, 1>(a, st);
+    if (a.row_len <= 512) return launch_topk_rows<16, 1>(a, st);
+    if (a.row_len <= 1024) return launch_topk_rows<32, 1>(a, st);
     int g = 1;
     while (g < kTopkMaxCluster && (a.row_len + g - 1) / g > kTopkChunkTarget) g *= 2;
     int chunk = (a.row_len + g - 1) / g;

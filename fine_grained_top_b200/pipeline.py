@@ -21,9 +21,10 @@ import math
 import torch
 
 from . import (sa_block_scores_workspace_bytes, sa_coarse_block_counts, sa_decode_workspace_bytes,
-               sa_expand_blocks, sa_indexer_scores, sa_indexer_scores_blocks, sa_indexer_scores_fp8,
+               sa_indexer_scores, sa_indexer_scores_blocks, sa_indexer_scores_fp8,
                sa_pool_index_keys,
-               sa_prefill_workspace_bytes, sa_sparse_attn_decode, sa_sparse_attn_prefill, sa_topk_select)
+               sa_prefill_workspace_bytes, sa_sparse_attn_decode, sa_sparse_attn_prefill, sa_topk_select,
+               sa_topk_select_blocks)
 
 
 def _ld(n: int) -> int:
@@ -78,8 +79,6 @@ class PrefillPlan:
             self.coarse = torch.empty((N, self.ld_coarse), dtype=f32, device=dev)
             self.blocks = torch.empty((N, keep), dtype=i32, device=dev)
             self.ld_cand = _ld(keep * block + block)
-            self.cand = torch.empty((N, self.ld_cand), dtype=i32, device=dev)
-            self.n_cand = torch.empty(N, dtype=i32, device=dev)
             self.fine = torch.empty((N, self.ld_cand), dtype=f32, device=dev)
             self.ws_bytes = sa_block_scores_workspace_bytes(N, S, keep)
             self.workspace = torch.empty(self.ws_bytes, dtype=torch.uint8, device=dev)
@@ -119,13 +118,11 @@ class PrefillPlan:
                                                          stream)),
             ("coarse_topk", lambda: sa_topk_select(self.coarse, self.ld_coarse, N, self.nb, self.n_blocks, None,
                                                    0, keep, self.blocks, ds, stream)),
-            ("expand", lambda: sa_expand_blocks(self.blocks, N, S, keep, blk, self.cand, self.ld_cand,
-                                                self.n_cand, ds, stream)),
             ("fine_indexer", lambda: sa_indexer_scores_blocks(x["qI"], x["w"], x["kI"], N, S, H, D, self.blocks,
                                                               keep, blk, self.fine, self.ld_cand, self.workspace,
                                                               self.ws_bytes, ds, stream)),
-            ("fine_topk", lambda: sa_topk_select(self.fine, self.ld_cand, N, self.ld_cand, self.n_cand,
-                                                 self.cand, self.ld_cand, K, self.topk, ds, stream)),
+            ("fine_topk", lambda: sa_topk_select_blocks(self.fine, self.ld_cand, N, S, self.blocks, keep, blk, K,
+                                                        self.topk, ds, stream)),
             attn]
 
     def run(self, q, k, v, qI, w, kI, stream=None):
@@ -136,10 +133,11 @@ class PrefillPlan:
     def launches(self) -> int:
         """Kernels one run() enqueues: indexer + top-K (per row block), or for
         the two-stage selection pool, block counts, coarse indexer, coarse
-        top-k, expand, the fine scores' invert count / scan / scatter and
-        block kernel, and the fine top-K (10); then the attention."""
+        top-k, the fine scores' invert count / scan / scatter and block
+        kernel, and the fine top-K over the kept block ids (9); then the
+        attention."""
         attn = 2 if self.attn_ws is not None else 1   # (selection bitmap +) attention
-        return (2 * self.row_blocks if self.block is None else 10) + attn
+        return (2 * self.row_blocks if self.block is None else 9) + attn
 
 
 class DecodePlan:

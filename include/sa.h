@@ -203,13 +203,38 @@ sa_status sa_indexer_scores_blocks(const sa_bf16 *qI, const sa_bf16 *w,
  *             `row_len` positions, n_valid = row_len - rows + r + 1).
  *   Order-preserving keys: NaN scores are not supported; -inf sorts last.
  *   Limits: row_len <= 524288; K >= 0.
- *   Rows are split over a thread-block cluster (1..16 CTAs, distributed
- *   shared memory for the histograms); no workspace is needed.
+ *   Rows of at most 1024 columns are selected by one warp holding the row
+ *   in registers; longer rows are split over a thread-block cluster
+ *   (1..16 CTAs, distributed shared memory for the histograms).  No
+ *   workspace is needed.
  * ---------------------------------------------------------------------- */
 sa_status sa_topk_select(const float *scores, int64_t ld_scores, int rows,
                          int row_len, const int32_t *n_valid,
                          const int32_t *cand_map, int64_t ld_cand, int K,
                          int32_t *topk, int *dev_status, sa_stream stream);
+
+/* The same select over the two-stage candidates, given by the kept block ids
+ * instead of a position map ("What Fine-Grained Means": the fine pass picks
+ * top-K tokens inside the blocks the coarse pass kept).
+ *
+ *   T queries at positions p = S - T + t.  Row t's columns are the tokens of
+ *   the valid ids of blocks[t*keep .. t*keep + keep) (as sa_topk_select wrote
+ *   them: ascending, each < p / block, then -1 padding), `block` columns per
+ *   id, followed by the query's own block p / block up to p -- the layout
+ *   sa_indexer_scores_blocks writes its scores in.  Column c of the n =
+ *   n_kept * block + (p % block + 1) valid columns is position
+ *   blocks[t, c / block] * block + c % block (c < n_kept * block), else
+ *   (p / block) * block + c - n_kept * block.
+ *   scores: [T, ld_scores] fp32, ld_scores >= keep*block + block, a multiple
+ *   of 4, 16-byte aligned.  topk: [T, K], ascending positions, then -1.
+ *   Device errors: an id >= p / block sets SA_DEV_INDEX, ids out of order
+ *   SA_DEV_ORDER.  Limits: keep*block + block <= 524288 (SA_ERR_UNSUPPORTED).
+ *   No workspace; blocks may be NULL when keep == 0.
+ */
+sa_status sa_topk_select_blocks(const float *scores, int64_t ld_scores, int T,
+                                int S, const int32_t *blocks, int keep,
+                                int block, int K, int32_t *topk,
+                                int *dev_status, sa_stream stream);
 
 /* ------------------------------------------------------------------------
  * Stage 3a -- sparse attention, prefill

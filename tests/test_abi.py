@@ -56,6 +56,19 @@ P = ctypes.c_void_p(16)   # a fake, 16-byte aligned, never dereferenced pointer
 N0 = None
 
 
+def test_topk_blocks_argument_checks(sa):
+    f = sa._lib.sa_topk_select_blocks
+    # scores, ld, T, S, blocks, keep, block, K, topk, dev_status, stream
+    assert f(P, 4160, 10, 9, P, 64, 64, 2048, P, N0, N0) == sa.SA_ERR_INVALID_ARG      # S < T
+    assert f(P, 4100, 10, 10, P, 64, 64, 2048, P, N0, N0) == sa.SA_ERR_INVALID_ARG     # ld < keep*block + block
+    assert f(P, 4162, 10, 10, P, 64, 64, 2048, P, N0, N0) == sa.SA_ERR_INVALID_ARG     # ld not a multiple of 4
+    assert f(P, 524352, 10, 10, P, 8192, 64, 2048, P, N0, N0) == sa.SA_ERR_UNSUPPORTED  # rows of 524352 columns
+    assert f(P, 4160, 10, 10, N0, 64, 64, 2048, P, N0, N0) == sa.SA_ERR_INVALID_ARG    # no block ids
+    assert f(ctypes.c_void_p(20), 4160, 10, 10, P, 64, 64, 2048, P, N0, N0) == sa.SA_ERR_INVALID_ARG   # misaligned
+    assert f(P, 4160, 0, 10, P, 64, 64, 2048, P, N0, N0) == sa.SA_OK                   # nothing to do
+    assert f(P, 64, 10, 10, N0, 0, 64, 0, P, N0, N0) == sa.SA_OK                       # K = 0
+
+
 def test_topk_argument_checks(sa):
     f = sa._lib.sa_topk_select
     assert f(P, 8, -1, 8, N0, N0, 0, 4, P, N0, N0) == sa.SA_ERR_INVALID_ARG      # rows < 0

@@ -50,6 +50,9 @@ def _scores(rows, L, dist, rng):
     (3, 40000, 100, "normal"), (8, 131072, 2048, "ints"), (4, 262144, 2048, "ties3"),
     (5, 393216, 3000, "ints"), (2, 524288, 2048, "normal"), (9, 33, 40, "normal"), (64, 1023, 64, "ints"),
     (300, 8192, 1024, "ties3"), (33, 16384, 16000, "ties3"),
+    # rows of at most 1024 columns (one warp per row)
+    (100, 1024, 64, "ties3"), (77, 257, 200, "normal"), (5, 1024, 1023, "ints"), (1000, 1000, 64, "ints"),
+    (3, 1, 1, "normal"), (20, 700, 699, "ties3"),
 ])
 def test_topk_matches_oracle(sa, rows, L, K, dist):
     rng = np.random.default_rng(rows * 7 + L)
@@ -81,19 +84,66 @@ def test_topk_causal_default_and_neg_inf(sa):
     assert np.array_equal(out.cpu().numpy(), want)
 
 
-def test_topk_candidate_map(sa):
-    rng = np.random.default_rng(4)
-    rows, L, K = 40, 4160, 2048
+@pytest.mark.parametrize("rows,L,K", [(40, 4160, 2048), (50, 1000, 64), (33, 300, 100)])
+def test_topk_candidate_map(sa, rows, L, K):
+    rng = np.random.default_rng(4 + L)
     sc = rng.integers(0, 50, size=(rows, L)).astype(np.float32)
     cand = np.sort(rng.choice(1 << 20, size=(rows, L), replace=True), axis=1).astype(np.int32)
     cand = cand + np.arange(L, dtype=np.int32)[None, :]          # strictly ascending
-    n_valid = rng.integers(1000, L + 1, size=rows).astype(np.int32)
+    n_valid = rng.integers(min(1000, L // 2), L + 1, size=rows).astype(np.int32)
     out = torch.empty((rows, K), dtype=torch.int32, device="cuda")
     ds = torch.zeros(1, dtype=torch.int32, device="cuda")
     sa.sa_topk_select(dev(sc), L, rows, L, dev(n_valid), dev(cand), L, K, out, ds)
     want = oracle.topk(sc.astype(np.float64), n_valid, K, cand=cand)
     assert status(ds) == 0
     assert np.array_equal(out.cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("T,S,keep,K,dist", [(300, 5000, 64, 2048, "ties3"), (257, 4097, 16, 500, "ints"),
+                                             (100, 100, 4, 50, "normal"), (130, 9000, 0, 40, "ints"),
+                                             (64, 64 * 70, 127, 1000, "ties3")])
+def test_topk_over_block_ids_matches_oracle(sa, T, S, keep, K, dist):
+    # the two-stage fine select reading its candidates from the kept block ids
+    rng = np.random.default_rng(T + keep)
+    blk = 64
+    pos = np.arange(S - T, S)
+    own = pos // blk
+    blocks = np.full((T, max(keep, 1)), -1, dtype=np.int32)
+    n_kept = np.zeros(T, dtype=np.int64)
+    for t in range(T):
+        k = min(keep, int(own[t]), int(rng.integers(0, keep + 1)) if t % 3 == 0 else keep)
+        blocks[t, :k] = np.sort(rng.choice(int(own[t]), size=k, replace=False)) if k else []
+        n_kept[t] = k
+    L = keep * blk + blk
+    ld = (L + 3) // 4 * 4
+    sc = _scores(T, ld, dist, rng)
+    # the oracle's view: candidate positions in column order
+    cand = np.zeros((T, L), dtype=np.int64)
+    for t in range(T):
+        toks = (blocks[t, :n_kept[t]][:, None] * blk + np.arange(blk)[None, :]).reshape(-1)
+        toks = np.r_[toks, own[t] * blk + np.arange(pos[t] - own[t] * blk + 1)]
+        cand[t, :len(toks)] = toks
+        cand[t, len(toks):] = toks[-1] + 1 + np.arange(L - len(toks))   # unused columns, ascending
+    n_valid = n_kept * blk + (pos - own * blk + 1)
+    out = torch.empty((T, K), dtype=torch.int32, device="cuda")
+    ds = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sa.sa_topk_select_blocks(dev(sc), ld, T, S, dev(blocks) if keep else None, keep, blk, K, out, ds)
+    want = oracle.topk(sc[:, :L].astype(np.float64), n_valid, K, cand=cand)
+    assert status(ds) == 0
+    assert np.array_equal(out.cpu().numpy(), want)
+
+
+def test_topk_over_block_ids_reports_bad_ids(sa):
+    T, S, keep, K = 8, 1000, 4, 16
+    blocks = np.tile(np.array([0, 1, 2, 3], dtype=np.int32), (T, 1))
+    blocks[3, 2] = 999                       # not below the own block
+    blocks[5] = [2, 1, 3, 4]                 # not ascending
+    sc = np.zeros((T, keep * 64 + 64), dtype=np.float32)
+    out = torch.empty((T, K), dtype=torch.int32, device="cuda")
+    ds = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sa.sa_topk_select_blocks(dev(sc), keep * 64 + 64, T, S, dev(blocks), keep, 64, K, out, ds)
+    st = status(ds)
+    assert st & sa.SA_DEV_INDEX and st & sa.SA_DEV_ORDER
 
 
 # ====================================================================== indexer

@@ -40,8 +40,11 @@ def test_two_stage_and_page_granular_plans(pl):
     _, pipeline = pl
     p = pipeline.PrefillPlan(4096, 16, 128, 4, 64, 512, 64, block=64, keep=16, device="cpu")
     assert p.nb == 64 and tuple(p.blocks.shape) == (4096, 16)
-    assert p.ld_cand == 16 * 64 + 64 and tuple(p.cand.shape) == (4096, p.ld_cand)
-    assert p.launches() == 10 + 2       # ncu launch list: 10 selection kernels, bitmap, masked attention
+    assert p.ld_cand == 16 * 64 + 64 and tuple(p.fine.shape) == (4096, p.ld_cand)
+    assert p.launches() == 9 + 2        # 9 selection kernels (no candidate map), bitmap, masked attention
+    names = [n for n, _ in p.stages({k: None for k in ("q", "k", "v", "qI", "w", "kI")})]
+    assert names == ["pool", "block_counts", "coarse_indexer", "coarse_topk", "fine_indexer", "fine_topk",
+                     "attention"]
     # page-granular: the fine top-K may keep every candidate
     q = pipeline.PrefillPlan(4096, 16, 128, 4, 64, 16 * 64 + 64, 64, block=64, keep=16, device="cpu")
     assert tuple(q.topk.shape) == (4096, q.ld_cand)
