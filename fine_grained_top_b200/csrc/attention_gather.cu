@@ -158,6 +158,25 @@ __device__ __forceinline__ bool gwait(uint64_t *bar, uint32_t parity, volatile i
         }
     }
 }
+// The two MMA-issuing threads poll with plain mbarrier.try_wait (no suspend
+// hint): each is one thread, and a parked issuer wakes late and delays the
+// hand-off it waits for.
+__device__ __forceinline__ bool try_wait_issuer(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool iwait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    if (try_wait_issuer(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    while (true) {
+        for (int i = 0; i < 16; ++i) if (try_wait_issuer(bar, parity)) return true;
+        if (*abort) return false;
+        if (globaltimer() - t0 > kWaitLimitNs) { *abort = 1; return false; }
+    }
+}
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 // Barrier `id` over `n` threads that also returns the OR / AND of a predicate.
@@ -468,13 +487,13 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
             for (int g = 0;; ++g) {
                 // the tile's record and K(g) (the record is written before K's
                 // completion), and S buffer g % 2 read by the softmax of tile g - 2
-                bool ok = gwait(&ti_full[g % kGInfo], (uint32_t)(g / kGInfo) & 1u, abort_flag);
+                bool ok = iwait(&ti_full[g % kGInfo], (uint32_t)(g / kGInfo) & 1u, abort_flag);
                 if (!ok) break;
                 const TileHdr h = ti[g % kGInfo];
                 if (h.end) break;
-                ok = gwait(&k_full[g % NK], (uint32_t)(g / NK) & 1u, abort_flag);
+                ok = iwait(&k_full[g % NK], (uint32_t)(g / NK) & 1u, abort_flag);
                 if (ok && g >= kGSB)   // S buffer g % kGSB, read by the softmax of tile g - kGSB
-                    ok = gwait(&p_full[g % kGSB], ((uint32_t)(g / kGSB) & 1u) ^ 1u, abort_flag);
+                    ok = iwait(&p_full[g % kGSB], ((uint32_t)(g / kGSB) & 1u) ^ 1u, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t dt = tmem + (uint32_t)((g % kGSB) * HQP);
@@ -492,7 +511,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
             }
             tc_commit(&drain[0]);
             volatile int no_abort = 0;
-            gwait(&drain[0], 0, &no_abort);
+            iwait(&drain[0], 0, &no_abort);
         }
         __syncwarp();
     } else if (warp == kWarpPV) {
@@ -502,17 +521,17 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
             const uint64_t v_d = desc_mn128(smem_u32(sm + C::kOffV), C::kHalf);
             const uint64_t p_d = smem_desc(smem_u32(sm + C::kOffP), 1024, 2);
             for (int g = 0;; ++g) {
-                bool ok = gwait(&ti_full[g % kGInfo], (uint32_t)(g / kGInfo) & 1u, abort_flag);
+                bool ok = iwait(&ti_full[g % kGInfo], (uint32_t)(g / kGInfo) & 1u, abort_flag);
                 if (!ok) break;
                 const TileHdr h = ti[g % kGInfo];
                 if (h.end) break;
                 mbar_arrive(&ti_empty[g % kGInfo]);   // every reader of the record is done with it
                 // P(g) written, V(g) landed and, for a query's first tile, its O
                 // buffer read by the epilogue of query j - 2
-                ok = gwait(&p_full[g % kGSB], (uint32_t)(g / kGSB) & 1u, abort_flag) &&
-                     gwait(&v_full[g % NV], (uint32_t)(g / NV) & 1u, abort_flag);
+                ok = iwait(&p_full[g % kGSB], (uint32_t)(g / kGSB) & 1u, abort_flag) &&
+                     iwait(&v_full[g % NV], (uint32_t)(g / NV) & 1u, abort_flag);
                 if (ok && h.i == 0 && h.j >= 2)
-                    ok = gwait(&o_empty[h.j & 1], ((uint32_t)(h.j >> 1) & 1u) ^ 1u, abort_flag);
+                    ok = iwait(&o_empty[h.j & 1], ((uint32_t)(h.j >> 1) & 1u) ^ 1u, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t dt = tmem + (uint32_t)((kGSB + (h.j & 1)) * HQP);
@@ -529,7 +548,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
             }
             tc_commit(&drain[1]);
             volatile int no_abort = 0;
-            gwait(&drain[1], 0, &no_abort);
+            iwait(&drain[1], 0, &no_abort);
         }
         __syncwarp();
     } else {

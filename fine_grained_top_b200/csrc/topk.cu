@@ -28,7 +28,7 @@
 
 namespace sa {
 
-constexpr int kTopkThreads = 512;
+constexpr int kTopkThreads = 256;
 constexpr int kTopkWarps = kTopkThreads / 32;
 #ifndef SA_TOPK_CHUNK
 #define SA_TOPK_CHUNK 8192
