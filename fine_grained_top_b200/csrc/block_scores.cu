@@ -154,9 +154,10 @@ __global__ void __launch_bounds__(kInvThreads) invert_scatter_kernel(const int32
     (void)dev_status;
 }
 
-// Pass 4: scores.  A persistent CTA takes blocks b = blockIdx.x + k*gridDim.x;
-// for each it loads the block's keys once and runs over its query groups with
-// the next group's gather in flight while the current one is multiplied.
+// Pass 4: scores.  A persistent CTA takes an equal range of the pairs; for
+// each block in it, it loads the block's keys once and runs over its query
+// groups with the next group's gather in flight while the current one is
+// multiplied.
 template <int D_I, int H_I>
 __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(const uint16_t *qI, const uint16_t *w,
                                                                      const uint16_t *kI, int T, int S, int nb,
@@ -197,8 +198,8 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(const uint1
         return (D_I == 64) ? (uint32_t)(r * ROWB + ((c ^ (r & 7)) << 4))
                            : (uint32_t)(r * ROWB + ((c ^ ((r >> 1) & 3)) << 4));
     };
-    auto gather_queries = [&](int b, int g, int buf) {
-        const int lo = ws.off[b] + g * QG, hi = ws.off[b + 1];
+    // the QG pairs of list entries [lo, min(lo + QG, hi)) into buffer buf
+    auto gather_queries = [&](int lo, int hi, int buf) {
         if (tid < QG) s_entry[buf][tid] = (lo + tid < hi) ? ws.list[lo + tid] : 0xffffffffu;
         for (int idx = tid; idx < 128 * CH; idx += kScoreThreads) {
             const int r = idx / CH, c = idx % CH;
@@ -213,11 +214,28 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(const uint1
         }
     };
 
+    // This CTA's share: an equal contiguous range [p0, p1) of the (query,
+    // slot) pairs of all blocks (the lists are grouped by block, and early
+    // blocks are kept by many more queries than late ones, so whole blocks
+    // per CTA would leave a few CTAs with most of the work).
+    const int total = ws.off[nb];
+    const int per = (total + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int p0 = min(total, (int)blockIdx.x * per), p1 = min(total, p0 + per);
+    int b0 = 0;   // the block whose list holds pair p0: the last b with off[b] <= p0
+    {
+        int hi_b = nb;
+        while (hi_b - b0 > 1) {
+            const int mid = (b0 + hi_b) >> 1;
+            if (ws.off[mid] <= p0) b0 = mid;
+            else hi_b = mid;
+        }
+    }
     uint32_t phase = 0;
-    for (int b = blockIdx.x; b < nb; b += gridDim.x) {
-        const int n_pairs = ws.off[b + 1] - ws.off[b];
-        if (n_pairs <= 0) continue;
-        const int groups = (n_pairs + QG - 1) / QG;
+    for (int b = b0; b < nb && p0 < p1; ++b) {
+        const int r0 = max(ws.off[b], p0), r1 = min(ws.off[b + 1], p1);
+        if (r0 >= p1) break;
+        if (r1 <= r0) continue;
+        const int groups = (r1 - r0 + QG - 1) / QG;
         __syncthreads();   // the previous block's MMAs and epilogues are done with sB / sA
         for (int idx = tid; idx < kBlk * CH; idx += kScoreThreads) {
             const int r = idx / CH, c = idx % CH;
@@ -226,11 +244,11 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(const uint1
             if (s < S) cp_async16(dst, kI + (int64_t)s * D_I + c * 8);
             else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
         }
-        gather_queries(b, 0, 0);
+        gather_queries(r0, r1, 0);
         cp_async_commit();
         for (int g = 0; g < groups; ++g) {
             const int buf = g & 1;
-            if (g + 1 < groups) gather_queries(b, g + 1, buf ^ 1);
+            if (g + 1 < groups) gather_queries(r0 + (g + 1) * QG, r1, buf ^ 1);
             cp_async_commit();
             cp_async_wait<1>();
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // cp.async writes -> tensor core reads

@@ -394,10 +394,12 @@ __global__ void __launch_bounds__(kRowsThreads) topk_rows_kernel(TopkArgs a) {
     auto group_sync = [&]() {
         if (W > 1) asm volatile("bar.sync %0, %1;" ::"r"(1 + grp), "r"(GT) : "memory");
     };
-    // sum of v over the group; `round` alternates the exchange buffer, so one
-    // barrier per sum suffices
+    // sum of v over the group (a shuffle butterfly: the warp reduction
+    // instruction runs on a slower pipe); `round` alternates the exchange
+    // buffer, so one barrier per sum suffices
     auto group_sum = [&](uint32_t v, int round) -> uint32_t {
-        v = __reduce_add_sync(0xffffffffu, v);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
         if (W == 1) return v;
         if (lane == 0) red[grp][round & 1][wg] = v;
         group_sync();
@@ -478,15 +480,41 @@ __global__ void __launch_bounds__(kRowsThreads) topk_rows_kernel(TopkArgs a) {
             key[e] = col < n ? order_key(__ldg(row + col)) : 0u;   // 0 ranks below every score
         }
     }
-    // tau = the largest value with at least K keys >= tau
+    // Bits on which every valid key agrees need no count: tau takes them from
+    // the keys (integer-valued or short-mantissa scores leave most low bits
+    // constant).  OR and AND over the row's valid keys:
+    uint32_t kor = 0u, kand = 0xffffffffu;
+#pragma unroll
+    for (int e = 0; e < PER; ++e)
+        if (c_lo + e < n) { kor |= key[e]; kand &= key[e]; }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        kor |= __shfl_xor_sync(0xffffffffu, kor, o);
+        kand &= __shfl_xor_sync(0xffffffffu, kand, o);
+    }
+    if (W > 1) {
+        if (lane == 0) { red[grp][0][wg] = kor; red[grp][1][wg] = kand; }
+        group_sync();
+        kor = 0u; kand = 0xffffffffu;
+#pragma unroll
+        for (int w = 0; w < W; ++w) { kor |= red[grp][0][w]; kand &= red[grp][1][w]; }
+        group_sync();   // the buffers are reused by the counts below
+    }
+    const uint32_t varying = kor ^ kand;
+    // tau = the largest value with at least K keys >= tau, bit by bit from the top
     uint32_t tau = 0u;
+    int round = 0;
 #pragma unroll 1
     for (int bit = 31; bit >= 0; --bit) {
+        if (!((varying >> bit) & 1u)) {
+            tau |= kand & (1u << bit);
+            continue;
+        }
         const uint32_t c = tau | (1u << bit);
         uint32_t cnt = 0;
 #pragma unroll
         for (int e = 0; e < PER; ++e) cnt += key[e] >= c ? 1u : 0u;
-        if (group_sum(cnt, bit) >= (uint32_t)a.K) tau = c;
+        if (group_sum(cnt, round++) >= (uint32_t)a.K) tau = c;
     }
     uint32_t gt = 0, eq = 0;
 #pragma unroll
