@@ -57,9 +57,16 @@ def load_peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, src="fallback")
 
 
+# Random 256-byte rows gathered from an L2-resident 32 MB K/V set into shared
+# memory with 16-byte cp.async on one B200 (gather_ceiling.cu at the repository
+# root; summary in profiles/gather_ceiling_l2.md): the rate a per-query gather
+# of selected K and V rows cannot beat.
+GATHER_CEILING_GBS = 20018.0
+
+
 # --------------------------------------------------------------------------- ncu traffic
 STAGE_SOURCE = {"indexer": "indexer.cu", "coarse_indexer": "indexer.cu", "topk": "topk.cu",
-                "coarse_topk": "topk.cu", "fine_topk": "topk.cu", "attention": "attention.cu+attention_tc.cu",
+                "coarse_topk": "topk.cu", "fine_topk": "topk.cu", "attention": "attention.cu+attention_tc.cu+attention_gather.cu",
                 "fine_indexer": "block_scores.cu", "pool": "two_stage.cu",
                 "block_counts": "two_stage.cu"}
 
@@ -172,7 +179,7 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- workloads
-def make_case(name, seed, device, index_fp8=False):
+def make_case(name, seed, device, index_fp8=False, rows=None):
     """Device-resident inputs, pinned host copies and a plan for one workload.
     index_fp8: the indexer operands qI and kI are quantised to e4m3 once, on
     the device, before any timing (keys enter an FP8 index cache when they
@@ -184,6 +191,11 @@ def make_case(name, seed, device, index_fp8=False):
     from workloads import CONFIGS, gen_decode, gen_prefill
 
     cfg = dict(CONFIGS[name])
+    if rows is not None:
+        # a chunk of the prompt: the last `rows` queries over the whole sequence's keys
+        if cfg["kind"] == "decode" or not 0 < rows <= cfg["N"]:
+            raise SystemExit("--rows takes 1..N query rows of a prefill workload")
+        cfg["rows"] = int(rows)
     if index_fp8 and cfg["kind"] == "two_stage":
         raise SystemExit("--index-fp8 serves the single-stage prefill and the decode workloads")
     inp = gen_prefill(seed=seed, **cfg) if cfg["kind"] != "decode" else gen_decode(seed=seed, **cfg)
@@ -195,7 +207,9 @@ def make_case(name, seed, device, index_fp8=False):
             t = torch.from_numpy(np.ascontiguousarray(x))
         return t.pin_memory()
 
-    hosts = {k: host(v) for k, v in inp.items() if isinstance(v, np.ndarray)}
+    T = cfg.get("rows", cfg.get("N"))
+    rows_only = ("q", "qI", "w") if cfg["kind"] != "decode" else ()
+    hosts = {k: host(v[len(v) - T:] if k in rows_only else v) for k, v in inp.items() if isinstance(v, np.ndarray)}
     devs = {k: v.to(device) for k, v in hosts.items()}
     if index_fp8:
         for k in ("qI", "kI"):
@@ -217,11 +231,11 @@ def make_case(name, seed, device, index_fp8=False):
         step_inputs = ["q", "qI", "w", "lengths"]
         units = B
     else:
-        make_plan = lambda: PrefillPlan(cfg["N"], cfg["Hq"], cfg["d"], cfg["H_I"], cfg["D_I"], cfg["K"], cfg["W"],
+        make_plan = lambda: PrefillPlan(T, cfg["Hq"], cfg["d"], cfg["H_I"], cfg["D_I"], cfg["K"], cfg["W"],
                                         block=cfg.get("block"), keep=cfg.get("keep"), index_fp8=index_fp8,
-                                        device=device)
+                                        device=device, S=cfg["N"])
         step_inputs = ["q", "k", "v", "qI", "w", "kI"]
-        units = cfg["N"]
+        units = T
     plan = make_plan()
     return dict(cfg=cfg, inp=inp, hosts=hosts, devs=devs, plan=plan, make_plan=make_plan,
                 stages=plan.stages(devs), units=units, step_inputs=step_inputs, index_fp8=index_fp8)
@@ -238,7 +252,8 @@ def stage_work(case):
         pos, rows, pairs = lengths - 1, len(lengths), int(lengths.sum())
     else:
         N = cfg["N"]
-        pos, rows, pairs = np.arange(N, dtype=np.int64), N, N * (N + 1) // 2
+        pos = np.arange(N - cfg.get("rows", N), N, dtype=np.int64)   # query positions (the last rows)
+        rows, pairs = len(pos), int((pos + 1).sum())
     n_sel = ((topk >= 0) & (topk <= (pos - W)[:, None])).sum(1) + np.minimum(W, pos + 1)
     sum_sel = int(n_sel.sum())
     eb = 1 if case.get("index_fp8") else 2   # bytes per qI / kI element
@@ -255,7 +270,8 @@ def stage_work(case):
     else:
         N = cfg["N"]
         kv_b = 2 * N * d * 2
-        st["attention"] = dict(bytes=2 * q_b + kv_b + idx_b, flops=4.0 * Hq * d * sum_sel, bound="tensor")
+        st["attention"] = dict(bytes=2 * q_b + kv_b + idx_b, flops=4.0 * Hq * d * sum_sel, bound="tensor",
+                               gathered=sum_sel * d * 2 * 2)
         if cfg["kind"] == "prefill":
             st["indexer"] = dict(bytes=qI_b + w_b + N * D * eb + 4 * pairs, flops=2.0 * pairs * H * D,
                                  bound="hbm")
@@ -263,8 +279,9 @@ def stage_work(case):
         else:
             blk, keep = cfg["block"], cfg["keep"]
             nb = N // blk
-            cpairs = int(sum(t // blk for t in range(N)))
-            t = np.arange(N, dtype=np.int64)   # candidates: min(keep, t // blk) kept blocks + own block up to t
+            t = pos
+            cpairs = int((t // blk).sum())
+            # candidates: min(keep, t // blk) kept blocks + own block up to t
             fpairs = int((np.minimum(keep, t // blk) * blk + t % blk + 1).sum())
             work.update(coarse_pairs=cpairs, fine_pairs=fpairs)
             st["pool"] = dict(bytes=N * D * 2 + nb * D * 2, flops=float(N * D), bound="hbm")
@@ -301,16 +318,17 @@ def oracle_sample(case, n):
         oracle.decode(inp, cfg["K"], cfg["W"], seqs=range(n))
         desc = "%d of %d sequences, all stages" % (n, cfg["B"])
     else:
-        rows = np.linspace(0, cfg["N"] - 1, n).astype(np.int64)
+        T = cfg.get("rows", cfg["N"])
+        rows = np.linspace(cfg["N"] - T, cfg["N"] - 1, n).astype(np.int64)
         oracle.prefill(inp, cfg["K"], cfg["W"], rows=rows, block=cfg.get("block"), keep=cfg.get("keep"))
-        desc = "%d evenly spaced query rows of %d, all stages" % (n, cfg["N"])
+        desc = "%d evenly spaced query rows of the last %d of %d, all stages" % (n, T, cfg["N"])
     return time.perf_counter() - t0, desc
 
 
 def oracle_calibrate(case, budget_s):
     """Smallest power-of-4 sample (from 16 rows / 1 sequence) that takes about budget_s / 4 or more."""
     cfg = case["cfg"]
-    total = cfg["B"] if cfg["kind"] == "decode" else cfg["N"]
+    total = cfg["B"] if cfg["kind"] == "decode" else cfg.get("rows", cfg["N"])
     n = 1 if cfg["kind"] == "decode" else 16
     while True:
         el, _ = oracle_sample(case, n)
@@ -333,7 +351,7 @@ def run_ours(args, rank, world, local_rank):
     device = "cuda:%d" % local_rank
     torch.cuda.set_device(local_rank)
     peaks = load_peaks()
-    case = make_case(args.workload, seed=rank, device=device, index_fp8=args.index_fp8)
+    case = make_case(args.workload, seed=rank, device=device, index_fp8=args.index_fp8, rows=args.rows)
     stream = torch.cuda.current_stream()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
     plan, d = case["plan"], case["devs"]
@@ -438,12 +456,18 @@ def run_ours(args, rank, world, local_rank):
         stages[name] = dict(ms=round(sec * 1e3, 4),
                             share=round(float(np.sum(times)) / max(1e-9, float(np.sum(staged_ms))), 4),
                             **roofline_entry(w["bound"], w["bytes"], w["flops"], sec, peaks))
+        if "gathered" in w:
+            # K and V rows of the selection, read from L2 into shared memory,
+            # against the measured random-row gather rate
+            ach = w["gathered"] / sec / 1e9
+            stages[name]["gather"] = {"achieved": round(ach, 1), "peak": GATHER_CEILING_GBS, "unit": "GB/s",
+                                      "frac": round(ach / GATHER_CEILING_GBS, 4), "bytes": int(w["gathered"])}
     dom = max(stages, key=lambda n: stages[n]["ms"])
     roof = {k: v for k, v in stages[dom].items() if k not in ("ms", "share")}
     w = work["stages"][dom]
     roof["kernel"] = dom
     roof["algorithmic"] = w["flops"] if roof["bound"] == "tensor" else w["bytes"]
-    tag = args.workload + ("+fp8-indexer" if args.index_fp8 else "")
+    tag = args.workload + ("+rows%d" % args.rows if args.rows else "") + ("+fp8-indexer" if args.index_fp8 else "")
     roof["traffic"] = ncu_traffic(tag, dom)   # per launch, from a capture of this exact source
     roof["peak_src"] = peaks["src"] + " (burst figure; kernel timed alone per step)"
     line = {
@@ -479,7 +503,9 @@ def run_reference(args, rank, world):
         return None
     import oracle
     from workloads import CONFIGS, config_inputs
-    cfg = CONFIGS[args.workload]
+    cfg = dict(CONFIGS[args.workload])
+    if args.rows:
+        cfg["rows"] = int(args.rows)
     case = {"cfg": cfg, "inp": config_inputs(args.workload, seed=0)}
     n, _ = oracle_calibrate(case, budget_s=4.0)          # also the first warm-up step
     for _ in range(max(0, args.warmup - 1)):
@@ -507,6 +533,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="prefill_64k_two_stage")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--rows", type=int, default=None,
+                    help="prefill workloads: time the last ROWS query rows of the sequence (a chunk of the prompt)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--index-fp8", action="store_true",
                     help="indexer on e4m3 operands (single-stage prefill and decode workloads)")

@@ -18,7 +18,7 @@
 //   S^T = K Q^T         M = 128 keys, N = heads, K = d        -> TMEM
 //   P^T = softmax over keys of S^T (per head; one thread per key lane)
 //   O^T += V^T P^T      M = d (V as an MN-major operand), N = heads,
-//                       K = 128 keys (P^T from shared memory) -> TMEM
+//                       K = 128 keys (P^T, MN-major, from shared memory) -> TMEM
 // The running maximum of a head is raised only when a tile exceeds it by more
 // than 2^8 (then O^T and the row sums are rescaled), so P stays below 256.
 //
@@ -57,7 +57,7 @@ constexpr int kGThreads = 15 * 32;
 constexpr int kWarpS = 12, kWarpBuild = 13, kWarpPV = 14;
 constexpr int kGRing = 6;                    // row-index tiles the builder runs ahead
 constexpr int kGMaxK = 2048;                 // top-K entries held in shared memory per query
-constexpr int kGInfo = 8;                    // tile records in flight (K issue .. P V done)
+constexpr int kGInfo = 16;                   // tile records in flight (built .. read by the P V issuer)
 constexpr int kGSB = 4;                      // S^T buffers in TMEM
 constexpr int kGPB = 3;                      // P^T buffers in shared memory
 constexpr size_t kGSmemLimit = 232448;
@@ -123,11 +123,6 @@ struct GCfg {
 };
 
 // ------------------------------------------------------------------ PTX helpers
-__device__ __forceinline__ void cp_async16_zfill(void *smem_dst, const void *gsrc, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
-                 "r"(src_bytes)
-                 : "memory");
-}
 // Arrive on `bar` once every cp.async this thread issued so far has landed
 // (the arrival counts against the barrier's expected count).
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
@@ -226,6 +221,20 @@ __device__ __forceinline__ uint64_t desc_mn128(uint32_t addr, uint32_t lbo) {
     return d;
 }
 
+// MN-major operand without swizzle: 8 x 16-byte core matrices (8 K rows of 8
+// MN elements, 128 contiguous bytes); K groups of 8 rows `kgroup` bytes apart,
+// MN chunks of 8 elements `mnchunk` bytes apart.  (For this layout the
+// descriptor's leading offset is the K-group stride and its stride offset the
+// MN-chunk stride.)
+__device__ __forceinline__ uint64_t desc_mn_plain(uint32_t addr, uint32_t kgroup, uint32_t mnchunk) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFF);
+    d |= (uint64_t)((kgroup >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)((mnchunk >> 4) & 0x3FFF) << 32;
+    d |= (uint64_t)1 << 46;   // layout type 0 (no swizzle) in bits 61-63
+    return d;
+}
+
 // Byte offset of 16-byte chunk `ch` (0..15) of row `r` in a 128B-swizzled
 // tile of 256-byte rows held as two 64-column halves `half` bytes apart.
 __device__ __forceinline__ uint32_t sw_off(int r, int ch, int half) {
@@ -262,7 +271,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NK; ++i) {
-            mbar_init(&k_full[i], 64 + 1);     // 64 cp.async arrivals + the record writer
+            mbar_init(&k_full[i], 64);         // 64 cp.async arrivals
             mbar_init(&k_empty[i], 1);
         }
         for (int i = 0; i < NV; ++i) {
@@ -374,33 +383,56 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
                 ok = __all_sync(0xffffffffu, gwait(&row_empty[slot], ((uint32_t)(g / kGRing) & 1u) ^ 1u,
                                                        abort_flag));
                 if (!ok) break;
+                // Byte offsets of the tile's 128 rows, in the order the gather
+                // lanes read them: key kk = 64 pw + 2 it + sub sits at 64 pw +
+                // 32 sub + it.  A slot past the selection repeats the tile's
+                // first row: its score is masked to -inf, so its P is exactly 0.
                 int32_t *rr = rows + slot * kGTile;
+                int first_row = 0;
 #pragma unroll
                 for (int u = 0; u < kGTile / 32; ++u) {
                     const int kk = i * kGTile + u * 32 + lane;
-                    const int row = kk < n_top ? list[kk] : (kk < n_keys ? w0 + (kk - n_top) : -1);
-                    rr[u * 32 + lane] = row >= 0 ? (int32_t)((uint32_t)row * (uint32_t)(D * 2)) : -1;
+                    int row = kk < n_top ? list[kk] : (kk < n_keys ? w0 + (kk - n_top) : -1);
+                    if (u == 0) first_row = __shfl_sync(0xffffffffu, row, 0);
+                    if (row < 0) row = first_row;
+                    rr[(u >> 1) * 64 + (lane & 1) * 32 + (u & 1) * 16 + (lane >> 1)] =
+                        (int32_t)((uint32_t)row * (uint32_t)(D * 2));
                 }
+                // the tile's record for the gather warps, and for the MMA and
+                // softmax warps (once the P V issuer has read the record of tile
+                // g - kGInfo from the slot)
+                if (g >= kGInfo)
+                    ok = __all_sync(0xffffffffu, gwait(&ti_empty[g % kGInfo], ((uint32_t)(g / kGInfo) & 1u) ^ 1u,
+                                                       abort_flag));
+                if (!ok) break;
                 if (lane == 0) {
                     TileHdr h;
                     h.end = 0; h.t = t; h.j = j; h.i = i;
                     h.nvalid = min(kGTile, n_keys - i * kGTile);
                     h.last = (i == n_tiles - 1); h.p = p; h.pad = 0;
                     rhdr[slot] = h;
+                    ti[g % kGInfo] = h;
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&row_full[slot]);
+                if (lane == 0) {
+                    mbar_arrive(&row_full[slot]);
+                    mbar_arrive(&ti_full[g % kGInfo]);
+                }
             }
             __syncwarp();   // the list is rewritten for the next query
         }
         if (ok) {   // end marker
             const int slot = g % kGRing;
             ok = __all_sync(0xffffffffu, gwait(&row_empty[slot], ((uint32_t)(g / kGRing) & 1u) ^ 1u, abort_flag));
+            if (ok && g >= kGInfo)
+                ok = __all_sync(0xffffffffu, gwait(&ti_empty[g % kGInfo], ((uint32_t)(g / kGInfo) & 1u) ^ 1u, abort_flag));
             if (ok && lane == 0) {
                 TileHdr h = {};
                 h.end = 1;
                 rhdr[slot] = h;
+                ti[g % kGInfo] = h;
                 mbar_arrive(&row_full[slot]);
+                mbar_arrive(&ti_full[g % kGInfo]);
             }
         }
         __syncwarp();
@@ -440,36 +472,23 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
                     if (!ok) break;
                     dst = sm + C::kOffV + (g % NV) * C::kKV;
                 }
-                // this warp's 64 keys: byte offsets first, then the copies (a key
-                // past the selection is zero-filled: source size 0)
-                const uint32_t *rr = reinterpret_cast<const uint32_t *>(rows + slot * kGTile) + pw * 64;
+                // this warp's 64 keys (key 64 pw + 2 it + sub for lane half sub):
+                // the byte offsets as eight 16-byte loads, then the copies
+                const uint4 *rr = reinterpret_cast<const uint4 *>(rows + slot * kGTile + pw * 64 + sub * 32);
                 uint32_t ro[32];
 #pragma unroll
-                for (int it = 0; it < 32; ++it) ro[it] = rr[2 * it + sub];
+                for (int q = 0; q < 8; ++q) {
+                    const uint4 o = rr[q];
+                    ro[4 * q] = o.x; ro[4 * q + 1] = o.y; ro[4 * q + 2] = o.z; ro[4 * q + 3] = o.w;
+                }
 #pragma unroll
                 for (int it = 0; it < 32; ++it) {
                     const int key = pw * 64 + 2 * it + sub;
-                    const bool valid = ro[it] != 0xffffffffu;
-                    cp_async16_zfill(dst + sw_off(key, ch, C::kHalf), base + (valid ? ro[it] : 0u), valid ? 16u : 0u);
+                    cp_async16(dst + sw_off(key, ch, C::kHalf), base + ro[it]);
                 }
             }
             if (kside) {
-                // the tile's record, once the P V issuer has read the record of
-                // tile g - kGInfo from the slot; then K(g) complete
-                if (t64 == 0) {
-                    if (g >= kGInfo)
-                        ok = gwait(&ti_empty[g % kGInfo], ((uint32_t)(g / kGInfo) & 1u) ^ 1u, abort_flag);
-                    if (ok) {
-                        ti[g % kGInfo] = h;
-                        mbar_arrive(&ti_full[g % kGInfo]);
-                    }
-                }
-                ok = __shfl_sync(0xffffffffu, ok, 0);   // lane 0 of warp 0 waited: its warp follows its result
-                if (!ok) break;
-                if (!h.end) {
-                    cp_async_arrive_noinc(&k_full[g % NK]);
-                    if (t64 == 0) mbar_arrive(&k_full[g % NK]);
-                }
+                if (!h.end) cp_async_arrive_noinc(&k_full[g % NK]);
             } else if (!h.end) {
                 cp_async_arrive_noinc(&v_full[g % NV]);
             }
@@ -485,8 +504,8 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
             const uint64_t k_d = smem_desc(smem_u32(sm + C::kOffK), 1024, 2);
             const uint64_t q_d = smem_desc(smem_u32(sm + C::kOffQ), 1024, 2);
             for (int g = 0;; ++g) {
-                // the tile's record and K(g) (the record is written before K's
-                // completion), and S buffer g % 2 read by the softmax of tile g - 2
+                // the tile's record, K(g), and S buffer g % kGSB read by the
+                // softmax of tile g - kGSB
                 bool ok = iwait(&ti_full[g % kGInfo], (uint32_t)(g / kGInfo) & 1u, abort_flag);
                 if (!ok) break;
                 const TileHdr h = ti[g % kGInfo];
@@ -517,9 +536,10 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
     } else if (warp == kWarpPV) {
         // ------------------------------------------------------------ P V issuer
         if (lane == 0) {
-            constexpr uint32_t idesc_o = idesc_bf16_f32(128, HQP) | (1u << 15);   // A (V^T) MN-major
+            // A (V^T) and B (P^T) both MN-major
+            constexpr uint32_t idesc_o = idesc_bf16_f32(128, HQP) | (1u << 15) | (1u << 16);
             const uint64_t v_d = desc_mn128(smem_u32(sm + C::kOffV), C::kHalf);
-            const uint64_t p_d = smem_desc(smem_u32(sm + C::kOffP), 1024, 2);
+            const uint64_t p_d = desc_mn_plain(smem_u32(sm + C::kOffP), HQP * 16, 128);
             for (int g = 0;; ++g) {
                 bool ok = iwait(&ti_full[g % kGInfo], (uint32_t)(g / kGInfo) & 1u, abort_flag);
                 if (!ok) break;
@@ -539,7 +559,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
                 const uint64_t pd = p_d + (uint64_t)(((g % kGPB) * C::kP) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < kGTile / 16; ++kk) {
-                    const uint64_t pa = (uint64_t)(((kk >> 2) * C::kQHalf + (kk & 3) * 32) >> 4);
+                    const uint64_t pa = (uint64_t)((kk * 2 * HQP * 16) >> 4);   // 16 keys = two key groups
                     mma_acc(dt, vd + (uint64_t)((kk * 2048) >> 4), pd + pa, idesc_o, (h.i == 0 && kk == 0) ? 0u : 1u);
                 }
                 tc_commit(&p_empty[g % kGPB]);
@@ -573,9 +593,11 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
                 for (int e = 0; e < 8; ++e) v[c + e] = __uint_as_float(u[e]);
             }
         };
-        // The epilogue of a query (O^T / l -> out, lse) runs one tile later, so
-        // that the softmax does not wait for the query's last P V.
-        int pend_j = -1, pend_t = 0;
+        // The epilogue of a query (O^T / l -> out, lse) runs kGPB tiles after
+        // its last one, when that tile's P V is known to be done (the P buffer
+        // wait of the current tile covers it), or earlier at the next query's
+        // last tile (one pending query at a time) or at the end.
+        int pend_j = -1, pend_t = 0, pend_g = 0;
         auto epilogue = [&]() -> bool {
             if (pend_j < 0) return true;
             const int jb = pend_j & 1;
@@ -616,29 +638,44 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
                 if (!h.end && w && g >= kGPB)
                     w = gwait(&p_empty[pb_i], ((uint32_t)(g / kGPB) & 1u) ^ 1u, abort_flag);
             }
-            ok = bar_and(bar_red, 128, w);
-            if (!ok) break;
-            if (h.end) {
-                ok = epilogue();
-                break;
-            }
+            // One vote per tile decides the common case: nobody stopped (a
+            // wait that ran out, or the end marker) and no head needs a new
+            // maximum.  (After a failed wait the S^T read below returns
+            // whatever TMEM holds; the vote discards it.)
+            const bool stop = !w || h.end;
             tc_fence_after();
             float x[HG];
             tload((uint32_t)(sb * HQP), x);
-            const bool valid = key < h.nvalid;
+            if (key >= h.nvalid) {   // a lane past the selection (a query's last tile)
 #pragma unroll
-            for (int hh = 0; hh < HG; ++hh) x[hh] = valid ? x[hh] * sl2 : -CUDART_INF_F;
-            // Is any score of this tile more than 2^8 above its head's running
-            // maximum?  (Always at a query's first tile, where the maximum is set.)
-            bool need = h.i == 0;
+                for (int hh = 0; hh < HG; ++hh) x[hh] = -CUDART_INF_F;
+            }
+            // e[h] = log2 of P before rounding: the scaled score less the
+            // head's running maximum.  Is any more than 8 (P above 2^8)?
+            // (Always decided anew at a query's first tile, where the maximum is set.)
+            float e[HG];
+            float emax = -CUDART_INF_F;
 #pragma unroll
-            for (int hh = 0; hh < HG; ++hh) need |= x[hh] > m[hh] + 8.f;
-            if (bar_or(bar_red, 128, need)) {
+            for (int hh = 0; hh < HG; ++hh) {
+                e[hh] = fmaf(x[hh], sl2, -m[hh]);
+                emax = fmaxf(emax, e[hh]);
+            }
+            bool need = h.i == 0 || emax > 8.f;
+            if (!bar_or(bar_red, 128, need || stop)) {
+                need = false;
+            } else if (bar_or(bar_red, 128, stop)) {
+                ok = bar_and(bar_red, 128, w);   // every wait succeeded: the end marker for all
+                if (ok) ok = epilogue();
+                break;
+            } else {
+                need = true;
+            }
+            if (need) {
                 // exact tile maximum of every head over the 128 key lanes:
                 // butterfly within each warp, then across the group's four warps
 #pragma unroll
                 for (int hh = 0; hh < HG; ++hh) {
-                    float v = x[hh];
+                    float v = x[hh] * sl2;
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
                     if (lane == 0) gmax[quad * HG + hh] = v;
@@ -678,24 +715,35 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
                     }
                     tmem_st_wait_all();
                 }
-            }
-            // P^T (heads x keys, K-major SW128): key = this lane, heads h0 ..
-            uint8_t *pbuf = sm + C::kOffP + pb_i * C::kP + (key >> 6) * C::kQHalf;
-            const int kc = key & 63;
 #pragma unroll
-            for (int hh = 0; hh < HG; ++hh) {
-                const int row = h0 + hh;
-                const float pv = ex2f(x[hh] - m[hh]);
-                l[hh] += pv;
-                const __nv_bfloat16 bv = __float2bfloat16_rn(pv);
-                *reinterpret_cast<__nv_bfloat16 *>(pbuf + row * 128 + ((((kc >> 3) ^ (row & 7)) << 4) | ((kc & 7) << 1))) = bv;
+                for (int hh = 0; hh < HG; ++hh) e[hh] = fmaf(x[hh], sl2, -m[hh]);
+            }
+            // P^T as an MN-major operand without swizzle: 16-byte rows of 8
+            // heads, the rows of 8 keys 16 bytes apart, the head chunks of a
+            // key group 128 bytes apart, key groups HQP * 16 bytes apart; each
+            // thread (one key) stores its heads h0 .. as whole 16-byte rows
+            uint8_t *pbuf = sm + C::kOffP + pb_i * C::kP + (key >> 3) * (HQP * 16) + (key & 7) * 16;
+#pragma unroll
+            for (int c = 0; c < HG; c += 8) {
+                uint32_t u[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float p0 = ex2f(e[c + 2 * q]);
+                    const float p1 = ex2f(e[c + 2 * q + 1]);
+                    l[c + 2 * q] += p0;
+                    l[c + 2 * q + 1] += p1;
+                    const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);   // p0 in the low half
+                    u[q] = *reinterpret_cast<const uint32_t *>(&b2);
+                }
+                *reinterpret_cast<uint4 *>(pbuf + ((h0 + c) >> 3) * 128) = make_uint4(u[0], u[1], u[2], u[3]);
             }
             fence_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[sb]);
-            // the previous query's epilogue, now that this tile is handed over
-            if (!(ok = epilogue())) break;
+            // a pending epilogue, now that this tile is handed over
+            if (pend_j >= 0 && (g - pend_g >= kGPB || h.last))
+                if (!(ok = epilogue())) break;
             if (h.last) {
                 // the query's row sums over all 128 key lanes and its maxima,
                 // kept for its epilogue
@@ -717,6 +765,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
                 bar_sync_n(bar_x, 128);   // epi_* written before any warp's epilogue reads them
                 pend_j = h.j;
                 pend_t = h.t;
+                pend_g = g;
             }
         }
     }

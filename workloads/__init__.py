@@ -25,7 +25,7 @@ import numpy as np
 
 STREAMS = ("q", "k", "v", "qI", "kI", "w", "lengths", "perm")
 
-# The five workloads, named by what they are.  Shapes follow the pages'
+# The workloads, named by what they are.  Shapes follow the pages'
 # long-context regimes: 8K-128K prefill, 128K-class decode, top-k 2048 and
 # 64-token KV pages.
 CONFIGS = {
@@ -36,6 +36,11 @@ CONFIGS = {
     "decode_8x128k": dict(kind="decode", B=8, L=131072, Hq=64, d=128, H_I=8,
                           D_I=64, K=2048, W=512, paged=False),
     "prefill_64k_two_stage": dict(kind="two_stage", N=65536, Hq=16, d=128,
+                                  H_I=4, D_I=64, block=64, keep=64, K=2048,
+                                  W=512),
+    # the 64K two-stage shapes on a 16K sequence: a case small enough for
+    # multi-pass profiler captures of the same kernels
+    "prefill_16k_two_stage": dict(kind="two_stage", N=16384, Hq=16, d=128,
                                   H_I=4, D_I=64, block=64, keep=64, K=2048,
                                   W=512),
     "decode_paged_16x256k": dict(kind="decode", B=16, L_min=16384,
