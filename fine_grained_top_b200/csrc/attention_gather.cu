@@ -172,7 +172,6 @@ __device__ __forceinline__ bool iwait(uint64_t *bar, uint32_t parity, volatile i
         if (globaltimer() - t0 > kWaitLimitNs) { *abort = 1; return false; }
     }
 }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 // Barrier `id` over `n` threads that also returns the OR / AND of a predicate.
 __device__ __forceinline__ bool bar_or(int id, int n, bool p) {

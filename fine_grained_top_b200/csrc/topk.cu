@@ -9,10 +9,13 @@
 //   * rows of at most 1024 columns: one warp per row, the keys in registers,
 //     a bitwise search for the K-th key (topk_rows_kernel);
 //   * longer rows: one row per thread-block cluster of G = 1..16 CTAs; CTA c of the
-//     cluster owns a contiguous chunk of the row, loaded once from HBM with
-//     16-byte vector loads into shared memory as order-preserving uint32 keys;
-//   * exact radix select over the keys in three passes of 12, 10 and 10 bits.
-//     The first histogram is built while the chunk is loaded; the later
+//     cluster owns a contiguous chunk of the row, copied once from HBM into
+//     shared memory with 16-byte cp.async (issued first, so the copy overlaps
+//     the row's argument checks) and rewritten there as order-preserving
+//     uint32 keys;
+//   * exact radix select over the keys in three passes of 11, 11 and 10 bits
+//     (12, 10 and 10 for a cluster row).
+//     The first histogram is built while the keys are rewritten; the later
 //     passes only count keys that match the prefix chosen so far.  Per-CTA
 //     histograms are summed over the cluster through distributed shared
 //     memory (no global workspace).  When the threshold bin is taken whole,
@@ -23,6 +26,8 @@
 //     span in column order (4 keys per lane per step, both counts packed in
 //     one word), a scan over lanes, warps and the cluster's CTAs gives every
 //     kept key its output slot, so the output comes out ascending.
+#include <algorithm>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -36,7 +41,11 @@ constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kTopkChunkTarget = SA_TOPK_CHUNK;   // columns per CTA before adding CTAs
 constexpr int kTopkMaxChunk = 32768;      // 128 KB of keys per CTA
 constexpr int kTopkMaxCluster = 16;
-constexpr int kBinsA = 4096;              // first pass: top 12 bits
+// First digit: the top 11 bits for a single-CTA row (then 11 and 10), the
+// top 12 bits for a cluster row (then 10 and 10: smaller refinement
+// histograms to sum across the cluster).
+template <int G> constexpr int bits_a() { return G == 1 ? 11 : 12; }
+constexpr int kBinsMax = 4096;
 
 int topk_max_row_len() { return kTopkMaxChunk * kTopkMaxCluster; }
 
@@ -120,7 +129,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     extern __shared__ __align__(16) uint32_t dsm[];
     uint32_t *keys = dsm;
     uint32_t *hist0 = dsm + a.chunk;
-    uint32_t *hsum = (G > 1) ? hist0 + kBinsA : nullptr;
+    constexpr int BA = bits_a<G>(), SA_ = 32 - BA, BINS_A = 1 << BA, BINS_1 = 1 << (SA_ - 10);
+    uint32_t *hsum = (G > 1) ? hist0 + BINS_A : nullptr;
     __shared__ uint32_t scan_tmp[64];
     __shared__ uint32_t sel[3];
     __shared__ uint32_t warp_gt[kTopkWarps];   // packed per-warp counts
@@ -130,6 +140,18 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     const int r = blockIdx.x / G;
     const uint32_t rank = (G > 1) ? cluster_rank() : 0u;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    // Start copying this CTA's chunk of the row into shared memory before
+    // anything waits.  The row's valid length is not known yet, so the copy
+    // runs to the row's allocated length; columns past the valid length are
+    // never read back.
+    const int c0 = (int)rank * a.chunk;
+    const float *row = a.scores + (int64_t)r * a.ld;
+    {
+        const int pre4 = max(0, min(c0 + a.chunk, a.row_len) - c0) >> 2;   // c0 and ld are multiples of 4
+        const float4 *src4 = reinterpret_cast<const float4 *>(row + c0);
+        for (int i = tid; i < pre4; i += kTopkThreads) cp_async16(keys + 4 * i, src4 + i);
+    }
 
     int n;
     int n_kept = 0, own0 = 0;   // block-id candidates: valid kept blocks, first token of the own block
@@ -170,17 +192,19 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
         n = a.row_len - a.rows + r + 1;
         n = n < 0 ? 0 : (n > a.row_len ? a.row_len : n);
     }
-    const int c0 = (int)rank * a.chunk;
     const int c1 = min(c0 + a.chunk, n);
     const int len = max(0, c1 - c0);
     int32_t *out = a.out + (int64_t)r * a.K;
-    const float *row = a.scores + (int64_t)r * a.ld;
     const int32_t *cand = a.cand ? a.cand + (int64_t)r * a.ld_cand : nullptr;
     // position of column col: through the block ids, the position map, or itself
+    // (a power-of-two block size, the usual case, takes shifts instead of divisions)
+    const int bshift = (a.block > 0 && (a.block & (a.block - 1)) == 0) ? __ffs(a.block) - 1 : -1;
     auto pos = [&](int col) -> int32_t {
         if (byb) {
             const int kb = n_kept * a.block;
-            return col < kb ? brow[col / a.block] * a.block + col % a.block : own0 + (col - kb);
+            if (col >= kb) return own0 + (col - kb);
+            if (bshift >= 0) return (brow[col >> bshift] << bshift) + (col & (a.block - 1));
+            return brow[col / a.block] * a.block + col % a.block;
         }
         return cand ? cand[col] : col;
     };
@@ -198,46 +222,41 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
         for (int i = tid; i < len; i += kTopkThreads) out[c0 + i] = pos(c0 + i);
         if (rank == 0)
             for (int i = n + tid; i < a.K; i += kTopkThreads) out[i] = -1;
+        cp_async_wait_all();   // the copies into this CTA's shared memory end before it exits
         return;   // uniform over the cluster: no distributed smem was touched
     }
 
-    // ---- load the chunk as order-preserving keys, counting the top 12 bits
-    for (int i = tid; i < kBinsA / 4; i += kTopkThreads) reinterpret_cast<uint4 *>(hist0)[i] = make_uint4(0u, 0u, 0u, 0u);
+    // ---- the chunk as order-preserving keys, counting the top 11 bits
+    for (int i = tid; i < BINS_A / 4; i += kTopkThreads) reinterpret_cast<uint4 *>(hist0)[i] = make_uint4(0u, 0u, 0u, 0u);
+    cp_async_wait_all();
     __syncthreads();
     {
-        const int len4 = len >> 2;   // c0 and ld are multiples of 4, base 16-byte aligned
-        const float4 *src4 = reinterpret_cast<const float4 *>(row + c0);
-        auto put = [&](int i, const float4 &f) {
+        const int len4 = len >> 2;
+        for (int i = tid; i < len4; i += kTopkThreads) {
+            const uint4 f = reinterpret_cast<const uint4 *>(keys)[i];
             uint4 k;
-            k.x = order_key(f.x); k.y = order_key(f.y);
-            k.z = order_key(f.z); k.w = order_key(f.w);
+            k.x = order_key(__uint_as_float(f.x)); k.y = order_key(__uint_as_float(f.y));
+            k.z = order_key(__uint_as_float(f.z)); k.w = order_key(__uint_as_float(f.w));
             reinterpret_cast<uint4 *>(keys)[i] = k;
-            atomicAdd(&hist0[k.x >> 20], 1u);
-            atomicAdd(&hist0[k.y >> 20], 1u);
-            atomicAdd(&hist0[k.z >> 20], 1u);
-            atomicAdd(&hist0[k.w >> 20], 1u);
-        };
-        int i = tid;
-        for (; i + kTopkThreads < len4; i += 2 * kTopkThreads) {   // two 16-byte loads in flight
-            const float4 f0 = __ldg(src4 + i), f1 = __ldg(src4 + i + kTopkThreads);
-            put(i, f0);
-            put(i + kTopkThreads, f1);
+            atomicAdd(&hist0[k.x >> SA_], 1u);
+            atomicAdd(&hist0[k.y >> SA_], 1u);
+            atomicAdd(&hist0[k.z >> SA_], 1u);
+            atomicAdd(&hist0[k.w >> SA_], 1u);
         }
-        if (i < len4) put(i, __ldg(src4 + i));
-        for (int i = (len4 << 2) + tid; i < len; i += kTopkThreads) {
+        for (int i = (len4 << 2) + tid; i < len; i += kTopkThreads) {   // the last len % 4 columns
             const uint32_t k = order_key(row[c0 + i]);
             keys[i] = k;
-            atomicAdd(&hist0[k >> 20], 1u);
+            atomicAdd(&hist0[k >> SA_], 1u);
         }
     }
     __syncthreads();
 
     uint32_t need = (uint32_t)a.K;      // keys still to take among those matching `prefix`
-    find_threshold<G, kBinsA>(hist0, hsum, need, scan_tmp, sel, tid);
-    uint32_t prefix = sel[0] << 20, mask = 0xFFF00000u;
+    find_threshold<G, BINS_A>(hist0, hsum, need, scan_tmp, sel, tid);
+    uint32_t prefix = sel[0] << SA_, mask = 0xFFFFFFFFu << SA_;
     need -= sel[1];
     bool whole = sel[2] == need;        // the threshold bin is taken entirely
-    // two 10-bit refinements over the keys that match the prefix.  A single-CTA
+    // refinements (11 or 10 bits, then 10) over the keys that match the prefix.  A single-CTA
     // row also takes, in the first, the OR and AND of the last digit (bits
     // 9..0) over those keys: when they agree, every key of the bin shares its
     // last digit and the second refinement is decided without a pass (keys with
@@ -245,15 +264,17 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
 #pragma unroll 1
     for (int pass = 1; pass < 3 && !whole; ++pass) {
         const int shift = pass == 1 ? 10 : 0;
+        const uint32_t dmask = pass == 1 ? (uint32_t)BINS_1 - 1u : 1023u;   // the digit: bits SA_-1..10, then 9..0
         const bool track = G == 1 && pass == 1;
         uint32_t *hl = hist0;
-        if (tid < 256) reinterpret_cast<uint4 *>(hl)[tid] = make_uint4(0u, 0u, 0u, 0u);
+        for (int i = tid; i < (int)(dmask + 1) / 4; i += kTopkThreads)
+            reinterpret_cast<uint4 *>(hl)[i] = make_uint4(0u, 0u, 0u, 0u);
         if (track && tid == 0) { low_bits[0] = 0u; low_bits[1] = 1023u; }
         __syncthreads();
         uint32_t lor = 0u, land = 1023u;
         auto count = [&](uint32_t u) {
             if ((u & mask) == prefix) {
-                atomicAdd(&hl[(u >> shift) & 1023u], 1u);
+                atomicAdd(&hl[(u >> shift) & dmask], 1u);
                 if (track) {
                     lor |= u & 1023u;
                     land &= u & 1023u;
@@ -278,9 +299,12 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
             }
         }
         __syncthreads();
-        find_threshold<G, 1024>(hl, hsum, need, scan_tmp, sel, tid);
+        if (pass == 1)
+            find_threshold<G, BINS_1>(hl, hsum, need, scan_tmp, sel, tid);
+        else
+            find_threshold<G, 1024>(hl, hsum, need, scan_tmp, sel, tid);
         prefix |= sel[0] << shift;
-        mask |= 1023u << shift;
+        mask |= dmask << shift;
         need -= sel[1];
         whole = sel[2] == need;
         if (track && !whole && low_bits[0] == low_bits[1]) {   // the last digit is the same for all
@@ -326,8 +350,9 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
         load4(j + 4 * lane, u);
         const uint32_t f = flags4(j + 4 * lane, u);
         flags[g * 32 + lane] = f;
-        wtot += __reduce_add_sync(0xffffffffu, (uint32_t)__popc(f & 15u) + ((uint32_t)__popc(f >> 4) << 16));
+        wtot += (uint32_t)__popc(f & 15u) + ((uint32_t)__popc(f >> 4) << 16);
     }
+    wtot = __reduce_add_sync(0xffffffffu, wtot);   // this warp's packed counts
     if (lane == 0) warp_gt[warp] = wtot;
     __syncthreads();
     const uint32_t wbase = __reduce_add_sync(0xffffffffu, lane < warp ? warp_gt[lane] : 0u);   // warps before
@@ -446,10 +471,14 @@ __global__ void __launch_bounds__(kRowsThreads) topk_rows_kernel(TopkArgs a) {
     const float *row = a.scores + (int64_t)r * a.ld;
     const int32_t *cand = a.cand ? a.cand + (int64_t)r * a.ld_cand : nullptr;
     // position of column col: through the block ids, the position map, or itself
+    // (a power-of-two block size, the usual case, takes shifts instead of divisions)
+    const int bshift = (a.block > 0 && (a.block & (a.block - 1)) == 0) ? __ffs(a.block) - 1 : -1;
     auto pos = [&](int col) -> int32_t {
         if (byb) {
             const int kb = n_kept * a.block;
-            return col < kb ? brow[col / a.block] * a.block + col % a.block : own0 + (col - kb);
+            if (col >= kb) return own0 + (col - kb);
+            if (bshift >= 0) return (brow[col >> bshift] << bshift) + (col & (a.block - 1));
+            return brow[col / a.block] * a.block + col % a.block;
         }
         return cand ? cand[col] : col;
     };
@@ -597,7 +626,10 @@ sa_status launch_topk(TopkArgs a, cudaStream_t st) {
     chunk = (chunk + 3) & ~3;
     if (chunk > kTopkMaxChunk) return SA_ERR_UNSUPPORTED;
     a.chunk = chunk;
-    const size_t hist_words = (g > 1) ? 2 * kBinsA : kBinsA;
+    // histograms, later reused for the compaction's per-lane flags (one word
+    // per lane and 128-key group of each warp's span)
+    const size_t flag_words = (size_t)kTopkWarps * (((size_t)chunk + 4 * kTopkThreads - 1) / (4 * kTopkThreads)) * 32;
+    const size_t hist_words = std::max((g > 1) ? 2 * (size_t)kBinsMax : (size_t)kBinsMax / 2, flag_words);
     const size_t smem = ((size_t)chunk + hist_words) * 4;
     switch (g) {
         case 1: return launch_topk_g<1>(a, smem, st);
