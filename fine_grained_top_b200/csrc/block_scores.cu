@@ -277,29 +277,42 @@ __global__ void __launch_bounds__(kScoreThreads) block_scores_kernel(const uint1
             phase ^= 1u;
             tc_fence_after();
             float* out = scores + (int64_t)t * ld + slot * kBlk;
+            // w_j ReLU(.) of the 64 keys for this lane's head, then the sum over
+            // the H_I heads (adjacent lanes) as a transposing butterfly: at each
+            // step a lane keeps one half of its values and adds the partner's
+            // copy of that half, so every lane ends with kBlk / H_I finished
+            // sums of consecutive keys (no lane idles in the stores)
+            float sc[kBlk];
 #pragma unroll
             for (int c0 = 0; c0 < kBlk; c0 += 16) {
                 uint32_t v[16];
                 tmem_ld_x16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
                 tmem_ld_wait();
-                float sc[16];
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    float x = wv * fmaxf(__uint_as_float(v[k]), 0.f);
+                for (int k = 0; k < 16; ++k) sc[c0 + k] = wv * fmaxf(__uint_as_float(v[k]), 0.f);
+            }
+            int ko = 0;   // first key of this lane's finished sums
 #pragma unroll
-                    for (int o = 1; o < H_I; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-                    sc[k] = x;
+            for (int o = 1, L = kBlk; o < H_I; o <<= 1, L >>= 1) {
+                const bool upper = (lane & o) != 0;   // keep the upper half of the current L values
+#pragma unroll
+                for (int i = 0; i < L / 2; ++i) {
+                    const float keep = upper ? sc[L / 2 + i] : sc[i];
+                    const float send = upper ? sc[i] : sc[L / 2 + i];
+                    sc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
                 }
-                if (valid && j == 0) {
-                    if (c0 + 15 <= last) {
+                ko += upper ? L / 2 : 0;
+            }
+            constexpr int NF = kBlk / H_I;   // finished sums per lane
+            if (valid) {
+                if (ko + NF - 1 <= last) {
 #pragma unroll
-                        for (int k = 0; k < 16; k += 4)
-                            *reinterpret_cast<float4 *>(out + c0 + k) = make_float4(sc[k], sc[k + 1], sc[k + 2], sc[k + 3]);
-                    } else {
+                    for (int k = 0; k < NF; k += 4)
+                        *reinterpret_cast<float4 *>(out + ko + k) = make_float4(sc[k], sc[k + 1], sc[k + 2], sc[k + 3]);
+                } else {
 #pragma unroll
-                        for (int k = 0; k < 16; ++k)
-                            if (c0 + k <= last) out[c0 + k] = sc[k];
-                    }
+                    for (int k = 0; k < NF; ++k)
+                        if (ko + k <= last) out[ko + k] = sc[k];
                 }
             }
             tc_fence_before();

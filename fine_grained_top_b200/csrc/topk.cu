@@ -33,8 +33,10 @@
 
 namespace sa {
 
-constexpr int kTopkThreads = 256;
-constexpr int kTopkWarps = kTopkThreads / 32;
+// Threads per CTA: 256 for a single-CTA row (rows of at most 8192 columns:
+// more rows resident per SM), 512 for the CTAs of a cluster row (chunks of up
+// to 32768 columns).
+template <int G> constexpr int topk_threads() { return G == 1 ? 256 : 512; }
 #ifndef SA_TOPK_CHUNK
 #define SA_TOPK_CHUNK 8192
 #endif
@@ -54,17 +56,17 @@ int topk_max_row_len() { return kTopkMaxChunk * kTopkMaxCluster; }
 // The cluster sum is a reduce-scatter plus all-gather over distributed shared
 // memory: CTA r adds up bin slice r from every CTA (all G loads in flight at
 // once) and stores the sums into slice r of every CTA's `hsum`.
-template <int G, int BINS>
+template <int G, int BINS, int NT>
 __device__ __forceinline__ void find_threshold(uint32_t *hl, uint32_t *hsum, uint32_t need,
                                                uint32_t *scan_tmp, uint32_t *sel, int tid) {
-    constexpr int PER = BINS / kTopkThreads;   // bins per thread (8 or 2)
+    constexpr int PER = BINS / NT;   // bins per thread
     const int lane = tid & 31, warp = tid >> 5;
     const uint32_t *h = hl;
     if (G > 1) {
         constexpr int SLICE = BINS / G;
         const uint32_t rank = cluster_rank();
         cluster_sync();   // every CTA's histogram is complete
-        for (int i = tid; i < SLICE; i += kTopkThreads) {
+        for (int i = tid; i < SLICE; i += NT) {
             const int bin = (int)rank * SLICE + i;
             uint32_t v[G];
 #pragma unroll
@@ -122,7 +124,8 @@ __device__ __forceinline__ void find_threshold(uint32_t *hl, uint32_t *hsum, uin
 }
 
 template <int G>
-__global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
+__global__ void __launch_bounds__(topk_threads<G>()) topk_kernel(TopkArgs a) {
+    constexpr int NT = topk_threads<G>(), NW = NT / 32;
     // dynamic smem: keys[chunk] | hist_local[4096] | (G > 1) hist_sum[4096]
     // (peers read this CTA's histogram of a pass only between that pass's two
     // cluster barriers, so one local buffer serves every pass)
@@ -133,7 +136,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     uint32_t *hsum = (G > 1) ? hist0 + BINS_A : nullptr;
     __shared__ uint32_t scan_tmp[64];
     __shared__ uint32_t sel[3];
-    __shared__ uint32_t warp_gt[kTopkWarps];   // packed per-warp counts
+    __shared__ uint32_t warp_gt[NW];   // packed per-warp counts
     __shared__ uint32_t cta_counts[2];
     __shared__ uint32_t low_bits[2];   // OR, AND of the last digit over the first refinement's keys
 
@@ -142,15 +145,20 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     // Start copying this CTA's chunk of the row into shared memory before
-    // anything waits.  The row's valid length is not known yet, so the copy
-    // runs to the row's allocated length; columns past the valid length are
-    // never read back.
+    // anything waits.  With block-id candidates the row's valid length is
+    // known only after the ids are checked, so that copy runs to the row's
+    // allocated length; columns past the valid length are never read back.
     const int c0 = (int)rank * a.chunk;
     const float *row = a.scores + (int64_t)r * a.ld;
+    int n_bound = a.row_len;
     {
-        const int pre4 = max(0, min(c0 + a.chunk, a.row_len) - c0) >> 2;   // c0 and ld are multiples of 4
+        if (!a.by_blocks) {
+            n_bound = a.n_valid ? a.n_valid[r] : a.row_len - a.rows + r + 1;
+            n_bound = n_bound < 0 ? 0 : (n_bound > a.row_len ? a.row_len : n_bound);
+        }
+        const int pre4 = max(0, min(c0 + a.chunk, n_bound) - c0) >> 2;   // c0 and ld are multiples of 4
         const float4 *src4 = reinterpret_cast<const float4 *>(row + c0);
-        for (int i = tid; i < pre4; i += kTopkThreads) cp_async16(keys + 4 * i, src4 + i);
+        for (int i = tid; i < pre4; i += NT) cp_async16(keys + 4 * i, src4 + i);
     }
 
     int n;
@@ -164,7 +172,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
         if (tid == 0) cta_counts[0] = 0u;
         __syncthreads();
         uint32_t valid = 0;
-        for (int i = tid; i < a.keep; i += kTopkThreads) {
+        for (int i = tid; i < a.keep; i += NT) {
             const int b = brow[i];
             if (b >= 0) {
                 ++valid;
@@ -210,7 +218,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     };
 
     if (cand) {   // the position map must be strictly ascending and non-negative
-        for (int i = tid; i < len; i += kTopkThreads) {
+        for (int i = tid; i < len; i += NT) {
             const int col = c0 + i;
             const int32_t c = cand[col];
             if (c < 0) report(a.dev_status, SA_DEV_INDEX);
@@ -219,31 +227,31 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     }
 
     if (n <= a.K) {   // every candidate is kept: no select needed
-        for (int i = tid; i < len; i += kTopkThreads) out[c0 + i] = pos(c0 + i);
+        for (int i = tid; i < len; i += NT) out[c0 + i] = pos(c0 + i);
         if (rank == 0)
-            for (int i = n + tid; i < a.K; i += kTopkThreads) out[i] = -1;
+            for (int i = n + tid; i < a.K; i += NT) out[i] = -1;
         cp_async_wait_all();   // the copies into this CTA's shared memory end before it exits
         return;   // uniform over the cluster: no distributed smem was touched
     }
 
     // ---- the chunk as order-preserving keys, counting the top 11 bits
-    for (int i = tid; i < BINS_A / 4; i += kTopkThreads) reinterpret_cast<uint4 *>(hist0)[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = tid; i < BINS_A / 4; i += NT) reinterpret_cast<uint4 *>(hist0)[i] = make_uint4(0u, 0u, 0u, 0u);
     cp_async_wait_all();
     __syncthreads();
     {
         const int len4 = len >> 2;
-        for (int i = tid; i < len4; i += kTopkThreads) {
+        for (int i = tid; i < len4; i += NT) {
             const uint4 f = reinterpret_cast<const uint4 *>(keys)[i];
-            uint4 k;
-            k.x = order_key(__uint_as_float(f.x)); k.y = order_key(__uint_as_float(f.y));
-            k.z = order_key(__uint_as_float(f.z)); k.w = order_key(__uint_as_float(f.w));
-            reinterpret_cast<uint4 *>(keys)[i] = k;
-            atomicAdd(&hist0[k.x >> SA_], 1u);
-            atomicAdd(&hist0[k.y >> SA_], 1u);
-            atomicAdd(&hist0[k.z >> SA_], 1u);
-            atomicAdd(&hist0[k.w >> SA_], 1u);
+            uint4 u;
+            u.x = order_key(__uint_as_float(f.x)); u.y = order_key(__uint_as_float(f.y));
+            u.z = order_key(__uint_as_float(f.z)); u.w = order_key(__uint_as_float(f.w));
+            reinterpret_cast<uint4 *>(keys)[i] = u;
+            atomicAdd(&hist0[u.x >> SA_], 1u);
+            atomicAdd(&hist0[u.y >> SA_], 1u);
+            atomicAdd(&hist0[u.z >> SA_], 1u);
+            atomicAdd(&hist0[u.w >> SA_], 1u);
         }
-        for (int i = (len4 << 2) + tid; i < len; i += kTopkThreads) {   // the last len % 4 columns
+        for (int i = (len4 << 2) + tid; i < len; i += NT) {   // the last len % 4 columns
             const uint32_t k = order_key(row[c0 + i]);
             keys[i] = k;
             atomicAdd(&hist0[k >> SA_], 1u);
@@ -252,7 +260,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     __syncthreads();
 
     uint32_t need = (uint32_t)a.K;      // keys still to take among those matching `prefix`
-    find_threshold<G, BINS_A>(hist0, hsum, need, scan_tmp, sel, tid);
+    find_threshold<G, BINS_A, NT>(hist0, hsum, need, scan_tmp, sel, tid);
     uint32_t prefix = sel[0] << SA_, mask = 0xFFFFFFFFu << SA_;
     need -= sel[1];
     bool whole = sel[2] == need;        // the threshold bin is taken entirely
@@ -267,7 +275,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
         const uint32_t dmask = pass == 1 ? (uint32_t)BINS_1 - 1u : 1023u;   // the digit: bits SA_-1..10, then 9..0
         const bool track = G == 1 && pass == 1;
         uint32_t *hl = hist0;
-        for (int i = tid; i < (int)(dmask + 1) / 4; i += kTopkThreads)
+        for (int i = tid; i < (int)(dmask + 1) / 4; i += NT)
             reinterpret_cast<uint4 *>(hl)[i] = make_uint4(0u, 0u, 0u, 0u);
         if (track && tid == 0) { low_bits[0] = 0u; low_bits[1] = 1023u; }
         __syncthreads();
@@ -282,14 +290,14 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
             }
         };
         const int len4 = len >> 2;
-        for (int i = tid; i < len4; i += kTopkThreads) {
+        for (int i = tid; i < len4; i += NT) {
             const uint4 k = reinterpret_cast<const uint4 *>(keys)[i];
             count(k.x);
             count(k.y);
             count(k.z);
             count(k.w);
         }
-        for (int i = (len4 << 2) + tid; i < len; i += kTopkThreads) count(keys[i]);
+        for (int i = (len4 << 2) + tid; i < len; i += NT) count(keys[i]);
         if (track) {
             lor = __reduce_or_sync(0xffffffffu, lor);
             land = __reduce_and_sync(0xffffffffu, land);
@@ -300,9 +308,9 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
         }
         __syncthreads();
         if (pass == 1)
-            find_threshold<G, BINS_1>(hl, hsum, need, scan_tmp, sel, tid);
+            find_threshold<G, BINS_1, NT>(hl, hsum, need, scan_tmp, sel, tid);
         else
-            find_threshold<G, 1024>(hl, hsum, need, scan_tmp, sel, tid);
+            find_threshold<G, 1024, NT>(hl, hsum, need, scan_tmp, sel, tid);
         prefix |= sel[0] << shift;
         mask |= dmask << shift;
         need -= sel[1];
@@ -319,7 +327,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     // visits them 128 at a time, 4 consecutive keys per lane; per-lane counts
     // of "> tau" (low 16 bits) and "== tau" (high 16 bits) are packed into one
     // word, so one warp sum or scan handles both (a CTA holds < 65536 keys).
-    const int sub = ((len + 4 * kTopkThreads - 1) / (4 * kTopkThreads)) * 128;
+    const int sub = ((len + 4 * NT - 1) / (4 * NT)) * 128;
     const int w0 = warp * sub, w1 = min(w0 + sub, len);
     auto load4 = [&](int p, uint32_t (&u)[4]) {
         if (p + 3 < w1) {
@@ -356,7 +364,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(TopkArgs a) {
     if (lane == 0) warp_gt[warp] = wtot;
     __syncthreads();
     const uint32_t wbase = __reduce_add_sync(0xffffffffu, lane < warp ? warp_gt[lane] : 0u);   // warps before
-    if (tid == kTopkThreads - 1) {
+    if (tid == NT - 1) {
         cta_counts[0] = (wbase + wtot) & 0xFFFFu;
         cta_counts[1] = (wbase + wtot) >> 16;
     }
@@ -600,7 +608,7 @@ static sa_status launch_topk_g(const TopkArgs &a, size_t smem, cudaStream_t st) 
     if (prepare_kernel<topk_kernel<G>>(smem, G > 8) != cudaSuccess) return SA_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.rows * G));
-    cfg.blockDim = dim3(kTopkThreads);
+    cfg.blockDim = dim3(topk_threads<G>());
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -628,7 +636,8 @@ sa_status launch_topk(TopkArgs a, cudaStream_t st) {
     a.chunk = chunk;
     // histograms, later reused for the compaction's per-lane flags (one word
     // per lane and 128-key group of each warp's span)
-    const size_t flag_words = (size_t)kTopkWarps * (((size_t)chunk + 4 * kTopkThreads - 1) / (4 * kTopkThreads)) * 32;
+    const size_t nt = g > 1 ? topk_threads<2>() : topk_threads<1>();
+    const size_t flag_words = (nt / 32) * (((size_t)chunk + 4 * nt - 1) / (4 * nt)) * 32;
     const size_t hist_words = std::max((g > 1) ? 2 * (size_t)kBinsMax : (size_t)kBinsMax / 2, flag_words);
     const size_t smem = ((size_t)chunk + hist_words) * 4;
     switch (g) {
