@@ -23,22 +23,26 @@
 // than 2^8 (then O^T and the row sums are rescaled), so P stays below 256.
 //
 // Persistent CTAs (one per SM) take queries T-1-c, T-1-c-G, ... (heavy first)
-// and stream their tiles through a pipeline of warp roles:
-//   warp 13     index builder: copies the query's top-K row to shared memory,
+// and stream their tiles through a pipeline of warp roles (kGW = 2 gather
+// warps per side; four per side measured slower: fewer registers per thread):
+//   index builder (one warp): copies the query's top-K row to shared memory,
 //               validates it (SA_DEV_INDEX / SA_DEV_ORDER), finds the prefix
-//               of entries <= p - W and writes the byte offsets of each
-//               128-key tile's cache rows (top-K prefix, then the window;
-//               0xffffffff past the selection) into a ring
-//   warps 0..3  gather: 16-byte cp.async of every selected K row (warps 0-1,
-//               with the query's Q rows at its first tile) and V row (warps
-//               2-3) into 128B-swizzled tiles of separate K and V rings (rows
-//               past the selection are zero-filled); completion is tracked by
-//               the slot's mbarrier (cp.async.mbarrier.arrive.noinc)
-//   warp 12     S issuer (one thread) and TMEM owner
-//   warp 14     P V issuer (one thread)
-//   warps 4..11 softmax of tile g in two groups of four warps, each group
-//               owning half of the heads (TMEM lane quadrant = warp % 4), then
-//               the epilogue of each query: O^T / l -> out (bf16), lse
+//               of entries <= p - W, writes the byte offsets of each 128-key
+//               tile's cache rows (top-K prefix, then the window; a slot past
+//               the selection repeats the tile's first row, whose score is
+//               masked) into a ring, and publishes the tile's record to the
+//               MMA and softmax warps
+//   gather (warps 0 .. 2 kGW - 1): 16-byte cp.async of every selected K row
+//               (with the query's Q rows at its first tile) and V row into
+//               128B-swizzled tiles of separate K and V rings; completion is
+//               tracked by the slot's mbarrier (cp.async.mbarrier.arrive.noinc)
+//   S issuer (one thread) and TMEM owner
+//   P V issuer (one thread)
+//   softmax (eight warps): tile g in two groups of four warps, each group
+//               owning half of the heads (TMEM lane quadrant = warp % 4), one
+//               vote per tile, P^T written MN-major (16-byte rows of 8 heads);
+//               each query's epilogue (O^T / l -> out bf16, lse) runs once its
+//               last P V is known to be done
 // Every wait is bounded (SA_DEV_TIMEOUT), and the softmax warps take each
 // wait's outcome together (bar.red) before any barrier among them.
 #include <math_constants.h>
@@ -51,10 +55,17 @@ namespace sa {
 namespace {
 
 constexpr int kGTile = 128;                  // keys per tile (MMA M)
-constexpr int kGThreads = 15 * 32;
-// warp roles: 0..3 gather, 4..11 softmax (two groups of four, each owning half
-// of the heads), then the S issuer (TMEM owner), the index builder, the P V issuer
-constexpr int kWarpS = 12, kWarpBuild = 13, kWarpPV = 14;
+#ifndef SA_GATHER_WARPS_PER_SIDE
+#define SA_GATHER_WARPS_PER_SIDE 2
+#endif
+constexpr int kGW = SA_GATHER_WARPS_PER_SIDE;   // gather warps per side (K, V)
+constexpr int kGKeys = kGTile / kGW;            // keys of a tile per gather warp
+constexpr int kWarpSmx = 2 * kGW;               // first softmax warp
+// warp roles: 0..2 kGW - 1 gather (K side first), then eight softmax warps (two
+// groups of four, each owning half of the heads), then the S issuer (TMEM
+// owner), the index builder, the P V issuer
+constexpr int kWarpS = kWarpSmx + 8, kWarpBuild = kWarpS + 1, kWarpPV = kWarpS + 2;
+constexpr int kGThreads = (kWarpPV + 1) * 32;
 constexpr int kGRing = 6;                    // row-index tiles the builder runs ahead
 constexpr int kGMaxK = 2048;                 // top-K entries held in shared memory per query
 constexpr int kGInfo = 16;                   // tile records in flight (built .. read by the P V issuer)
@@ -270,11 +281,11 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NK; ++i) {
-            mbar_init(&k_full[i], 64);         // 64 cp.async arrivals
+            mbar_init(&k_full[i], 32 * kGW);   // one cp.async arrival per K-side thread
             mbar_init(&k_empty[i], 1);
         }
         for (int i = 0; i < NV; ++i) {
-            mbar_init(&v_full[i], 64);         // 64 cp.async arrivals
+            mbar_init(&v_full[i], 32 * kGW);   // one cp.async arrival per V-side thread
             mbar_init(&v_empty[i], 1);
         }
         for (int i = 0; i < kGInfo; ++i) {
@@ -283,7 +294,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
         }
         for (int i = 0; i < kGRing; ++i) {
             mbar_init(&row_full[i], 1);
-            mbar_init(&row_empty[i], 4);
+            mbar_init(&row_empty[i], 2 * kGW);   // every gather warp has issued the tile
         }
         for (int i = 0; i < kGSB; ++i) {
             mbar_init(&s_full[i], 1);
@@ -383,9 +394,10 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
                                                        abort_flag));
                 if (!ok) break;
                 // Byte offsets of the tile's 128 rows, in the order the gather
-                // lanes read them: key kk = 64 pw + 2 it + sub sits at 64 pw +
-                // 32 sub + it.  A slot past the selection repeats the tile's
-                // first row: its score is masked to -inf, so its P is exactly 0.
+                // lanes read them: key kk = kGKeys pw + 2 it + sub sits at
+                // kGKeys pw + (kGKeys / 2) sub + it.  A slot past the selection
+                // repeats the tile's first row: its score is masked to -inf, so
+                // its P is exactly 0.
                 int32_t *rr = rows + slot * kGTile;
                 int first_row = 0;
 #pragma unroll
@@ -394,7 +406,8 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
                     int row = kk < n_top ? list[kk] : (kk < n_keys ? w0 + (kk - n_top) : -1);
                     if (u == 0) first_row = __shfl_sync(0xffffffffu, row, 0);
                     if (row < 0) row = first_row;
-                    rr[(u >> 1) * 64 + (lane & 1) * 32 + (u & 1) * 16 + (lane >> 1)] =
+                    const int kt = u * 32 + lane;   // key within the tile
+                    rr[(kt / kGKeys) * kGKeys + (kt & 1) * (kGKeys / 2) + ((kt % kGKeys) >> 1)] =
                         (int32_t)((uint32_t)row * (uint32_t)(D * 2));
                 }
                 // the tile's record for the gather warps, and for the MMA and
@@ -435,13 +448,14 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
             }
         }
         __syncwarp();
-    } else if (warp < 4) {
+    } else if (warp < kWarpSmx) {
         // ------------------------------------------------------------ gather
-        // Warps 0-1 copy K rows (and a query's Q rows with its first tile),
-        // warps 2-3 copy V rows, each pair on its own ring: K(g) waits only for
-        // S(g - kNK) to finish with its slot, V(g) only for P V(g - kNV).
-        const bool kside = warp < 2;
-        const int pw = warp & 1, t64 = pw * 32 + lane;   // thread within the side
+        // The first kGW warps copy K rows (and a query's Q rows with its first
+        // tile), the next kGW copy V rows, each side on its own ring: K(g)
+        // waits only for S(g - kNK) to finish with its slot, V(g) only for
+        // P V(g - kNV).
+        const bool kside = warp < kGW;
+        const int pw = warp % kGW, ts = pw * 32 + lane;   // thread within the side
         const int sub = lane >> 4, ch = lane & 15;
         const uint8_t *base = reinterpret_cast<const uint8_t *>(kside ? P.k : P.v) + ch * 16;
         bool ok = true;
@@ -460,7 +474,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
                     if (h.i == 0) {
                         uint8_t *sq = sm + C::kOffQ + (h.j & 1) * C::kQ;
                         const uint16_t *qrow = P.q + (int64_t)h.t * P.Hq * D;
-                        for (int idx = t64; idx < P.Hq * 16; idx += 64) {
+                        for (int idx = ts; idx < P.Hq * 16; idx += 32 * kGW) {
                             const int r = idx >> 4, c = idx & 15;
                             cp_async16(sq + sw_off(r, c, C::kQHalf), qrow + (int64_t)r * D + c * 8);
                         }
@@ -471,18 +485,19 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
                     if (!ok) break;
                     dst = sm + C::kOffV + (g % NV) * C::kKV;
                 }
-                // this warp's 64 keys (key 64 pw + 2 it + sub for lane half sub):
-                // the byte offsets as eight 16-byte loads, then the copies
-                const uint4 *rr = reinterpret_cast<const uint4 *>(rows + slot * kGTile + pw * 64 + sub * 32);
-                uint32_t ro[32];
+                // this warp's kGKeys keys (key kGKeys pw + 2 it + sub for lane
+                // half sub): the byte offsets as 16-byte loads, then the copies
+                constexpr int NIT = kGKeys / 2;
+                const uint4 *rr = reinterpret_cast<const uint4 *>(rows + slot * kGTile + pw * kGKeys + sub * NIT);
+                uint32_t ro[NIT];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
+                for (int q = 0; q < NIT / 4; ++q) {
                     const uint4 o = rr[q];
                     ro[4 * q] = o.x; ro[4 * q + 1] = o.y; ro[4 * q + 2] = o.z; ro[4 * q + 3] = o.w;
                 }
 #pragma unroll
-                for (int it = 0; it < 32; ++it) {
-                    const int key = pw * 64 + 2 * it + sub;
+                for (int it = 0; it < NIT; ++it) {
+                    const int key = pw * kGKeys + 2 * it + sub;
                     cp_async16(dst + sw_off(key, ch, C::kHalf), base + ro[it]);
                 }
             }
@@ -571,9 +586,9 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------------------ softmax + epilogue (warps 4..11)
+        // ------------------------------------------------------------ softmax + epilogue (eight warps)
         constexpr int HG = HQP / 2;                       // heads of this group
-        const int quad = warp & 3, hg = (warp - 4) >> 2, h0 = hg * HG;
+        const int quad = warp & 3, hg = (warp - kWarpSmx) >> 2, h0 = hg * HG;
         const int bar_red = 2 + 2 * hg, bar_x = 3 + 2 * hg;   // this group's named barriers
         const int key = quad * 32 + lane;                 // TMEM lane: key (S^T) or head dim (O^T)
         const uint32_t lane_t = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)h0;
@@ -768,7 +783,7 @@ __global__ void __launch_bounds__(kGThreads, 1) gather_attn_tc_kernel(GParams P)
             }
         }
     }
-    // Once every role is past its last TMEM access, warp 8 frees TMEM.
+    // Once every role is past its last TMEM access, the S issuer's warp frees TMEM.
     tc_fence_before();
     bar_sync_n(1, kGThreads);
     if (warp == kWarpS) {
