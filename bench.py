@@ -64,9 +64,14 @@ def load_peaks():
 GATHER_CEILING_GBS = 20018.0
 
 
+def CONFIG_KIND(name):
+    from workloads import CONFIGS
+    return CONFIGS[name]["kind"]
+
+
 # --------------------------------------------------------------------------- ncu traffic
 STAGE_SOURCE = {"indexer": "indexer.cu", "coarse_indexer": "indexer.cu", "topk": "topk.cu",
-                "coarse_topk": "topk.cu", "fine_topk": "topk.cu", "attention": "attention.cu+attention_tc.cu+attention_gather.cu",
+                "coarse_topk": "topk.cu", "fine_topk": "topk.cu", "indexer_topk": "topk.cu", "attention": "attention.cu+attention_tc.cu+attention_gather.cu",
                 "fine_indexer": "block_scores.cu", "pool": "two_stage.cu",
                 "block_counts": "two_stage.cu"}
 
@@ -179,7 +184,7 @@ class ClockSampler:
 
 
 # --------------------------------------------------------------------------- workloads
-def make_case(name, seed, device, index_fp8=False, rows=None):
+def make_case(name, seed, device, index_fp8=False, rows=None, fused=False):
     """Device-resident inputs, pinned host copies and a plan for one workload.
     index_fp8: the indexer operands qI and kI are quantised to e4m3 once, on
     the device, before any timing (keys enter an FP8 index cache when they
@@ -223,10 +228,12 @@ def make_case(name, seed, device, index_fp8=False, rows=None):
         if cfg.get("paged", False):
             make_plan = lambda: DecodePlan(B, cfg["Hq"], cfg["d"], cfg["H_I"], cfg["D_I"], cfg["K"], cfg["W"],
                                            S_max=0, paged=True, max_pages=inp["page_table"].shape[1],
-                                           pool_pages=inp["k"].shape[0], index_fp8=index_fp8, device=device)
+                                           pool_pages=inp["k"].shape[0], index_fp8=index_fp8, fused=fused,
+                                           device=device)
         else:
             make_plan = lambda: DecodePlan(B, cfg["Hq"], cfg["d"], cfg["H_I"], cfg["D_I"], cfg["K"], cfg["W"],
-                                           S_max=inp["k"].shape[1], index_fp8=index_fp8, device=device)
+                                           S_max=inp["k"].shape[1], index_fp8=index_fp8, fused=fused,
+                                           device=device)
         # per step a decode call receives the new tokens; the KV cache is resident state
         step_inputs = ["q", "qI", "w", "lengths"]
         units = B
@@ -265,6 +272,9 @@ def stage_work(case):
         st["indexer"] = dict(bytes=qI_b + w_b + pairs * D * eb + 4 * pairs, flops=2.0 * pairs * H * D,
                              bound="hbm")
         st["topk"] = dict(bytes=4 * pairs + idx_b, flops=0.0, bound="hbm")
+        # fused: the scores stay in shared memory, so the stage reads the keys and writes the selection
+        st["indexer_topk"] = dict(bytes=qI_b + w_b + pairs * D * eb + idx_b, flops=2.0 * pairs * H * D,
+                                  bound="hbm")
         st["attention"] = dict(bytes=2 * q_b + sum_sel * d * 2 * 2 + idx_b, flops=4.0 * Hq * d * sum_sel,
                                bound="hbm")
     else:
@@ -351,7 +361,8 @@ def run_ours(args, rank, world, local_rank):
     device = "cuda:%d" % local_rank
     torch.cuda.set_device(local_rank)
     peaks = load_peaks()
-    case = make_case(args.workload, seed=rank, device=device, index_fp8=args.index_fp8, rows=args.rows)
+    case = make_case(args.workload, seed=rank, device=device, index_fp8=args.index_fp8, rows=args.rows,
+                     fused=args.fused_select)
     stream = torch.cuda.current_stream()
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=device)
     plan, d = case["plan"], case["devs"]
@@ -467,7 +478,8 @@ def run_ours(args, rank, world, local_rank):
     w = work["stages"][dom]
     roof["kernel"] = dom
     roof["algorithmic"] = w["flops"] if roof["bound"] == "tensor" else w["bytes"]
-    tag = args.workload + ("+rows%d" % args.rows if args.rows else "") + ("+fp8-indexer" if args.index_fp8 else "")
+    tag = (args.workload + ("+rows%d" % args.rows if args.rows else "") + ("+fp8-indexer" if args.index_fp8 else "")
+           + ("+fused-select" if args.fused_select else ""))
     roof["traffic"] = ncu_traffic(tag, dom)   # per launch, from a capture of this exact source
     roof["peak_src"] = peaks["src"] + " (burst figure; kernel timed alone per step)"
     line = {
@@ -477,6 +489,7 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic",
         "config": {"workload": args.workload, **{k: v for k, v in case["cfg"].items() if k != "kind"},
                    "indexer_operands": "e4m3 (quantised before timing)" if args.index_fp8 else "bf16",
+                   **({"select": "indexer and top-K fused in one kernel"} if args.fused_select else {}),
                    "parallelism": "replicas (an independent sequence per GPU)" if world > 1 else "single GPU",
                    "l2": "flushed between steps (512 MB write outside the timed brackets)",
                    "launch": "step replayed as a captured CUDA graph"},
@@ -533,12 +546,16 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="prefill_64k_two_stage")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--fused-select", action="store_true",
+                    help="decode workloads: the indexer and the top-K as one kernel (scores kept on chip)")
     ap.add_argument("--rows", type=int, default=None,
                     help="prefill workloads: time the last ROWS query rows of the sequence (a chunk of the prompt)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--index-fp8", action="store_true",
                     help="indexer on e4m3 operands (single-stage prefill and decode workloads)")
     args = ap.parse_args()
+    if args.fused_select and CONFIG_KIND(args.workload) != "decode":
+        raise SystemExit("--fused-select serves the decode workloads")
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

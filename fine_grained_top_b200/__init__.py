@@ -41,6 +41,8 @@ SIGNATURES = {
                                         _vp, _sz, _vp, _vp]),
     "sa_topk_select": (_i32, [_vp, _i64, _i32, _i32, _vp, _vp, _i64, _i32, _vp, _vp, _vp]),
     "sa_topk_select_blocks": (_i32, [_vp, _i64, _i32, _i32, _vp, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "sa_indexer_topk_decode": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _i32,
+                                      _vp, _vp, _vp]),
     "sa_prefill_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
     "sa_sparse_attn_prefill": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp,
                                       _vp, _vp, _sz, _vp, _vp]),
@@ -144,6 +146,13 @@ def sa_topk_select(scores, ld_scores, rows, row_len, n_valid, cand_map, ld_cand,
 def sa_topk_select_blocks(scores, ld_scores, T, S, blocks, keep, block, K, topk, dev_status=None, stream=None):
     _check(_lib.sa_topk_select_blocks(_ptr(scores), ld_scores, T, S, _ptr(blocks), keep, block, K, _ptr(topk),
                                       _ptr(dev_status), _stream(stream)), "sa_topk_select_blocks")
+
+
+def sa_indexer_topk_decode(qI, w, kI, page_table, max_pages, pool_pages, page_size, B, S, H_I, D_I, seq_lens, K,
+                           topk, dev_status=None, stream=None):
+    _check(_lib.sa_indexer_topk_decode(_ptr(qI), _ptr(w), _ptr(kI), _ptr(page_table), max_pages, pool_pages,
+                                       page_size, B, S, H_I, D_I, _ptr(seq_lens), K, _ptr(topk),
+                                       _ptr(dev_status), _stream(stream)), "sa_indexer_topk_decode")
 
 
 def sa_prefill_workspace_bytes(T, S, K, W, Hq, d) -> int:

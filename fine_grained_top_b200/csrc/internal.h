@@ -28,6 +28,16 @@ struct TopkArgs {
     bool by_blocks = false;
     const int32_t *blocks = nullptr;   // [rows, keep]; may be NULL when keep == 0
     int keep = 0, block = 0, S = 0;
+    // fused indexer (decode, one query per row): the scores of row r are
+    // computed in shared memory from qI [rows, H_I, D_I], w [rows, H_I] and
+    // the row's keys of kI (contiguous [rows, f_S, D_I], or a pool of 64-key
+    // pages through f_page_table [rows, f_max_pages]) instead of read from
+    // `scores`; n_valid gives each row's key count
+    bool fused = false;
+    const uint16_t *f_qI = nullptr, *f_w = nullptr, *f_kI = nullptr;
+    const int32_t *f_page_table = nullptr;
+    int f_max_pages = 0, f_pool_pages = 0, f_HI = 0, f_DI = 0, f_S = 0;
+    int ring_off = 0;   // (set by the launcher) words from the chunk start to the key-tile ring
 };
 sa_status launch_topk(TopkArgs a, cudaStream_t st);
 int topk_max_row_len();

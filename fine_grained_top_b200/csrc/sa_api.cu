@@ -177,6 +177,26 @@ sa_status sa_topk_select_blocks(const float *scores, int64_t ld_scores, int T, i
     });
 }
 
+sa_status sa_indexer_topk_decode(const sa_bf16 *qI, const sa_bf16 *w, const sa_bf16 *kI, const int32_t *page_table,
+                                 int max_pages, int pool_pages, int page_size, int B, int S, int H_I, int D_I,
+                                 const int32_t *seq_lens, int K, int32_t *topk, int *dev_status, sa_stream stream) {
+    if (B < 0 || S < 0 || K < 0 || H_I < 1) return SA_ERR_INVALID_ARG;
+    if (page_table && (page_size != 64 || max_pages < 0 || pool_pages < 1 || (int64_t)max_pages * 64 < S))
+        return page_size != 64 ? SA_ERR_UNSUPPORTED : SA_ERR_INVALID_ARG;
+    if (H_I > 8 || (D_I != 64 && D_I != 128) || S > topk_max_row_len()) return SA_ERR_UNSUPPORTED;
+    if (B == 0 || K == 0) return SA_OK;
+    if (!qI || !w || !kI || !seq_lens || !topk) return SA_ERR_INVALID_ARG;
+    if (!aligned16(qI) || !aligned16(kI) || (reinterpret_cast<uintptr_t>(w) & 1u)) return SA_ERR_INVALID_ARG;
+    return guarded([&] {
+        TopkArgs a;
+        a.scores = nullptr; a.ld = 0; a.rows = B; a.row_len = S; a.n_valid = seq_lens;
+        a.cand = nullptr; a.ld_cand = 0; a.K = K; a.out = topk; a.dev_status = dev_status; a.chunk = 0;
+        a.fused = true; a.f_qI = qI; a.f_w = w; a.f_kI = kI; a.f_page_table = page_table;
+        a.f_max_pages = max_pages; a.f_pool_pages = pool_pages; a.f_HI = H_I; a.f_DI = D_I; a.f_S = S;
+        return launch_topk(a, cs(stream));
+    });
+}
+
 size_t sa_prefill_workspace_bytes(int T, int S, int K, int W, int Hq, int d) {
     if (T < 0 || S < 0 || K < 0 || W < 0) return 0;
     PrefillArgs a = {};

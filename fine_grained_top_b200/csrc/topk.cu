@@ -123,8 +123,115 @@ __device__ __forceinline__ void find_threshold(uint32_t *hl, uint32_t *hsum, uin
     __syncthreads();
 }
 
-template <int G>
-__global__ void __launch_bounds__(topk_threads<G>()) topk_kernel(TopkArgs a) {
+// ---------------------------------------------------------------- fused indexer
+// Decode rows with the indexer fused in: the scores of columns [c0, c0 + len)
+// of row r (keys c0 .. of sequence r),
+//   I[s] = sum_{j < H_I} w[j] * max(0, qI[j, :] . kI[s, :]),
+// are computed on the tensor cores and written straight into keys[] as
+// order-preserving keys while the first histogram is counted; they never
+// reach global memory.  mma.sync m16n8k16 (bf16 x bf16 -> fp32) with M = 16
+// keys, N = 8 heads (H_I <= 8, missing heads zero), K = 16 dims; the key rows
+// come through a ring of four 32 KB tiles in shared memory, three in flight
+// while one is used (16-byte cp.async, 16-byte chunks XOR-swizzled by row for
+// conflict-free ldmatrix).  The head sum runs over the four lanes of a quad (two heads per
+// lane), so for integer-valued inputs every sum is exact and the result equals
+// the unfused indexer's.
+constexpr int kFusedSlotBytes = 32768;   // one ring slot: 256 keys of 128 bytes (128 of 256)
+constexpr int kFusedStages = 4;          // ring slots (up to three tiles in flight while one is used)
+
+template <int ROWB>
+__device__ __forceinline__ uint32_t ring_swz(int row, int c) {
+    return (uint32_t)(row * ROWB + ((c ^ (row & 7)) << 4));
+}
+
+template <int NT, int D_I, int SHIFT>
+__device__ void fused_scores(const TopkArgs &a, int r, int c0, int len, uint32_t *keys, uint32_t *hist0,
+                             uint8_t *ring, int tid) {
+    constexpr int ROWB = D_I * 2, CH = ROWB / 16, KS = D_I / 16, NW = NT / 32;
+    constexpr int TILE = kFusedSlotBytes / ROWB;   // keys per slot
+    const int lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
+    const int H = a.f_HI;
+    // B fragments (K x N = dims x heads, "col"): head g, dims 16 ks + 2t, +1
+    // and 16 ks + 2t + 8, +9 (two consecutive bf16 in each 32-bit register)
+    uint32_t bq[KS][2];
+    const uint32_t *q32 = reinterpret_cast<const uint32_t *>(a.f_qI + (int64_t)r * H * D_I);
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+        bq[ks][0] = g < H ? q32[(g * D_I + 16 * ks + 2 * t) >> 1] : 0u;
+        bq[ks][1] = g < H ? q32[(g * D_I + 16 * ks + 2 * t + 8) >> 1] : 0u;
+    }
+    // this lane's heads in the accumulator: 2t and 2t + 1
+    const uint16_t *wr = a.f_w + (int64_t)r * H;
+    const float w0 = 2 * t < H ? __uint_as_float((uint32_t)wr[2 * t] << 16) : 0.f;
+    const float w1 = 2 * t + 1 < H ? __uint_as_float((uint32_t)wr[2 * t + 1] << 16) : 0.f;
+    const int32_t *pt = a.f_page_table ? a.f_page_table + (int64_t)r * a.f_max_pages : nullptr;
+
+    // tile `tile` into slot tile % kFusedStages; one commit group per call
+    auto issue = [&](int tile) {
+        uint8_t *dst = ring + (tile % kFusedStages) * kFusedSlotBytes;
+        const int k0 = tile * TILE;
+        for (int idx = tid; idx < TILE * CH; idx += NT) {
+            const int i = idx / CH, c = idx % CH;
+            if (k0 + i >= len) break;   // idx grows with i: the rest of this thread's copies are past the chunk
+            const int s = c0 + k0 + i;  // key position in the sequence
+            int64_t row;
+            if (pt) {
+                int pid = pt[s >> 6];
+                if (pid < 0 || pid >= a.f_pool_pages) {
+                    if (c == 0) report(a.dev_status, SA_DEV_INDEX);
+                    pid = 0;   // any valid row: the result is flagged
+                }
+                row = (int64_t)pid * 64 + (s & 63);
+            } else {
+                row = (int64_t)r * a.f_S + s;
+            }
+            cp_async16(dst + ring_swz<ROWB>(i, c), a.f_kI + row * D_I + c * 8);
+        }
+    };
+    const int ntile = (len + TILE - 1) / TILE;
+#pragma unroll
+    for (int p = 0; p < kFusedStages - 1; ++p) {
+        if (p < ntile) issue(p);
+        cp_async_commit();   // (empty groups keep the count uniform)
+    }
+    for (int tile = 0; tile < ntile; ++tile) {
+        cp_async_wait<kFusedStages - 2>();   // this thread's copies of `tile` have landed
+        __syncthreads();                     // ... everyone's; and every warp is past tile - 1
+        if (tile + kFusedStages - 1 < ntile) issue(tile + kFusedStages - 1);   // into the slot of tile - 1
+        cp_async_commit();
+        const uint8_t *buf = ring + (tile % kFusedStages) * kFusedSlotBytes;
+        for (int mt = warp; mt < TILE / 16; mt += NW) {
+            const int k0 = tile * TILE + mt * 16;   // first column of the 16-key group
+            if (k0 >= len) break;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+                uint32_t af[4];
+                const int row = mt * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+                ldmatrix_x4(af, buf + ring_swz<ROWB>(row, ks * 2 + (lane >> 4)));
+                mma_bf16_16816(acc, af, bq[ks]);
+            }
+            // acc: (key g, heads 2t, 2t+1), (key g + 8, heads 2t, 2t+1)
+            float s_lo = w0 * fmaxf(acc[0], 0.f) + w1 * fmaxf(acc[1], 0.f);
+            float s_hi = w0 * fmaxf(acc[2], 0.f) + w1 * fmaxf(acc[3], 0.f);
+            s_lo += __shfl_xor_sync(0xffffffffu, s_lo, 1);
+            s_hi += __shfl_xor_sync(0xffffffffu, s_hi, 1);
+            s_lo += __shfl_xor_sync(0xffffffffu, s_lo, 2);
+            s_hi += __shfl_xor_sync(0xffffffffu, s_hi, 2);
+            const int col = k0 + g + (t == 1 ? 8 : 0);
+            if (t < 2 && col < len) {
+                const uint32_t u = order_key(t == 0 ? s_lo : s_hi);
+                keys[col] = u;
+                atomicAdd(&hist0[u >> SHIFT], 1u);
+            }
+        }
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+}
+
+template <int G, bool FUSED>
+__device__ __forceinline__ void topk_body(const TopkArgs &a) {
     constexpr int NT = topk_threads<G>(), NW = NT / 32;
     // dynamic smem: keys[chunk] | hist_local[4096] | (G > 1) hist_sum[4096]
     // (peers read this CTA's histogram of a pass only between that pass's two
@@ -149,16 +256,18 @@ __global__ void __launch_bounds__(topk_threads<G>()) topk_kernel(TopkArgs a) {
     // known only after the ids are checked, so that copy runs to the row's
     // allocated length; columns past the valid length are never read back.
     const int c0 = (int)rank * a.chunk;
-    const float *row = a.scores + (int64_t)r * a.ld;
+    const float *row = FUSED ? nullptr : a.scores + (int64_t)r * a.ld;
     int n_bound = a.row_len;
     {
         if (!a.by_blocks) {
             n_bound = a.n_valid ? a.n_valid[r] : a.row_len - a.rows + r + 1;
             n_bound = n_bound < 0 ? 0 : (n_bound > a.row_len ? a.row_len : n_bound);
         }
-        const int pre4 = max(0, min(c0 + a.chunk, n_bound) - c0) >> 2;   // c0 and ld are multiples of 4
-        const float4 *src4 = reinterpret_cast<const float4 *>(row + c0);
-        for (int i = tid; i < pre4; i += NT) cp_async16(keys + 4 * i, src4 + i);
+        if (!FUSED) {
+            const int pre4 = max(0, min(c0 + a.chunk, n_bound) - c0) >> 2;   // c0 and ld are multiples of 4
+            const float4 *src4 = reinterpret_cast<const float4 *>(row + c0);
+            for (int i = tid; i < pre4; i += NT) cp_async16(keys + 4 * i, src4 + i);
+        }
     }
 
     int n;
@@ -238,7 +347,11 @@ __global__ void __launch_bounds__(topk_threads<G>()) topk_kernel(TopkArgs a) {
     for (int i = tid; i < BINS_A / 4; i += NT) reinterpret_cast<uint4 *>(hist0)[i] = make_uint4(0u, 0u, 0u, 0u);
     cp_async_wait_all();
     __syncthreads();
-    {
+    if (FUSED) {
+        uint8_t *ring = reinterpret_cast<uint8_t *>(keys + a.ring_off);
+        if (a.f_DI == 64) fused_scores<NT, 64, SA_>(a, r, c0, len, keys, hist0, ring, tid);
+        else fused_scores<NT, 128, SA_>(a, r, c0, len, keys, hist0, ring, tid);
+    } else {
         const int len4 = len >> 2;
         for (int i = tid; i < len4; i += NT) {
             const uint4 f = reinterpret_cast<const uint4 *>(keys)[i];
@@ -404,6 +517,15 @@ __global__ void __launch_bounds__(topk_threads<G>()) topk_kernel(TopkArgs a) {
     }
     if (G > 1) cluster_sync();   // peers may still read this CTA's counters
 }
+
+// The select alone, and the select with the indexer fused in (which keeps
+// its operand fragments and key tiles in registers and shared memory, so it
+// asks for one resident CTA's worth of registers rather than the select's
+// occupancy).
+template <int G>
+__global__ void __launch_bounds__(topk_threads<G>()) topk_kernel(TopkArgs a) { topk_body<G, false>(a); }
+template <int G>
+__global__ void __launch_bounds__(topk_threads<G>(), 1) topk_fused_kernel(TopkArgs a) { topk_body<G, true>(a); }
 
 // Short rows (the coarse block selection, small prefills): a group of W warps
 // per row (W = 1 for the rows of at most 1024 columns it is used for), the row's keys
@@ -602,10 +724,12 @@ static sa_status launch_topk_rows(const TopkArgs &a, cudaStream_t st) {
     return cuda_ok(cudaGetLastError());
 }
 
-template <int G>
+template <int G, bool FUSED>
 static sa_status launch_topk_g(const TopkArgs &a, size_t smem, cudaStream_t st) {
-    auto kern = topk_kernel<G>;
-    if (prepare_kernel<topk_kernel<G>>(smem, G > 8) != cudaSuccess) return SA_ERR_CUDA;
+    auto kern = FUSED ? topk_fused_kernel<G> : topk_kernel<G>;
+    if ((FUSED ? prepare_kernel<topk_fused_kernel<G>>(smem, G > 8) : prepare_kernel<topk_kernel<G>>(smem, G > 8)) !=
+        cudaSuccess)
+        return SA_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.rows * G));
     cfg.blockDim = dim3(topk_threads<G>());
@@ -625,9 +749,10 @@ sa_status launch_topk(TopkArgs a, cudaStream_t st) {
     // Rows of at most 1024 columns: the register search (32 rounds over at most
     // 32 keys per lane).  Longer rows: the histogram select, whose passes cost
     // a few operations per key rather than 32.
-    if (a.row_len <= 256) return launch_topk_rows<8, 1>(a, st);
-    if (a.row_len <= 512) return launch_topk_rows<16, 1>(a, st);
-    if (a.row_len <= 1024) return launch_topk_rows<32, 1>(a, st);
+    // (The fused indexer lives in the histogram kernel only.)
+    if (!a.fused && a.row_len <= 256) return launch_topk_rows<8, 1>(a, st);
+    if (!a.fused && a.row_len <= 512) return launch_topk_rows<16, 1>(a, st);
+    if (!a.fused && a.row_len <= 1024) return launch_topk_rows<32, 1>(a, st);
     int g = 1;
     while (g < kTopkMaxCluster && (a.row_len + g - 1) / g > kTopkChunkTarget) g *= 2;
     int chunk = (a.row_len + g - 1) / g;
@@ -639,13 +764,25 @@ sa_status launch_topk(TopkArgs a, cudaStream_t st) {
     const size_t nt = g > 1 ? topk_threads<2>() : topk_threads<1>();
     const size_t flag_words = (nt / 32) * (((size_t)chunk + 4 * nt - 1) / (4 * nt)) * 32;
     const size_t hist_words = std::max((g > 1) ? 2 * (size_t)kBinsMax : (size_t)kBinsMax / 2, flag_words);
-    const size_t smem = ((size_t)chunk + hist_words) * 4;
+    size_t smem = ((size_t)chunk + hist_words) * 4;
+    if (a.fused) {   // then the key-tile ring, 128-byte aligned
+        a.ring_off = (int)((((size_t)chunk + hist_words) + 31) & ~(size_t)31);
+        smem = (size_t)a.ring_off * 4 + (size_t)kFusedStages * kFusedSlotBytes;
+        if (smem > 227 * 1024) return SA_ERR_UNSUPPORTED;
+        switch (g) {
+            case 1: return launch_topk_g<1, true>(a, smem, st);
+            case 2: return launch_topk_g<2, true>(a, smem, st);
+            case 4: return launch_topk_g<4, true>(a, smem, st);
+            case 8: return launch_topk_g<8, true>(a, smem, st);
+            default: return launch_topk_g<16, true>(a, smem, st);
+        }
+    }
     switch (g) {
-        case 1: return launch_topk_g<1>(a, smem, st);
-        case 2: return launch_topk_g<2>(a, smem, st);
-        case 4: return launch_topk_g<4>(a, smem, st);
-        case 8: return launch_topk_g<8>(a, smem, st);
-        default: return launch_topk_g<16>(a, smem, st);
+        case 1: return launch_topk_g<1, false>(a, smem, st);
+        case 2: return launch_topk_g<2, false>(a, smem, st);
+        case 4: return launch_topk_g<4, false>(a, smem, st);
+        case 8: return launch_topk_g<8, false>(a, smem, st);
+        default: return launch_topk_g<16, false>(a, smem, st);
     }
 }
 

@@ -21,7 +21,7 @@ import math
 import torch
 
 from . import (sa_block_scores_workspace_bytes, sa_coarse_block_counts, sa_decode_workspace_bytes,
-               sa_indexer_scores, sa_indexer_scores_blocks, sa_indexer_scores_fp8,
+               sa_indexer_scores, sa_indexer_scores_blocks, sa_indexer_scores_fp8, sa_indexer_topk_decode,
                sa_pool_index_keys,
                sa_prefill_workspace_bytes, sa_sparse_attn_decode, sa_sparse_attn_prefill, sa_topk_select,
                sa_topk_select_blocks)
@@ -148,16 +148,27 @@ class DecodePlan:
     index_fp8: the qI and kI cache hold e4m3 bytes (uint8); FP8 indexer."""
 
     def __init__(self, B, Hq, d, H_I, D_I, K, W, S_max, paged=False, max_pages=0, pool_pages=0,
-                 index_fp8=False, device="cuda"):
+                 index_fp8=False, fused=None, device="cuda"):
         self.B, self.Hq, self.d, self.H_I, self.D_I, self.K, self.W = B, Hq, d, H_I, D_I, K, W
         self.index = sa_indexer_scores_fp8 if index_fp8 else sa_indexer_scores
         self.paged, self.max_pages, self.pool_pages = paged, max_pages, pool_pages
         self.S = max_pages * 64 if paged else S_max
         self.S_max = S_max
+        # fused=True: indexer and top-K in one kernel (the scores never leave
+        # shared memory).  It takes bf16 operands, H_I <= 8, D_I in (64, 128)
+        # and rows of at most 262144 keys.  It is not the default: on the
+        # decode workloads the two kernels apart are faster (the fused kernel
+        # holds one CTA per SM for the whole select, so its key reads run at
+        # about half the separate indexer's rate).
+        fusable = not index_fp8 and H_I <= 8 and D_I in (64, 128) and self.S <= 262144
+        self.fused = False if fused is None else bool(fused)
+        if self.fused and not fusable:
+            raise ValueError("the fused indexer + top-K takes bf16 operands, H_I <= 8, D_I in (64, 128) and "
+                             "rows of at most 262144 keys")
         self.scale = 1.0 / math.sqrt(d)
         dev = torch.device(device)
         self.ld = _ld(self.S)
-        self.scores = torch.empty((B, self.ld), dtype=torch.float32, device=dev)
+        self.scores = None if self.fused else torch.empty((B, self.ld), dtype=torch.float32, device=dev)
         self.topk = torch.empty((B, K), dtype=torch.int32, device=dev)
         self.out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
@@ -167,12 +178,18 @@ class DecodePlan:
 
     def stages(self, x, stream=None):
         ds, pt = self.dev_status, x.get("page_table")
-        return [
-            ("indexer", lambda: self.index(x["qI"], x["w"], x["kI"], pt, self.max_pages, self.pool_pages,
-                                           64, self.B, 1, self.S, self.H_I, self.D_I, x["lengths"],
-                                           self.scores, self.ld, ds, stream)),
-            ("topk", lambda: sa_topk_select(self.scores, self.ld, self.B, self.S, x["lengths"], None, 0, self.K,
-                                            self.topk, ds, stream)),
+        if self.fused:
+            select = [("indexer_topk", lambda: sa_indexer_topk_decode(
+                x["qI"], x["w"], x["kI"], pt, self.max_pages, self.pool_pages, 64, self.B, self.S, self.H_I,
+                self.D_I, x["lengths"], self.K, self.topk, ds, stream))]
+        else:
+            select = [
+                ("indexer", lambda: self.index(x["qI"], x["w"], x["kI"], pt, self.max_pages, self.pool_pages,
+                                               64, self.B, 1, self.S, self.H_I, self.D_I, x["lengths"],
+                                               self.scores, self.ld, ds, stream)),
+                ("topk", lambda: sa_topk_select(self.scores, self.ld, self.B, self.S, x["lengths"], None, 0,
+                                                self.K, self.topk, ds, stream))]
+        return select + [
             ("attention", lambda: sa_sparse_attn_decode(
                 x["q"], x["k"], x["v"], pt, self.max_pages, self.pool_pages, 64, self.S_max, x["lengths"],
                 self.topk, self.K, self.W, self.B, self.Hq, self.d, self.scale, self.out, self.lse,
@@ -186,14 +203,15 @@ class DecodePlan:
         return self.out
 
     def launches(self) -> int:
-        """Kernels one run() enqueues: indexer, top-K, then the attention of
+        """Kernels one run() enqueues: the fused indexer + top-K (or, unfused,
+        the indexer and the top-K), then the attention of
         sa_sparse_attn_decode.  That is one kernel when a thread-block cluster
         of G = min(16, max(1, ceil((K+W)/128), ceil(Hq/8))) CTAs per sequence
         leaves each CTA at most 1024 keys (partials merged in distributed
         shared memory), else a split-K kernel and a merge kernel."""
         kw = self.K + self.W
         G = min(16, max(1, -(-kw // 128), -(-self.Hq // 8)))
-        return 2 + (1 if -(-kw // G) <= 1024 else 2)
+        return (1 if self.fused else 2) + (1 if -(-kw // G) <= 1024 else 2)
 
 
 class HostPipeline:

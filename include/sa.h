@@ -237,6 +237,45 @@ sa_status sa_topk_select_blocks(const float *scores, int64_t ld_scores, int T,
                                 int *dev_status, sa_stream stream);
 
 /* ------------------------------------------------------------------------
+ * Stages 1 + 2 fused, decode -- indexer scores and top-K select in one
+ * kernel ("A Guide to Sparse Attention in Large Models", section 4.3: the
+ * fused operator; "Where Sparse Attention Is Actually Sparse": the indexer
+ * feeds Top-K).  The scores are never written to memory.
+ *
+ *   For each sequence b (one query each):
+ *     I_b[s] = sum_{j < H_I} w[b,j] * max(0, sum_{c < D_I} qI[b,j,c] * kI_b[s,c])
+ *   for 0 <= s < seq_lens[b], then topk[b*K + i], i < K: the min(K,
+ *   seq_lens[b]) positions of the largest I_b[s], equal scores ranked by
+ *   lower position, in ascending order, then -1.
+ *   The same result as sa_indexer_scores (T = 1, n_valid = seq_lens)
+ *   followed by sa_topk_select whenever the fp32 sums are exact (e.g. the
+ *   integer-valued inputs of the tests); otherwise the two may order their
+ *   sums differently.
+ *
+ *   qI        [B, H_I, D_I] bf16, 16-byte aligned; w [B, H_I] bf16
+ *   kI        contiguous (page_table == NULL): [B, S, D_I] bf16, 16-byte
+ *             aligned; paged: a pool [pool_pages, 64, D_I] through
+ *             page_table [B, max_pages] (page_size must be 64)
+ *   seq_lens  [B] keys per sequence, 0 .. S
+ *   Limits: H_I <= 8, D_I in {64, 128}, S <= 524288 (and shared memory for
+ *   the longest rows with D_I = 128: SA_ERR_UNSUPPORTED when it does not fit).
+ *   Each sequence's row is split over a thread-block cluster; every CTA
+ *   computes the scores of its chunk of keys on the tensor cores (mma.sync
+ *   bf16 -> fp32) into shared memory and selects there.  No workspace.
+ *   Errors: SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED, SA_ERR_CUDA; device:
+ *   SA_DEV_INDEX for a seq_lens entry outside [0, S] or a page id outside
+ *   [0, pool_pages) among the pages of the keys that are scored (a sequence
+ *   of at most K keys keeps all of them without reading its pages).
+ * ---------------------------------------------------------------------- */
+sa_status sa_indexer_topk_decode(const sa_bf16 *qI, const sa_bf16 *w,
+                                 const sa_bf16 *kI, const int32_t *page_table,
+                                 int max_pages, int pool_pages, int page_size,
+                                 int B, int S, int H_I, int D_I,
+                                 const int32_t *seq_lens, int K,
+                                 int32_t *topk, int *dev_status,
+                                 sa_stream stream);
+
+/* ------------------------------------------------------------------------
  * Stage 3a -- sparse attention, prefill
  *
  *   Query t (t < T) sits at position p = S - T + t.  Its key set is

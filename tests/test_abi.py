@@ -69,6 +69,22 @@ def test_topk_blocks_argument_checks(sa):
     assert f(P, 64, 10, 10, N0, 0, 64, 0, P, N0, N0) == sa.SA_OK                       # K = 0
 
 
+def test_fused_indexer_topk_decode_argument_checks(sa):
+    f = sa._lib.sa_indexer_topk_decode
+    # qI, w, kI, page_table, max_pages, pool_pages, page_size, B, S, H_I, D_I, seq_lens, K, topk, dev_status, stream
+    assert f(P, P, P, N0, 0, 0, 64, -1, 1024, 8, 64, P, 64, P, N0, N0) == sa.SA_ERR_INVALID_ARG     # B < 0
+    assert f(P, P, P, N0, 0, 0, 64, 2, 1024, 9, 64, P, 64, P, N0, N0) == sa.SA_ERR_UNSUPPORTED      # H_I > 8
+    assert f(P, P, P, N0, 0, 0, 64, 2, 1024, 8, 32, P, 64, P, N0, N0) == sa.SA_ERR_UNSUPPORTED      # D_I = 32
+    assert f(P, P, P, N0, 0, 0, 64, 2, 600000, 8, 64, P, 64, P, N0, N0) == sa.SA_ERR_UNSUPPORTED    # S too long
+    assert f(P, P, P, P, 16, 10, 32, 2, 1024, 8, 64, P, 64, P, N0, N0) == sa.SA_ERR_UNSUPPORTED     # page_size 32
+    assert f(P, P, P, P, 8, 10, 64, 2, 1024, 8, 64, P, 64, P, N0, N0) == sa.SA_ERR_INVALID_ARG      # 8 pages < S
+    assert f(P, P, P, P, 16, 0, 64, 2, 1024, 8, 64, P, 64, P, N0, N0) == sa.SA_ERR_INVALID_ARG      # empty pool
+    assert f(P, P, N0, N0, 0, 0, 64, 2, 1024, 8, 64, P, 64, P, N0, N0) == sa.SA_ERR_INVALID_ARG     # no keys
+    assert f(P, P, ctypes.c_void_p(24), N0, 0, 0, 64, 2, 1024, 8, 64, P, 64, P, N0, N0) == sa.SA_ERR_INVALID_ARG
+    assert f(P, P, P, N0, 0, 0, 64, 0, 1024, 8, 64, P, 64, P, N0, N0) == sa.SA_OK                    # nothing to do
+    assert f(P, P, P, N0, 0, 0, 64, 2, 1024, 8, 64, P, 0, P, N0, N0) == sa.SA_OK                     # K = 0
+
+
 def test_topk_argument_checks(sa):
     f = sa._lib.sa_topk_select
     assert f(P, 8, -1, 8, N0, N0, 0, 4, P, N0, N0) == sa.SA_ERR_INVALID_ARG      # rows < 0

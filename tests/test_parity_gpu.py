@@ -544,7 +544,7 @@ def test_e2e_two_stage_64k(sa):
     assert np.array_equal(plan.topk.cpu().numpy(), want_top)
 
 
-def _decode_e2e(sa, inp, K, W, index_fp8=False):
+def _decode_e2e(sa, inp, K, W, index_fp8=False, fused=None):
     _, DecodePlan = _pl()
     B, Hq, d = inp["q"].shape
     H_I, D_I = inp["qI"].shape[1:]
@@ -557,10 +557,10 @@ def _decode_e2e(sa, inp, K, W, index_fp8=False):
         pt = dev(inp["page_table"])
         plan = DecodePlan(B, Hq, d, H_I, D_I, K, W, S_max=0, paged=True,
                           max_pages=inp["page_table"].shape[1], pool_pages=inp["k"].shape[0],
-                          index_fp8=index_fp8)
+                          index_fp8=index_fp8, fused=fused)
     else:
         pt = None
-        plan = DecodePlan(B, Hq, d, H_I, D_I, K, W, S_max=inp["k"].shape[1], index_fp8=index_fp8)
+        plan = DecodePlan(B, Hq, d, H_I, D_I, K, W, S_max=inp["k"].shape[1], index_fp8=index_fp8, fused=fused)
     plan.run(t["q"], t["k"], t["v"], t["qI"], t["w"], t["kI"], sl, pt)
     assert status(plan.dev_status) == 0
     ref = oracle.decode(inp, K, W)
@@ -569,16 +569,47 @@ def _decode_e2e(sa, inp, K, W, index_fp8=False):
     assert np.max(np.abs(host_f64(plan.lse) - ref["lse"])) < 1e-3
 
 
-@pytest.mark.parametrize("index_fp8", [False, True])
-def test_e2e_decode_8x128k(sa, index_fp8):
+# (bf16 indexer fused with the top-K, the same two kernels apart, the FP8 indexer)
+DECODE_SELECTIONS = [(False, True), (False, False), (True, False)]
+
+
+@pytest.mark.parametrize("index_fp8,fused", DECODE_SELECTIONS)
+def test_e2e_decode_8x128k(sa, index_fp8, fused):
     c = CONFIGS["decode_8x128k"]
-    _decode_e2e(sa, config_inputs("decode_8x128k"), c["K"], c["W"], index_fp8=index_fp8)
+    _decode_e2e(sa, config_inputs("decode_8x128k"), c["K"], c["W"], index_fp8=index_fp8, fused=fused)
 
 
-@pytest.mark.parametrize("index_fp8", [False, True])
-def test_e2e_decode_paged_16(sa, index_fp8):
+@pytest.mark.parametrize("index_fp8,fused", DECODE_SELECTIONS)
+def test_e2e_decode_paged_16(sa, index_fp8, fused):
     c = CONFIGS["decode_paged_16x256k"]
-    _decode_e2e(sa, config_inputs("decode_paged_16x256k"), c["K"], c["W"], index_fp8=index_fp8)
+    _decode_e2e(sa, config_inputs("decode_paged_16x256k"), c["K"], c["W"], index_fp8=index_fp8, fused=fused)
+
+
+@pytest.mark.parametrize("paged", [False, True])
+@pytest.mark.parametrize("H_I,D_I", [(8, 64), (4, 128), (3, 64), (1, 128)])
+def test_fused_indexer_topk_decode_matches_oracle(sa, paged, H_I, D_I):
+    # lengths around the 256-key tiles, the 8192-key chunks of a cluster CTA
+    # and K; one sequence of a single key; heads below 8 leave MMA columns empty
+    lengths = [131072, 5000, 1, 2048, 2049, 8193, 255, 70001]
+    B, K = len(lengths), 2048
+    inp = gen_decode(B=B, lengths=lengths, Hq=8, d=64, H_I=H_I, D_I=D_I, paged=paged, seed=6)
+    t = _to_dev(inp, ("qI", "w", "kI"))
+    sl = dev(inp["lengths"])
+    if paged:
+        S = inp["page_table"].shape[1] * 64
+        pt, mp, pp = dev(inp["page_table"]), inp["page_table"].shape[1], inp["kI"].shape[0]
+    else:
+        S, pt, mp, pp = inp["kI"].shape[1], None, 0, 0
+    topk = torch.full((B, K), -7, dtype=torch.int32, device="cuda")
+    ds = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sa.sa_indexer_topk_decode(t["qI"], t["w"], t["kI"], pt, mp, pp, 64, B, S, H_I, D_I, sl, K, topk, ds)
+    got = topk.cpu().numpy()
+    assert status(ds) == 0
+    for b, L in enumerate(lengths):
+        _, _, kI = oracle.decode_sequence(inp, b)
+        sc = oracle.indexer(inp["qI"][b:b + 1], inp["w"][b:b + 1], kI, [L - 1])
+        want = oracle.topk(sc, [L], K)
+        assert np.array_equal(got[b], want[0]), (paged, b)
 
 
 @pytest.mark.parametrize("lengths,K,W", [([1, 2, 63, 64, 65, 3000], 100, 16), ([5000, 700], 4096, 0),

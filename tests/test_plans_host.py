@@ -64,10 +64,19 @@ def test_decode_plans(pl):
     sa, pipeline = pl
     d = pipeline.DecodePlan(8, 64, 128, 8, 64, 2048, 512, S_max=131072, device="cpu")
     assert d.ws_bytes == sa.sa_decode_workspace_bytes(8, 64, 128, 2048, 512) > 0
-    assert d.launches() == 3 and d.index is sa.sa_indexer_scores   # cluster decode: no merge kernel
+    # indexer and top-K apart by default; cluster decode: no merge kernel
+    assert not d.fused and d.launches() == 3 and d.index is sa.sa_indexer_scores
+    fd = pipeline.DecodePlan(8, 64, 128, 8, 64, 2048, 512, S_max=131072, fused=True, device="cpu")
+    assert fd.fused and fd.launches() == 2 and fd.scores is None
+    names = [n for n, _ in fd.stages({k: None for k in ("q", "k", "v", "qI", "w", "kI", "lengths")})]
+    assert names == ["indexer_topk", "attention"]
     # K + W beyond 16 CTAs x 1024 keys takes split-K + merge
     big = pipeline.DecodePlan(2, 64, 128, 8, 64, 20000, 512, S_max=65536, device="cpu")
     assert big.launches() == 4
+    # shapes the fused kernel does not take
+    for H_I, D_I, S in ((16, 64, 4096), (8, 32, 4096), (8, 64, 524288)):
+        with pytest.raises(ValueError):
+            pipeline.DecodePlan(2, 64, 128, H_I, D_I, 2048, 512, S_max=S, fused=True, device="cpu")
     assert d.ld >= 131072 and d.ld % 4 == 0
     f = pipeline.DecodePlan(16, 64, 128, 8, 64, 2048, 512, S_max=0, paged=True, max_pages=4096,
                             pool_pages=40000, index_fp8=True, device="cpu")
