@@ -674,6 +674,34 @@ def test_planted_bad_page_is_reported(sa):
     assert torch.isfinite(plan.out.float()).all()
 
 
+def test_fused_select_reports_bad_page_and_length(sa):
+    # a page id outside the pool among the pages of a scored sequence, and a
+    # sequence length beyond S, are reported; the other rows' selections stand
+    inp = gen_decode(B=3, lengths=[3000, 2500, 4000], Hq=8, d=64, H_I=8, D_I=64, paged=True, seed=12)
+    table = inp["page_table"].copy()
+    table[1, 5] = 10 ** 6
+    S = table.shape[1] * 64
+    lengths = inp["lengths"].copy()
+    t = _to_dev(inp, ("qI", "w", "kI"))
+    K = 1024
+    topk = torch.empty((3, K), dtype=torch.int32, device="cuda")
+    ds = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sa.sa_indexer_topk_decode(t["qI"], t["w"], t["kI"], dev(table), table.shape[1], inp["kI"].shape[0], 64, 3, S,
+                              8, 64, dev(lengths), K, topk, ds)
+    assert status(ds) & sa.SA_DEV_INDEX
+    got = topk.cpu().numpy()
+    for b in (0, 2):
+        _, _, kI = oracle.decode_sequence(inp, b)
+        want = oracle.topk(oracle.indexer(inp["qI"][b:b + 1], inp["w"][b:b + 1], kI, [lengths[b] - 1]),
+                           [lengths[b]], K)
+        assert np.array_equal(got[b], want[0]), b
+    lengths[2] = S + 1   # longer than the row
+    ds.zero_()
+    sa.sa_indexer_topk_decode(t["qI"], t["w"], t["kI"], dev(inp["page_table"]), table.shape[1], inp["kI"].shape[0],
+                              64, 3, S, 8, 64, dev(lengths), K, topk, ds)
+    assert status(ds) & sa.SA_DEV_INDEX
+
+
 def test_bounded_wait_reports_timeout_and_context_survives(sa):
     # a wait on a barrier that nothing arrives at gives up after 20 ms and
     # reports SA_DEV_TIMEOUT; the context keeps working afterwards
