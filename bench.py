@@ -295,14 +295,14 @@ def stage_work(case):
             fpairs = int((np.minimum(keep, t // blk) * blk + t % blk + 1).sum())
             work.update(coarse_pairs=cpairs, fine_pairs=fpairs)
             st["pool"] = dict(bytes=N * D * 2 + nb * D * 2, flops=float(N * D), bound="hbm")
-            st["block_counts"] = dict(bytes=4 * N, flops=0.0, bound="hbm")
-            st["coarse_indexer"] = dict(bytes=qI_b + w_b + nb * D * 2 + 4 * N + 4 * cpairs,
+            st["block_counts"] = dict(bytes=4 * rows, flops=0.0, bound="hbm")
+            st["coarse_indexer"] = dict(bytes=qI_b + w_b + nb * D * 2 + 4 * rows + 4 * cpairs,
                                         flops=2.0 * cpairs * H * D, bound="hbm")
-            st["coarse_topk"] = dict(bytes=4 * cpairs + 4 * N + 4 * N * keep, flops=0.0, bound="hbm")
+            st["coarse_topk"] = dict(bytes=4 * cpairs + 4 * rows + 4 * rows * keep, flops=0.0, bound="hbm")
             # the (query, slot) lists of the kept blocks, then one fp32 score per candidate
             st["fine_indexer"] = dict(bytes=qI_b + w_b + N * D * 2 + 4 * rows * (keep + 1) + 4 * fpairs,
                                       flops=2.0 * fpairs * H * D, bound="hbm")
-            st["fine_topk"] = dict(bytes=4 * fpairs + 4 * N * keep + idx_b, flops=0.0, bound="hbm")
+            st["fine_topk"] = dict(bytes=4 * fpairs + 4 * rows * keep + idx_b, flops=0.0, bound="hbm")
     work["stages"] = st
     return work
 
