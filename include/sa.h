@@ -34,9 +34,10 @@
  *   - bf16 values are passed as raw 16-bit patterns (sa_bf16), e4m3 values
  *     as raw bytes (sa_e4m3).
  *   - Supported shapes: d (attention head dim) in {64, 128}; D_I (indexer
- *     dim) in {32, 64} with bf16 operands, {64, 128} with e4m3 operands;
- *     H_I in {1, 2, 4, 8}; 1 <= Hq <= 64 query heads; page_size 64.  Other
- *     shapes return SA_ERR_UNSUPPORTED.  There is no fallback path.
+ *     dim) in {32, 64} with bf16 operands, {64, 128} with e4m3 operands and
+ *     for the fused decode select; H_I in {1, 2, 4, 8} (1 .. 8 for the fused
+ *     decode select); 1 <= Hq <= 64 query heads; page_size 64.  Other shapes
+ *     return SA_ERR_UNSUPPORTED.  There is no fallback path.
  */
 #ifndef FINE_GRAINED_TOP_SA_H
 #define FINE_GRAINED_TOP_SA_H
