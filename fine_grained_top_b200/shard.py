@@ -14,7 +14,8 @@ any earlier key.  The two partitions here are the ones the path allows:
   are never needed).  That all-gather is the only exchange; remote rows are
   copied into this GPU's memory before any kernel reads them.
 * Decode, sequences.  Whole sequences are dealt to ranks, longest first to the
-  least loaded rank.  There is no exchange at all.
+  least loaded rank.  The step has no exchange; the outputs are collected in
+  batch order by one all-gather when a caller needs them on every rank.
 
 Nothing here computes any part of the method: it picks bounds, moves rows
 and hands each rank's share to a plan (``pipeline.PrefillPlan`` /
@@ -77,24 +78,31 @@ def decode_assignment(lengths, world: int) -> list:
     return [sorted(o) for o in owned]
 
 
-def all_gather_rows(shard, N: int, world: int, group=None):
-    """The full [N, ...] tensor from every rank's equal shard (rows
-    key_shard_bounds(N, world)[r] .. [r+1] on rank r): one all_gather of
-    shards padded to the same row count."""
+def gather_chunks(local, bounds, group=None):
+    """The [bounds[-1], ...] tensor whose rows bounds[r] .. bounds[r+1]-1 are
+    rank r's `local` rows (chunks may differ in length, and may be empty):
+    one all_gather of chunks padded to the longest.  Rows travel as raw bytes,
+    so any element type works on any backend."""
     import torch
     import torch.distributed as dist
-    b = key_shard_bounds(N, world)
-    per = max(b[r + 1] - b[r] for r in range(world)) if world else 0
-    row_shape = tuple(shard.shape[1:])
-    # rows travel as raw bytes, so any element type works on any backend
-    row_elems = int(np.prod(row_shape)) if row_shape else 1
-    raw = shard.contiguous().reshape(shard.shape[0], row_elems).view(torch.uint8)
-    pad = torch.zeros((per, raw.shape[1]), dtype=torch.uint8, device=shard.device)
+    world = len(bounds) - 1
+    N = bounds[-1]
+    per = max(bounds[r + 1] - bounds[r] for r in range(world)) if world else 0
+    row_shape = tuple(local.shape[1:])
+    row_bytes = (int(np.prod(row_shape)) if row_shape else 1) * local.element_size()
+    raw = local.contiguous().view(torch.uint8).reshape(local.shape[0], row_bytes)
+    pad = torch.zeros((max(per, 1), row_bytes), dtype=torch.uint8, device=local.device)
     pad[:raw.shape[0]] = raw
     parts = [torch.empty_like(pad) for _ in range(world)]
     dist.all_gather(parts, pad, group=group)
-    rows = torch.cat([parts[r][:b[r + 1] - b[r]] for r in range(world)], dim=0)
-    return rows.view(shard.dtype).reshape((N,) + row_shape)
+    rows = torch.cat([parts[r][:bounds[r + 1] - bounds[r]] for r in range(world)], dim=0)
+    return rows.contiguous().view(local.dtype).reshape((N,) + row_shape)
+
+
+def all_gather_rows(shard, N: int, world: int, group=None):
+    """The full [N, ...] tensor from every rank's equal shard (rows
+    key_shard_bounds(N, world)[r] .. [r+1] on rank r)."""
+    return gather_chunks(shard, key_shard_bounds(N, world), group)
 
 
 class ShardedPrefill:
@@ -133,3 +141,43 @@ class ShardedPrefill:
         if self.plan is None:
             return None
         return self.plan.run(q_rows, k, v, qI_rows, w_rows, kI)
+
+    def collect(self, rows):
+        """Every rank's result rows (this rank's: `rows`, [t1 - t0, ...], any
+        dtype) -> the full [N, ...] tensor on every rank, in query order."""
+        return gather_chunks(rows, self.bounds, self.group)
+
+
+class ShardedDecode:
+    """One rank's share of a decode step over a batch split.
+
+    Whole sequences are dealt by decode_assignment (longest first to the rank
+    with the fewest cached tokens); each rank holds the caches of its own
+    sequences and runs its plan on them alone, so the step itself has no
+    exchange.  select() picks this rank's rows out of a batch-ordered array,
+    collect() puts every rank's result rows back in batch order on every
+    rank (one all_gather)."""
+
+    def __init__(self, lengths, rank, world, group=None):
+        self.lengths = [int(x) for x in lengths]
+        self.rank, self.world, self.group = rank, world, group
+        self.owned_by = decode_assignment(self.lengths, world)
+        self.owned = self.owned_by[rank]
+        counts = [len(o) for o in self.owned_by]
+        self.bounds = [0] + list(np.cumsum(counts).astype(int))
+        # batch index of each row of the gathered tensor
+        self.order = [b for o in self.owned_by for b in o]
+
+    def select(self, x):
+        """Rows of this rank's sequences (ascending batch index) of a
+        batch-ordered array or tensor."""
+        return x[self.owned]
+
+    def collect(self, rows):
+        """This rank's result rows ([len(owned), ...]) -> the batch-ordered
+        [B, ...] tensor on every rank."""
+        import torch
+        gathered = gather_chunks(rows, self.bounds, self.group)
+        out = torch.empty_like(gathered)
+        out[torch.as_tensor(self.order, dtype=torch.long, device=gathered.device)] = gathered
+        return out

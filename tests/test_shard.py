@@ -180,3 +180,64 @@ def test_two_gloo_ranks_decode_split_equals_whole(tmp_path):
     for key in ("topk", "out", "lse"):
         got = np.concatenate([p[key] for p in parts])
         assert np.array_equal(got, whole[key][seqs])
+
+
+# ---------------------------------------------------------------- collecting results on every rank
+def _collect_rank(rank, world, port, out_dir):
+    import sys
+    sys.path.insert(0, ROOT)
+    import torch
+    import torch.distributed as dist
+    import oracle
+    from fine_grained_top_b200.shard import ShardedDecode, ShardedPrefill, gather_chunks
+    from workloads import gen_decode, gen_prefill
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), ORACLE_THREADS="2")
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # prefill: each rank's rows, then the whole sequence's results on every rank
+        N, Hq, d, H_I, D_I, K, W = 600, 4, 64, 2, 32, 64, 16
+        inp = gen_prefill(N=N, Hq=Hq, d=d, H_I=H_I, D_I=D_I, seed=9)
+        sp = ShardedPrefill(N, Hq, d, H_I, D_I, K, W, rank, world, device="cpu", make_plan=lambda T, S: None)
+        rows = np.arange(sp.t0, sp.t1)
+        mine = oracle.prefill(inp, K, W, rows=rows) if len(rows) else \
+            {"topk": np.zeros((0, K), np.int64), "out": np.zeros((0, Hq, d)), "lse": np.zeros((0, Hq))}
+        full_p = {k: sp.collect(torch.from_numpy(np.ascontiguousarray(mine[k]))).numpy()
+                  for k in ("topk", "out", "lse")}
+        # decode: whole sequences per rank, results back in batch order on every rank
+        lengths = [3000, 70, 9000, 1, 4097, 640]
+        dinp = gen_decode(B=len(lengths), lengths=lengths, Hq=8, d=64, H_I=2, D_I=32, paged=True, seed=4)
+        sd = ShardedDecode(lengths, rank, world)
+        dres = oracle.decode(dinp, 64, 16, seqs=sd.owned)
+        full_d = {k: sd.collect(torch.from_numpy(np.ascontiguousarray(dres[k]))).numpy() for k in ("topk", "out", "lse")}
+        picked = sd.select(np.asarray(lengths))
+        # an empty chunk on one rank, and a dtype other than the defaults
+        local = (torch.arange(3 * rank, dtype=torch.int16).reshape(rank, 3) if rank
+                 else torch.zeros((0, 3), dtype=torch.int16))
+        ragged = gather_chunks(local, [0, 0] + [world - 1], None).numpy() if world == 2 else None
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+    np.savez(os.path.join(out_dir, "c%d.npz" % rank), owned=np.array(sd.owned, np.int64), picked=picked,
+             ragged=ragged, **{"p_" + k: v for k, v in full_p.items()}, **{"d_" + k: v for k, v in full_d.items()})
+
+
+def test_two_gloo_ranks_collect_full_results():
+    import tempfile
+    import torch.multiprocessing as mp
+    import oracle
+    from workloads import gen_decode, gen_prefill
+    world = 2
+    with tempfile.TemporaryDirectory() as tmp:
+        mp.start_processes(_collect_rank, args=(world, _free_port(), tmp), nprocs=world, start_method="spawn",
+                           join=True)
+        parts = [dict(np.load(os.path.join(tmp, "c%d.npz" % r), allow_pickle=True)) for r in range(world)]
+    whole = oracle.prefill(gen_prefill(N=600, Hq=4, d=64, H_I=2, D_I=32, seed=9), 64, 16)
+    lengths = [3000, 70, 9000, 1, 4097, 640]
+    dwhole = oracle.decode(gen_decode(B=6, lengths=lengths, Hq=8, d=64, H_I=2, D_I=32, paged=True, seed=4), 64, 16)
+    for p in parts:   # every rank holds the whole result, in query / batch order
+        for k in ("topk", "out", "lse"):
+            assert np.array_equal(p["p_" + k], whole[k]), k
+            assert np.array_equal(p["d_" + k], dwhole[k]), k
+        assert np.array_equal(p["picked"], np.asarray(lengths)[p["owned"]])
+        assert np.array_equal(p["ragged"], np.arange(3, dtype=np.int16).reshape(1, 3))   # rank 0 sent no rows
+    assert sorted(np.concatenate([p["owned"] for p in parts]).tolist()) == list(range(6))
