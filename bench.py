@@ -1,7 +1,7 @@
 """Benchmark: fine-grained top-K sparse attention on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
-                    [--index-fp8]
+                    [--rows T] [--index-fp8] [--fused-select] [--no-cpu-baseline]
 
 A step is one pass of the whole path -- indexer -> top-K -> sparse attention
 (for the two-stage workload: pool, block counts, coarse scores, coarse top-k,
@@ -24,7 +24,13 @@ neighbouring steps run on their own streams under each step's kernels
 fp64 oracle on a bounded sample of query rows of the same workload.
 `--index-fp8` runs the indexer on e4m3 operands (quantised before timing);
 the workloads' integer-valued indexer inputs are exact in e4m3, so the
-selected positions are unchanged.
+selected positions are unchanged.  `--rows T` times the last T query rows of
+a prefill workload's sequence over all of its keys (a chunk of a prompt).
+`--fused-select` runs a decode workload's indexer inside its top-K kernel.
+The attention's line also reports its K/V gather rate against the measured
+L2 -> shared-memory ceiling, and `roofline.traffic` is the DRAM bytes of the
+dominant kernel from a one-pass ncu capture of the same sources
+(profiles/dram_traffic.json), else null.
 """
 
 from __future__ import annotations
