@@ -74,3 +74,22 @@ def test_roofline_entry_fractions():
     assert e["achieved"] == 2000.0 and e["frac"] == 2.0 and e["unit"] == "GB/s"
     t = bench.roofline_entry("tensor", 0.0, 5e10, 1e-3, peaks)
     assert t["achieved"] == 50.0 and t["frac"] == 0.5 and t["unit"] == "TFLOP/s"
+
+
+def test_traffic_lookup_follows_the_source_hash(tmp_path, monkeypatch):
+    # roofline.traffic comes from a capture of the exact sources that are built:
+    # a matching hash gives bytes x scale, any other hash or stage gives None
+    import json
+    import os
+    import bench
+    (tmp_path / "profiles").mkdir()
+    os.symlink(os.path.join(bench.ROOT, "fine_grained_top_b200"), tmp_path / "fine_grained_top_b200")
+    real = bench.source_hash(bench.STAGE_SOURCE["attention"])
+    entries = [dict(workload="w", stage="attention", sources="x", source_hash=real, bytes_per_launch=1000, scale=2.0),
+               dict(workload="w", stage="fine_topk", sources="x", source_hash="000000000000", bytes_per_launch=5)]
+    (tmp_path / "profiles" / "dram_traffic.json").write_text(json.dumps({"entries": entries}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.ncu_traffic("w", "attention") == 2000
+    assert bench.ncu_traffic("w", "fine_topk") is None         # captured from other sources
+    assert bench.ncu_traffic("other", "attention") is None     # another workload
+    assert bench.ncu_traffic("w", "no_such_stage") is None
