@@ -338,7 +338,8 @@ def oracle_sample(case, n):
         T = cfg.get("rows", cfg["N"])
         rows = np.linspace(cfg["N"] - T, cfg["N"] - 1, n).astype(np.int64)
         oracle.prefill(inp, cfg["K"], cfg["W"], rows=rows, block=cfg.get("block"), keep=cfg.get("keep"))
-        desc = "%d evenly spaced query rows of the last %d of %d, all stages" % (n, T, cfg["N"])
+        desc = ("%d evenly spaced query rows of %d, all stages" % (n, cfg["N"]) if T == cfg["N"] else
+                "%d evenly spaced query rows of the last %d of %d, all stages" % (n, T, cfg["N"]))
     return time.perf_counter() - t0, desc
 
 
