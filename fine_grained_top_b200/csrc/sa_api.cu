@@ -208,6 +208,7 @@ sa_status sa_sparse_attn_prefill(const sa_bf16 *q, const sa_bf16 *k, const sa_bf
                                  int W, int T, int S, int Hq, int d, float scale, sa_bf16 *out, float *lse,
                                  void *workspace, size_t workspace_bytes, int *dev_status, sa_stream stream) {
     if (K < 0 || W < 0 || T < 0 || S < 0 || T > S) return SA_ERR_INVALID_ARG;
+    if (T > 0 && K + W == 0) return SA_ERR_INVALID_ARG;   // every key set would be empty
     if (!head_dim_ok(d) || Hq < 1 || Hq > 64) return SA_ERR_UNSUPPORTED;
     if ((int64_t)K + W > 32768) return SA_ERR_UNSUPPORTED;   // the per-query key list lives in shared memory
     if (T == 0) return SA_OK;

@@ -289,9 +289,10 @@ sa_status sa_indexer_topk_decode(const sa_bf16 *qI, const sa_bf16 *w,
  *   sa_topk_select writes it), out [T, Hq, d] bf16, lse [T, Hq] fp32.
  *   Softmax and accumulation are fp32; probabilities are rounded to bf16 for
  *   the P.V product; out is rounded to bf16 (nearest even).
- *   Two kernels compute this.  Gathered: each query's selected K/V rows are
- *   gathered into shared memory (any shape; the only one when workspace is
- *   NULL).  Masked tensor-core tiles: when every query keeps a large share of
+ *   Two kinds of kernel compute this.  Gathered: each query's selected K/V
+ *   rows are gathered into shared memory (the only kind when workspace is
+ *   NULL): on tcgen05 tiles with keys on M for d = 128, Hq <= 32, K <= 2048,
+ *   else on mma.sync tiles.  Masked tensor-core tiles: when every query keeps a large share of
  *   its causal keys (S * Hq <= 256 * (K + W), Hq in {4, 8, 16, 32}, d in
  *   {64, 128}), groups of 128 / Hq queries stream the causal K/V once in
  *   128-key tiles through tcgen05 MMAs, masked by a per-query selection
@@ -303,6 +304,11 @@ sa_status sa_indexer_topk_decode(const sa_bf16 *qI, const sa_bf16 *w,
  *   Device errors: a top-K entry > p sets SA_DEV_INDEX and is skipped; a row
  *   that is not strictly ascending sets SA_DEV_ORDER.
  *   Limit: K + W <= 32768 (each query's key list is held in shared memory). 
+ *   Every key set must be non-empty (a softmax over no keys is undefined):
+ *   K + W = 0 returns SA_ERR_INVALID_ARG, and with W = 0 every top-K row
+ *   must hold a valid entry (rows from sa_topk_select always do, since
+ *   they keep min(K, p + 1) positions <= p); the out and lse rows of a query
+ *   whose set is empty anyway are unspecified.
  * ---------------------------------------------------------------------- */
 size_t sa_prefill_workspace_bytes(int T, int S, int K, int W, int Hq, int d);
 

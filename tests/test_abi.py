@@ -137,6 +137,8 @@ def test_attention_argument_checks(sa):
     assert sa.sa_prefill_workspace_bytes(8192, 8192, 1024, 128, 16, 128) == 8192 * 256 * 4
     assert sa.sa_prefill_workspace_bytes(65536, 65536, 2048, 512, 16, 128) == 0       # sparse: gathered path
     assert f(P, P, P, P, 4, 2, 0, 8, 16, 128, 0.1, P, N0, N0, 0, N0, N0) == sa.SA_OK
+    assert f(P, P, P, P, 0, 0, 8, 8, 16, 128, 0.1, P, N0, N0, 0, N0, N0) == sa.SA_ERR_INVALID_ARG  # empty key sets
+    assert f(P, P, P, P, 0, 0, 0, 8, 16, 128, 0.1, P, N0, N0, 0, N0, N0) == sa.SA_OK               # no queries
     g = sa._lib.sa_sparse_attn_decode
     need = sa.sa_decode_workspace_bytes(8, 64, 128, 2048, 512)
     assert need > 8 * 64 * 128 * 4
